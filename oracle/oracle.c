@@ -1,0 +1,395 @@
+/*
+ * Plain fp64 CPU oracle for attention over a paged KV cache.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference leg of bench.py may build, load or call this file.
+ * It shares no code, header, table or helper with the CUDA library; the two
+ * meet only through the seeded inputs of paged_kv_attention_34_b200.workloads.
+ *
+ * What it computes, and where the pages say so:
+ *
+ *   attention     Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V
+ *                 (ybb.press "LLM 推理优化", section 1, the attention formula).
+ *                 The scale is an argument (1/sqrt(d) by default).
+ *   paging        the cache is a pool of fixed 16-token blocks; a per-request
+ *                 page table maps logical page p to a physical block
+ *                 (iopencloud "大模型推理加速技术全景", section 3.2 and its
+ *                 page-table figure; zhihu roofline page, "显存管理").
+ *   varlen        sequences are packed back to back and delimited by a
+ *                 cu_seqlens prefix sum; each sequence attends only to itself
+ *                 (interview Q&A page, ragged batching answer).
+ *   causal        query i of a sequence with q_b new tokens and ctx_b cached
+ *                 keys (new tokens included) sits at position ctx_b - q_b + i
+ *                 and sees keys 0 .. ctx_b - q_b + i.  The pages do not spell
+ *                 out this alignment; it is the reading that makes a decode
+ *                 query see its whole context and a chunk see its prefix.
+ *   standard      the three-pass form: S = Q K^T materialised, softmax, then
+ *                 S V (iopencloud section 2.1).  Used on tiny inputs.
+ *   online        the running-max / running-sum recurrence over key blocks,
+ *                 normalised once after the last block (iopencloud section
+ *                 2.2, pseudocode; the final diag(l)^-1 is read as following
+ *                 the loop).
+ *   split merge   per-split partial results combined by their log-sum-exp
+ *                 (interview Q&A page, FlashDecoding answer: split the KV
+ *                 sequence across blocks, then a cross-block reduction).
+ *   cache write   scatter of new K/V rows to slot = block*16 + offset; a
+ *                 negative slot is a padding token and is skipped.
+ *   block copy    copy-on-write of a shared block: all heads and 16 rows of
+ *                 K and V of block src are copied to block dst (zhihu roofline
+ *                 page, "显存管理": refcounted blocks, copy-on-write).
+ *
+ * 16-bit inputs are widened exactly to double from their bit patterns
+ * (IEEE 754 binary16, and bfloat16 = the upper half of binary32).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_BLOCK 16
+
+enum { ORACLE_F16 = 0, ORACLE_BF16 = 1 };
+
+/* ---- 16-bit formats -------------------------------------------------------- */
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double oracle_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24); /* subnormal: f * 2^-14 * 2^-10 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp(1.0 + (double)f / 1024.0, e - 15);
+    return sign ? -v : v;
+}
+
+/* bfloat16: 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits. */
+double oracle_bf16_to_f64(uint16_t b)
+{
+    int sign = (b >> 15) & 1;
+    int e = (b >> 7) & 0xff;
+    int f = b & 0x7f;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -133); /* subnormal: f * 2^-126 * 2^-7 */
+    else if (e == 255)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp(1.0 + (double)f / 128.0, e - 127);
+    return sign ? -v : v;
+}
+
+static double widen(uint16_t x, int dtype)
+{
+    return dtype == ORACLE_F16 ? oracle_f16_to_f64(x) : oracle_bf16_to_f64(x);
+}
+
+/* ---- cache write and block copy (exact copies) ---------------------------- */
+
+/* key_cache/value_cache: [num_blocks][H_kv][16][d]; k_new/v_new: [T][H_kv][d].
+ * Returns the number of tokens whose slot was out of range (not written). */
+int64_t oracle_kv_cache_write(const uint16_t *k_new, const uint16_t *v_new, const int32_t *slot_mapping,
+                              int64_t T, uint16_t *key_cache, uint16_t *value_cache, int64_t num_blocks,
+                              int H_kv, int d)
+{
+    int64_t bad = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue; /* padding token */
+        if (slot >= num_blocks * ORACLE_BLOCK) {
+            ++bad;
+            continue;
+        }
+        int64_t block = slot / ORACLE_BLOCK;
+        int64_t offset = slot % ORACLE_BLOCK;
+        for (int h = 0; h < H_kv; ++h)
+            for (int k = 0; k < d; ++k) {
+                int64_t dst = ((block * H_kv + h) * ORACLE_BLOCK + offset) * d + k;
+                int64_t src = (t * H_kv + h) * (int64_t)d + k;
+                key_cache[dst] = k_new[src];
+                value_cache[dst] = v_new[src];
+            }
+    }
+    return bad;
+}
+
+/* pairs: [n][2] = (src, dst).  Returns the number of pairs skipped as out of range. */
+int64_t oracle_kv_block_copy(uint16_t *key_cache, uint16_t *value_cache, int64_t num_blocks, int H_kv, int d,
+                             const int32_t *pairs, int64_t n)
+{
+    int64_t bad = 0;
+    int64_t per_block = (int64_t)H_kv * ORACLE_BLOCK * d;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t src = pairs[2 * i], dst = pairs[2 * i + 1];
+        if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) {
+            ++bad;
+            continue;
+        }
+        for (int64_t e = 0; e < per_block; ++e) {
+            key_cache[dst * per_block + e] = key_cache[src * per_block + e];
+            value_cache[dst * per_block + e] = value_cache[src * per_block + e];
+        }
+    }
+    return bad;
+}
+
+/* ---- attention over the paged cache ---------------------------------------- */
+
+/* One output row: query token t (of sequence b, index i within its q_b new
+ * tokens), query head h.  Keys are gathered one by one through the block
+ * table.  out_row receives d doubles.  Also returns the natural-log
+ * log-sum-exp of the scaled scores when lse != NULL. */
+static int attention_row(double *out_row, double *lse, const uint16_t *q, const uint16_t *key_cache,
+                         const uint16_t *value_cache, int dtype, const int32_t *block_tables, int max_blocks,
+                         int b, int i, int q_b, int ctx_b, int64_t t, int h, int H_q, int H_kv, int d,
+                         double scale, double *s /* scratch, >= ctx_b doubles */)
+{
+    int G = H_q / H_kv;
+    int g = h / G; /* consecutive query heads share one KV head */
+    int last = ctx_b - q_b + i; /* causal: keys 0 .. last */
+    if (last < 0)
+        return -1;
+    const uint16_t *qrow = q + (t * H_q + h) * (int64_t)d;
+
+    /* scores s_j = scale * <q, K_j> */
+    for (int j = 0; j <= last; ++j) {
+        int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
+        int64_t off = j % ORACLE_BLOCK;
+        const uint16_t *krow = key_cache + ((block * H_kv + g) * ORACLE_BLOCK + off) * d;
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k)
+            acc += widen(qrow[k], dtype) * widen(krow[k], dtype);
+        s[j] = scale * acc;
+    }
+    /* softmax with the row maximum subtracted */
+    double m = -INFINITY;
+    for (int j = 0; j <= last; ++j)
+        if (s[j] > m)
+            m = s[j];
+    double z = 0.0;
+    for (int j = 0; j <= last; ++j) {
+        s[j] = exp(s[j] - m);
+        z += s[j];
+    }
+    /* O = sum_j softmax_j V_j */
+    for (int k = 0; k < d; ++k)
+        out_row[k] = 0.0;
+    for (int j = 0; j <= last; ++j) {
+        int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
+        int64_t off = j % ORACLE_BLOCK;
+        const uint16_t *vrow = value_cache + ((block * H_kv + g) * ORACLE_BLOCK + off) * d;
+        double w = s[j] / z;
+        for (int k = 0; k < d; ++k)
+            out_row[k] += w * widen(vrow[k], dtype);
+    }
+    if (lse)
+        *lse = m + log(z);
+    return 0;
+}
+
+/* out: [n_rows][d] doubles.  rows: flattened (t * H_q + h) row ids to compute,
+ * or NULL for all T*H_q rows (then out is [T][H_q][d]).  lse_out: optional
+ * [n_rows] natural-log log-sum-exp per row.
+ * Returns 0, or -1 if some sequence has ctx_b < q_b or q_b < 0,
+ * -2 if H_q is not a multiple of H_kv. */
+int oracle_paged_attention(double *out, double *lse_out, const uint16_t *q, const uint16_t *key_cache,
+                           const uint16_t *value_cache, int dtype, const int32_t *block_tables, int max_blocks,
+                           const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int H_q, int H_kv,
+                           int d, double scale, const int64_t *rows, int64_t n_rows, int n_threads)
+{
+    if (H_kv <= 0 || H_q % H_kv != 0)
+        return -2;
+    int max_ctx = 0;
+    for (int b = 0; b < B; ++b) {
+        int q_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+        if (q_b < 0 || context_lens[b] < q_b)
+            return -1;
+        if (context_lens[b] > max_ctx)
+            max_ctx = context_lens[b];
+    }
+    int64_t T = cu_seqlens_q[B];
+    int64_t total = rows ? n_rows : T * H_q;
+    int status = 0;
+#ifdef _OPENMP
+    if (n_threads > 0)
+        omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(max_ctx > 0 ? max_ctx : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < total; ++r) {
+            int64_t row = rows ? rows[r] : r;
+            int64_t t = row / H_q;
+            int h = (int)(row % H_q);
+            int b = 0; /* sequence owning token t */
+            while (b < B && cu_seqlens_q[b + 1] <= t)
+                ++b;
+            int i = (int)(t - cu_seqlens_q[b]);
+            int q_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+            int rc = attention_row(out + r * d, lse_out ? lse_out + r : NULL, q, key_cache, value_cache, dtype,
+                                   block_tables, max_blocks, b, i, q_b, context_lens[b], t, h, H_q, H_kv, d,
+                                   scale, s);
+            if (rc) {
+#pragma omp atomic write
+                status = rc;
+            }
+        }
+        free(s);
+    }
+    return status;
+}
+
+/* ---- dense forms on contiguous fp64 data (tiny inputs) ---------------------- */
+
+/* Standard three-pass attention: S = Q K^T * scale held in full, row softmax,
+ * then P V.  q: [n_q][d], k, v: [n_k][d].  Query i sees keys j <= i + offset
+ * (offset = n_k - n_q aligns the last query with the last key; a huge offset
+ * disables the mask). */
+void oracle_dense_attention(double *out, const double *q, const double *k, const double *v, int n_q, int n_k,
+                            int d, double scale, int64_t offset)
+{
+    double *S = (double *)malloc(sizeof(double) * (size_t)n_q * (size_t)n_k);
+    for (int i = 0; i < n_q; ++i)
+        for (int j = 0; j < n_k; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += q[(int64_t)i * d + c] * k[(int64_t)j * d + c];
+            S[(int64_t)i * n_k + j] = (j <= i + offset) ? scale * acc : -INFINITY;
+        }
+    for (int i = 0; i < n_q; ++i) {
+        double *row = S + (int64_t)i * n_k;
+        double m = -INFINITY, z = 0.0;
+        for (int j = 0; j < n_k; ++j)
+            if (row[j] > m)
+                m = row[j];
+        for (int j = 0; j < n_k; ++j) {
+            row[j] = (row[j] == -INFINITY) ? 0.0 : exp(row[j] - m);
+            z += row[j];
+        }
+        for (int j = 0; j < n_k; ++j)
+            row[j] /= z;
+    }
+    for (int i = 0; i < n_q; ++i)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < n_k; ++j)
+                acc += S[(int64_t)i * n_k + j] * v[(int64_t)j * d + c];
+            out[(int64_t)i * d + c] = acc;
+        }
+    free(S);
+}
+
+/* Online softmax for one query row over keys in blocks of `block` keys:
+ * running max m and running sum l, the accumulator rescaled by
+ * exp(m_prev - m_new) whenever the max moves, and one division by l after
+ * the last block.  q: [d], k, v: [n_k][d]. */
+void oracle_online_softmax(double *out, const double *q, const double *k, const double *v, int n_k, int d,
+                           double scale, int block)
+{
+    double m = -INFINITY, l = 0.0;
+    double *o = (double *)calloc((size_t)d, sizeof(double));
+    double *s = (double *)malloc(sizeof(double) * (size_t)(block > 0 ? block : 1));
+    for (int j0 = 0; j0 < n_k; j0 += block) {
+        int nb = (n_k - j0 < block) ? n_k - j0 : block;
+        double bmax = -INFINITY;
+        for (int j = 0; j < nb; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += q[c] * k[(int64_t)(j0 + j) * d + c];
+            s[j] = scale * acc;
+            if (s[j] > bmax)
+                bmax = s[j];
+        }
+        double m_new = m > bmax ? m : bmax;
+        double alpha = exp(m - m_new); /* 0 on the first block */
+        double rowsum = 0.0;
+        for (int j = 0; j < nb; ++j) {
+            s[j] = exp(s[j] - m_new);
+            rowsum += s[j];
+        }
+        l = alpha * l + rowsum;
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < nb; ++j)
+                acc += s[j] * v[(int64_t)(j0 + j) * d + c];
+            o[c] = alpha * o[c] + acc;
+        }
+        m = m_new;
+    }
+    for (int c = 0; c < d; ++c)
+        out[c] = o[c] / l;
+    free(o);
+    free(s);
+}
+
+/* Attention of one query row restricted to keys [lo, hi): the normalised
+ * partial output and its natural-log log-sum-exp (-inf and zeros when the
+ * range is empty).  This is one split of split-KV decoding. */
+void oracle_attention_partial(double *out, double *lse, const double *q, const double *k, const double *v, int lo,
+                              int hi, int d, double scale)
+{
+    double m = -INFINITY;
+    for (int c = 0; c < d; ++c)
+        out[c] = 0.0;
+    if (hi <= lo) {
+        *lse = -INFINITY;
+        return;
+    }
+    double *s = (double *)malloc(sizeof(double) * (size_t)(hi - lo));
+    for (int j = lo; j < hi; ++j) {
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c)
+            acc += q[c] * k[(int64_t)j * d + c];
+        s[j - lo] = scale * acc;
+        if (s[j - lo] > m)
+            m = s[j - lo];
+    }
+    double z = 0.0;
+    for (int j = lo; j < hi; ++j) {
+        s[j - lo] = exp(s[j - lo] - m);
+        z += s[j - lo];
+    }
+    for (int j = lo; j < hi; ++j)
+        for (int c = 0; c < d; ++c)
+            out[c] += s[j - lo] / z * v[(int64_t)j * d + c];
+    *lse = m + log(z);
+    free(s);
+}
+
+/* Cross-split reduction: O = sum_s exp(lse_s - lse) O_s with
+ * lse = log sum_s exp(lse_s).  Splits with lse_s = -inf contribute nothing.
+ * parts: [n_splits][d], lses: [n_splits]. */
+void oracle_lse_merge(double *out, double *lse_out, const double *parts, const double *lses, int n_splits, int d)
+{
+    double m = -INFINITY;
+    for (int s = 0; s < n_splits; ++s)
+        if (lses[s] > m)
+            m = lses[s];
+    for (int c = 0; c < d; ++c)
+        out[c] = 0.0;
+    if (m == -INFINITY) {
+        *lse_out = -INFINITY;
+        return;
+    }
+    double z = 0.0;
+    for (int s = 0; s < n_splits; ++s)
+        z += exp(lses[s] - m);
+    for (int s = 0; s < n_splits; ++s) {
+        double w = exp(lses[s] - m) / z;
+        for (int c = 0; c < d; ++c)
+            out[c] += w * parts[(int64_t)s * d + c];
+    }
+    *lse_out = m + log(z);
+}
