@@ -1,0 +1,555 @@
+"""Benchmark of the paged-KV attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline workload (N = 1): the LLaMA-2-13B-shaped decode layer -- 64
+sequences, one new token each, 40/40 heads, d 128, fp16, contexts uniform in
+[128, 4096], 16-token blocks shuffled over the pool.  One step = the hot path
+of a decode iteration: ``kv_cache_write`` of the 64 new K/V rows, then
+``paged_attn_decode`` (split-KV kernel + log-sum-exp merge kernel).  ``value``
+is the step's algorithmic HBM bytes (every context key's K and V, Q, O, table
+entries, the new rows written) over the device time of the step: GB/s.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch of 64
+sequences (independent seed): the sequences are independent, so there is no
+data-path collective ("weak" scaling); the only collectives are the barriers
+and the max-over-ranks of the elapsed time.
+
+The same JSON line carries:
+  roofline      decode call (split kernel + merge) vs the measured HBM copy peak
+  prefill       causal varlen prefill (8 prompts U[256,2048], 40/40 heads, bf16):
+                TFLOP/s of exact causal pairs vs the measured bf16 peak
+  legs          the GQA shared-prefix decode step and the mixed continuous-batching step
+  e2e           the same metric with host buffers: pinned H2D of the step inputs and
+                D2H of the output inside the timed region
+  cpu_baseline  the fp64 CPU oracle, timed on a bounded sample of the same workload
+  clocks        SM clock / throttle reasons sampled through NVML during the timed region
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+method has) on the host cores on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attn HBM GB/s & prefill attn TFLOPS, as % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HEADLINE = "LLaMA-2-13B-shaped decode layer: B 64, q_len 1, 40/40 heads, d 128, fp16, ctx U[128,4096], block 16"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---- distributed plumbing (also exercised on CPU with gloo by the tests) --------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def shard_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent batch of sequences."""
+    return base + 1000 * rank
+
+
+def reduce_max(x: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---- clocks -------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML in a thread (every ~2 ms)."""
+
+    REASONS = {
+        "hw_slowdown": 0x8,
+        "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80,
+        "sw_power_cap": 0x4,
+    }
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = device_index
+            if vis:
+                try:
+                    idx = int(vis.split(",")[device_index])
+                except ValueError:
+                    idx = device_index
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: clocks are reported as unavailable
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or getattr(
+                    nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                r = get(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+            time.sleep(0.005)
+        return self
+
+    def __exit__(self, *exc):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.nv or not self.samples:
+            return None
+        s = sorted(self.samples)
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(s), "source": "NVML"}
+
+
+# ---- timing helpers ----------------------------------------------------------------------------------
+
+def time_calls(fn_list, steps, stream):
+    """Run `steps` iterations of the step; per-call CUDA-event durations on `stream`.
+
+    Returns (total_ms, [avg_ms per call]) with the total bracketed by events."""
+    import torch
+
+    n = len(fn_list)
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+           for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for s in range(steps):
+            for i, fn in enumerate(fn_list):
+                evs[s][i][0].record(stream)
+                fn()
+                evs[s][i][1].record(stream)
+        end.record(stream)
+    end.synchronize()
+    per = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(steps)) / steps for i in range(n)]
+    return start.elapsed_time(end), per
+
+
+def bench_leg(w, steps, warmup, stream, device):
+    """Time one workload's step (copy, write, attention calls) with per-call events."""
+    import torch
+
+    from paged_kv_attention_34_b200.step import DeviceStep
+
+    with torch.cuda.stream(stream):
+        st = DeviceStep(w, device=device)
+    fns = []
+    names = []
+    if st.pairs is not None:
+        fns.append(st.copy_blocks)
+        names.append("kv_block_copy")
+    fns.append(st.write)
+    names.append("kv_cache_write")
+    for c in st.calls:
+        fns.append(lambda c=c: st.attend(c))
+        names.append("paged_attn_" + c.kind)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            for fn in fns:
+                fn()
+    torch.cuda.synchronize()
+    total, per = time_calls(fns, steps, stream)
+    stat = st.statuses()
+    if any(stat):
+        raise RuntimeError(f"{w.name}: device status {stat}")
+    return st, dict(zip(names, per)), total / steps
+
+
+# ---- our arm -------------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import paged_kv_attention_34_b200 as pa
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import DeviceStep, attn_bytes, attn_flops, copy_bytes, write_bytes
+
+    rank, local_rank, world = dist_env()
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    pa.lib()
+    peaks, peak_src = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    bf16_peak = float(peaks["bf16_tflops"])
+    stream = torch.cuda.Stream(device=device)
+
+    # ---- headline: 13B-shaped decode step ----
+    w = W.config2(seed=shard_seed(34_002, rank))
+    with torch.cuda.stream(stream):
+        st = DeviceStep(w, device=device)
+    call = st.calls[0]
+    fns = [st.write, lambda: st.attend(call)]
+    step_bytes = attn_bytes(w) + write_bytes(w)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for fn in fns:
+                fn()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    n_launch0 = pa.launch_count()
+    with ClockSampler(local_rank) as clk:
+        total_ms, per = time_calls(fns, args.steps, stream)
+    n_launch = pa.launch_count() - n_launch0
+    torch.cuda.synchronize()
+    barrier()
+    total_ms_max = reduce_max(total_ms, device)
+    bytes_all = reduce_sum(float(step_bytes * args.steps), device)
+    value = bytes_all / (total_ms_max * 1e-3) / 1e9
+    status = st.statuses()
+    if any(status):
+        raise RuntimeError(f"device status {status}")
+    decode_ms = per[1]
+    decode_bytes = attn_bytes(w)
+    achieved = decode_bytes / (decode_ms * 1e-3) / 1e9
+
+    # ---- e2e through the public API with host buffers ----
+    e2e = run_e2e(st, w, args, stream, device, step_bytes)
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic: seeded N(0,1) fp16 Q/K/V, uniform context lengths, shuffled 16-token blocks (no dataset)",
+        "config": {
+            "workload": HEADLINE,
+            "global_batch": 64 * world,
+            "seq_len": "context U[128,4096] (sum %d per rank 0)" % sum(w.ctx_lens),
+            "parallelism": f"dp{world} (independent sequences per rank, no data-path collective)",
+            "step": "kv_cache_write(64 new tokens) + paged_attn_decode (split kernel + merge)",
+            "l2": "no flush: the KV read per step (2.8 GB) is larger than the 126 MB L2",
+        },
+        "roofline": {
+            "kernel": "paged_attn_decode (split-KV kernel + LSE merge kernel, timed together)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": hbm_peak,
+            "peak_source": f"{peak_src} HBM copy bandwidth",
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4),
+            "frac_of_nominal_8TBs": round(achieved / 8000.0, 4),
+            "traffic": None,
+            "bytes_per_launch": decode_bytes,
+            "avg_launch_ms": round(decode_ms, 5),
+        },
+        "gpu_launches": n_launch,
+        "e2e": e2e,
+        "per_call_ms": {"kv_cache_write": round(per[0], 5), "paged_attn_decode": round(per[1], 5)},
+    }
+    clk_sum = clk.summary()
+    result["clocks"] = clk_sum if clk_sum else {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                                                 "note": "NVML unavailable"}
+
+    # ---- other legs (rank-local, reported for rank 0) ----
+    if not args.no_legs:
+        result["prefill"] = leg_prefill(args, stream, device, bf16_peak, peak_src, rank)
+        result["legs"] = {
+            "gqa_shared_prefix": leg_gqa(args, stream, device, hbm_peak, rank),
+            "mixed_step": leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank),
+        }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    del st
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(st, w, args, stream, device, step_bytes):
+    """The step with host buffers: H2D of the step inputs (pinned), the calls, D2H of the output."""
+    import torch
+
+    call = st.calls[0]
+    host = {
+        "q": w.q.pin_memory(),
+        "k_new": w.k_new.pin_memory(),
+        "v_new": w.v_new.pin_memory(),
+        "slot": w.slot_mapping.pin_memory(),
+        "bt": call.bt.cpu().pin_memory(),
+        "ctx": call.ctx.cpu().pin_memory(),
+        "cu": call.cu.cpu().pin_memory(),
+    }
+    out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one():
+        st.q.copy_(host["q"], non_blocking=True)
+        st.k_new.copy_(host["k_new"], non_blocking=True)
+        st.v_new.copy_(host["v_new"], non_blocking=True)
+        st.slot_mapping.copy_(host["slot"], non_blocking=True)
+        call.bt.copy_(host["bt"], non_blocking=True)
+        call.ctx.copy_(host["ctx"], non_blocking=True)
+        call.cu.copy_(host["cu"], non_blocking=True)
+        st.write()
+        st.attend(call)
+        out_host.copy_(st.out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one()
+    torch.cuda.synchronize()
+    barrier()
+    total_ms, _ = time_calls([one], args.steps, stream)
+    total_ms = reduce_max(total_ms, device)
+    bytes_all = reduce_sum(float(step_bytes * args.steps), device)
+    return {"value": round(bytes_all / (total_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(total_ms / args.steps, 6)}
+
+
+def leg_prefill(args, stream, device, bf16_peak, peak_src, rank):
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import attn_flops, write_bytes
+
+    w = W.config3(seed=shard_seed(34_003, rank))
+    st, per, step_ms = bench_leg(w, max(args.steps, 5), args.warmup, stream, device)
+    flops = attn_flops(w)
+    ms = per["paged_attn_prefill"]
+    tf = flops / (ms * 1e-3) / 1e12
+    wb = write_bytes(w)
+    return {
+        "workload": W.CONFIG_NAMES[3],
+        "metric": "prefill attn TFLOP/s (exact causal pairs, 4 d FLOP per pair)",
+        "value": round(tf, 2),
+        "unit": "TFLOP/s",
+        "bound": "tensor",
+        "peak": bf16_peak,
+        "peak_source": f"{peak_src} cuBLAS bf16 burst",
+        "frac": round(tf / bf16_peak, 4),
+        "frac_of_nominal_2250": round(tf / 2250.0, 4),
+        "flop_per_launch": flops,
+        "avg_launch_ms": round(ms, 5),
+        "kv_cache_write": {"GB/s": round(wb / (per["kv_cache_write"] * 1e-3) / 1e9, 1), "bytes": wb,
+                           "avg_launch_ms": round(per["kv_cache_write"], 5)},
+        "tokens_per_s": round(w.T / (step_ms * 1e-3), 1),
+    }
+
+
+def leg_gqa(args, stream, device, hbm_peak, rank):
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import attn_bytes
+
+    w = W.config4(seed=shard_seed(34_004, rank))
+    st, per, step_ms = bench_leg(w, max(args.steps, 5), args.warmup, stream, device)
+    b = attn_bytes(w)
+    ms = per["paged_attn_decode"]
+    gbs = b / (ms * 1e-3) / 1e9
+    return {"workload": W.CONFIG_NAMES[4], "decode_GB/s": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
+            "unique_bytes": b, "decode_ms": round(ms, 5), "step_ms": round(step_ms, 5),
+            "per_call_ms": {k: round(v, 5) for k, v in per.items()},
+            "note": "shared prefix counted once; its blocks may stay in L2 across sequences"}
+
+
+def leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank):
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import attn_bytes, attn_flops, write_bytes
+
+    w = W.config5(seed=shard_seed(34_005, rank))
+    st, per, step_ms = bench_leg(w, max(args.steps, 5), args.warmup, stream, device)
+    t_roof = {
+        "kv_cache_write": write_bytes(w) / (hbm_peak * 1e9),
+        "paged_attn_prefill": attn_flops(w, "prefill") / (bf16_peak * 1e12) + attn_bytes(w, "prefill") / (hbm_peak * 1e9),
+        "paged_attn_decode": attn_bytes(w, "decode") / (hbm_peak * 1e9),
+    }
+    meas = {k: per[k] * 1e-3 for k in t_roof}
+    return {"workload": W.CONFIG_NAMES[5], "frac": round(sum(t_roof.values()) / sum(meas.values()), 4),
+            "per_call_ms": {k: round(v, 5) for k, v in per.items()},
+            "per_call_frac": {k: round(t_roof[k] / meas[k], 4) for k in t_roof},
+            "tokens_per_s": round(w.T / (step_ms * 1e-3), 1), "step_ms": round(step_ms, 5)}
+
+
+# ---- the CPU oracle ---------------------------------------------------------------------------------------------
+
+def oracle_caches(w):
+    """The caches after the step's block copies and cache write, as the oracle computes them."""
+    import oracle
+
+    kc = oracle._u16(w.key_cache).copy()
+    vc = oracle._u16(w.value_cache).copy()
+    if w.copy_pairs is not None:
+        oracle.kv_block_copy(kc, vc, w.copy_pairs)
+    oracle.kv_cache_write(w.k_new, w.v_new, w.slot_mapping, kc, vc)
+    return kc, vc
+
+
+def oracle_sample_rate(w, caches, n_seq: int, threads: int):
+    """Run the fp64 oracle on the first n_seq sequences of a decode workload; returns (GB/s, seconds, bytes)."""
+    import numpy as np
+
+    import oracle
+    from paged_kv_attention_34_b200.step import attn_bytes
+    from paged_kv_attention_34_b200.workloads import AttnCall, Workload
+
+    kc, vc = caches
+    cu = w.cu_seqlens_q
+    t1 = int(cu[n_seq])
+    rows = np.arange(t1 * w.H_q, dtype=np.int64)
+    sub = Workload(**{**w.__dict__, "q_lens": w.q_lens[:n_seq], "ctx_lens": w.ctx_lens[:n_seq],
+                      "calls": [AttnCall("decode", 0, n_seq)]})
+    t0 = time.perf_counter()
+    oracle.paged_attention(w.q[:t1], kc, vc, oracle.dtype_code(w.dtype), w.block_tables[:n_seq], cu[: n_seq + 1],
+                           w.context_lens[:n_seq], w.H_kv, w.scale, rows=rows, n_threads=threads)
+    dt = time.perf_counter() - t0
+    b = attn_bytes(sub)
+    return b / dt / 1e9, dt, b
+
+
+def cpu_baseline(w, seconds: float):
+    """fp64 oracle on the host cores, on a bounded sample of the headline workload."""
+    threads = os.cpu_count() or 1
+    caches = oracle_caches(w)
+    rate, dt, _ = oracle_sample_rate(w, caches, 2, threads)  # calibration
+    n = max(2, min(w.B, int(math.ceil(2 * seconds / max(dt, 1e-3)))))
+    rate, dt, b = oracle_sample_rate(w, caches, n, threads)
+    return {"value": round(rate, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {n} of {w.B} sequences (all 40 heads), {b/1e9:.3f} GB of KV, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the fp64 oracle on host cores, bounded samples of the headline workload."""
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    from paged_kv_attention_34_b200 import workloads as W
+
+    w = W.config2(seed=shard_seed(34_002, 0))
+    threads = os.cpu_count() or 1
+    caches = oracle_caches(w)
+    _, dt, _ = oracle_sample_rate(w, caches, 2, threads)
+    # each step: a sample sized to about 2 s of host time
+    n = max(1, min(w.B, int(round(2 * 2.0 / max(dt, 1e-3)))))
+    for _ in range(args.warmup):
+        oracle_sample_rate(w, caches, n, threads)
+    tot_b, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        _, dt, b = oracle_sample_rate(w, caches, n, threads)
+        tot_b += b
+        tot_t += dt
+    value = tot_b / tot_t / 1e9
+    res = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic: seeded N(0,1) fp16 Q/K/V (same generator as the GPU arm)",
+        "config": {"workload": HEADLINE, "global_batch": 64, "seq_len": "context U[128,4096]",
+                   "parallelism": "host threads (OpenMP)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {n} of 64 sequences per step (all 40 heads)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

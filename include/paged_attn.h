@@ -1,0 +1,178 @@
+/*
+ * paged_attn.h -- C ABI of libpagedattn.so: exact attention over a paged KV
+ * cache on NVIDIA B200 (sm_100a).
+ *
+ * The method: softmax(Q K^T * scale) V computed tile by tile with an online
+ * softmax (running max m, running sum l), so the score matrix never reaches
+ * HBM ("大模型推理加速技术全景", iopencloud, sections 2.1-2.2), over a
+ * PagedAttention cache: K/V live in fixed 16-token blocks of a global pool,
+ * each sequence reaches its blocks through a block table (same page, section
+ * 3.2 and its page-table figure; the zhihu roofline page, "显存管理", gives
+ * 16 tokens as the default and adds refcounted copy-on-write blocks).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every pointer argument is a DEVICE pointer owned by the caller unless its
+ *   comment says otherwise.  Nothing is retained after the call returns and
+ *   nothing is freed.  The library allocates no device memory.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call only enqueues work on it and never synchronises.
+ * - Element type: pa_dtype, PA_F16 (IEEE binary16) or PA_BF16 (bfloat16), for
+ *   Q, O and the caches alike.  Accumulation and softmax are fp32.
+ * - Layouts (dense, row-major, no padding):
+ *     q, out              [T][H_q][d]        token-major; sequence b owns rows
+ *                                            cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *     k_new, v_new        [T][H_kv][d]
+ *     key_cache,
+ *     value_cache         [num_blocks][H_kv][16][d]   one (block, head) = 16*d contiguous
+ *     block_tables        int32 [B][max_blocks_per_seq]; page p of sequence b is
+ *                         block block_tables[b][p]; entries past the last page
+ *                         are never read
+ *     cu_seqlens_q        int32 [B+1], cu_seqlens_q[0] = 0, non-decreasing
+ *     context_lens        int32 [B], keys of sequence b INCLUDING its q_b new tokens
+ * - Positions: query i (0 <= i < q_b) of sequence b sits at absolute position
+ *   ctx_b - q_b + i and attends to keys 0 .. ctx_b - q_b + i (causal,
+ *   bottom-right aligned).  Keys past ctx_b in the last block are never used,
+ *   whatever they hold (NaN included).
+ * - GQA: H_q % H_kv == 0 and query head h reads KV head h / (H_q / H_kv).
+ * - Supported head sizes: d = 64 or 128.  All pointers 16-byte aligned.
+ * - Return value: PA_OK (0) or a negative pa_status.  Host-detectable argument
+ *   errors return at once and launch nothing.  Errors that only the device can
+ *   see (a block id or slot out of range, ctx_b > max_ctx, a bounded wait that
+ *   ran out) are written to a device status word (see pa_read_status); the
+ *   offending work item is skipped, never faulted.
+ */
+#ifndef PAGED_ATTN_H
+#define PAGED_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_ARG = -1,         /* a size, pointer or count is invalid */
+    PA_ERR_UNSUPPORTED = -2, /* d not in {64,128}, H_q % H_kv != 0, q_len > 8 in decode, ... */
+    PA_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned */
+    PA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than the *_workspace_bytes query */
+    PA_ERR_CUDA = -5,        /* a CUDA runtime call failed (launch, attribute, driver entry point) */
+    PA_ERR_TIMEOUT = -6,     /* device: a bounded wait on an asynchronous copy ran out */
+    PA_ERR_BOUNDS = -7,      /* device: a block id, slot or length was out of range; item skipped */
+    PA_ERR_SEQ = -8          /* device: cu_seqlens_q / context_lens inconsistent (q_b < 1, ctx_b < q_b, ...) */
+} pa_status;
+
+/* Size of the device status word area at the start of every workspace, bytes. */
+#define PA_STATUS_BYTES 256
+
+/*
+ * pa_kv_cache_write -- scatter the step's new K/V rows into the paged cache.
+ * For every token t with s = slot_mapping[t] >= 0:
+ *     key_cache[s / 16][h][s % 16][:] = k_new[t][h][:]   (h < H_kv), same for V.
+ * A negative slot marks a padding token and is skipped.  Slots >= 16*num_blocks
+ * are skipped and reported through `status` (PA_ERR_BOUNDS) when status != NULL.
+ * Bit-exact copy.  Slots must be distinct (two tokens on one slot: either wins).
+ * Follows: "Continuous Batching" answer of the interview Q&A page (a new
+ * token goes into the current block, a new block when it is full) and the
+ * page-table figure of iopencloud section 3.2.
+ *   k_new, v_new  [T][H_kv][d]         slot_mapping int32 [T]
+ *   status        optional device int32 (may be NULL); written only on error
+ */
+int pa_kv_cache_write(const void *k_new, const void *v_new, const int32_t *slot_mapping, int64_t T,
+                      void *key_cache, void *value_cache, int64_t num_blocks, int H_kv, int d, pa_dtype dtype,
+                      int32_t *status, void *stream);
+
+/*
+ * pa_kv_block_copy -- copy-on-write of shared blocks.  For each pair
+ * (src, dst) = (pairs[2i], pairs[2i+1]) copy K and V of every head and all 16
+ * rows of block src to block dst.  Pairs with an id outside [0, num_blocks)
+ * are skipped and reported through `status`.  A dst must not be the src of
+ * another pair in the same call (the copies run concurrently).  Bit-exact.
+ * Follows: zhihu roofline page, "显存管理" (refcounted blocks shared by
+ * several sequences are copied when one of them writes).
+ *   pairs  int32 [n][2], device memory
+ */
+int pa_kv_block_copy(void *key_cache, void *value_cache, int64_t num_blocks, int H_kv, int d, pa_dtype dtype,
+                     const int32_t *pairs, int64_t n, int32_t *status, void *stream);
+
+/*
+ * pa_decode_workspace_bytes -- device workspace that pa_paged_attn_decode needs
+ * for these sizes (status word + split-KV partial outputs and log-sum-exps).
+ * Pure host function.  Returns 0 for invalid sizes.
+ */
+size_t pa_decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx);
+
+/*
+ * pa_paged_attn_decode -- attention for 1..8 new query tokens per sequence
+ * (decode, and speculative verification of up to 7 drafted tokens), all
+ * query heads of one KV head processed together (GQA rows share each K/V tile).
+ * The KV range of each sequence is split across CTAs (split-KV decoding); each
+ * split keeps its own running max / sum and the splits are merged by
+ * log-sum-exp in a second kernel on the same stream ("FlashDecoding" answer
+ * of the interview Q&A page: split the long KV sequence over blocks, local
+ * softmax per block, then a cross-block reduction).
+ *   out          [T][H_q][d] written (same dtype as q)
+ *   q            [T][H_q][d], T = cu_seqlens_q[B]
+ *   cu_seqlens_q [B+1], each q_b in 1..8      context_lens [B], q_b <= ctx_b <= max_ctx
+ *   max_ctx      host upper bound of context_lens (sizes the split grid and workspace)
+ *   scale        multiplies Q K^T (normally 1/sqrt(d))
+ *   workspace    >= pa_decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx) bytes; its
+ *                first PA_STATUS_BYTES hold the status word, which this call resets
+ *                to PA_OK on `stream` before launching.
+ */
+int pa_paged_attn_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
+                         int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
+                         const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int max_ctx, int64_t T,
+                         int H_q, int H_kv, int d, float scale, pa_dtype dtype, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
+/*
+ * pa_prefill_workspace_bytes -- device workspace of pa_paged_attn_prefill
+ * (status word and the tile scheduler's state).  Pure host function.
+ */
+size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len);
+
+/*
+ * pa_paged_attn_prefill -- causal variable-length attention for prompts or
+ * prompt chunks whose K/V were already written into the paged cache (by
+ * pa_kv_cache_write).  Sequences are packed through cu_seqlens_q (no padding,
+ * block-diagonal mask: the ragged-batching answer of the interview Q&A page);
+ * a chunk with earlier context attends to that context too (chunked prefill).
+ * Tiles of 128 queries x 128 keys run on the tcgen05 tensor cores with fp32
+ * accumulators in tensor memory, fed by TMA from the cache blocks; the online
+ * softmax of iopencloud section 2.2 runs between the two products.
+ *   out, q        [T][H_q][d]        cu_seqlens_q [B+1] (q_b >= 1)   context_lens [B]
+ *   max_q_len     host upper bound of q_b;  max_ctx host upper bound of ctx_b
+ *   workspace     >= pa_prefill_workspace_bytes(...) bytes; status word reset on stream.
+ */
+int pa_paged_attn_prefill(void *out, const void *q, const void *key_cache, const void *value_cache,
+                          int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int max_q_len,
+                          int max_ctx, int64_t T, int H_q, int H_kv, int d, float scale, pa_dtype dtype,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * pa_read_status -- copy the device status word at the start of `workspace`
+ * (or any device int32 given to the write/copy calls) into *host_status.
+ * This call synchronises `stream`.  Returns PA_OK or PA_ERR_CUDA.
+ */
+int pa_read_status(const void *workspace, int32_t *host_status, void *stream);
+
+/* pa_strerror -- static text for a pa_status value. */
+const char *pa_strerror(int code);
+
+/* pa_launch_count -- number of kernels this library has launched in this process. */
+uint64_t pa_launch_count(void);
+
+/* pa_version -- library ABI version (major * 100 + minor). */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_ATTN_H */

@@ -1,0 +1,260 @@
+"""Python binding of libpagedattn (exact attention over a paged KV cache, B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libpagedattn.so``, reached through its C ABI
+(``include/paged_attn.h``) with ctypes.  Tensors are torch CUDA tensors;
+the current torch stream is passed to every call.  There is no fallback: if
+the library is not built, or a tensor is not on a CUDA device, the call
+raises.
+
+Calls (same names as the C ABI without the ``pa_`` prefix):
+
+* ``kv_cache_write(k_new, v_new, slot_mapping, key_cache, value_cache)``
+* ``kv_block_copy(key_cache, value_cache, pairs)``
+* ``paged_attn_decode(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, max_ctx, scale)``
+* ``paged_attn_prefill(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, max_q_len, max_ctx, scale)``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpagedattn.so")
+
+PA_F16, PA_BF16 = 0, 1
+PA_STATUS_BYTES = 256
+STATUS_NAMES = {
+    0: "PA_OK",
+    -1: "PA_ERR_ARG",
+    -2: "PA_ERR_UNSUPPORTED",
+    -3: "PA_ERR_ALIGN",
+    -4: "PA_ERR_WORKSPACE",
+    -5: "PA_ERR_CUDA",
+    -6: "PA_ERR_TIMEOUT",
+    -7: "PA_ERR_BOUNDS",
+    -8: "PA_ERR_SEQ",
+}
+
+_lib = None
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)} ({strerror(code)})")
+
+
+def _declare(L):
+    c = ctypes
+    P, I, I64, SZ = c.c_void_p, c.c_int, c.c_int64, c.c_size_t
+    L.pa_kv_cache_write.restype = I
+    L.pa_kv_cache_write.argtypes = [P, P, P, I64, P, P, I64, I, I, I, P, P]
+    L.pa_kv_block_copy.restype = I
+    L.pa_kv_block_copy.argtypes = [P, P, I64, I, I, I, P, I64, P, P]
+    L.pa_decode_workspace_bytes.restype = SZ
+    L.pa_decode_workspace_bytes.argtypes = [I64, I, I, I, I, I]
+    L.pa_paged_attn_decode.restype = I
+    L.pa_paged_attn_decode.argtypes = [P, P, P, P, I64, P, I, P, P, I, I, I64, I, I, I, c.c_float, I, P, SZ, P]
+    L.pa_prefill_workspace_bytes.restype = SZ
+    L.pa_prefill_workspace_bytes.argtypes = [I, I, I, I, I]
+    L.pa_paged_attn_prefill.restype = I
+    L.pa_paged_attn_prefill.argtypes = [P, P, P, P, I64, P, I, P, P, I, I, I, I64, I, I, I, c.c_float, I, P, SZ, P]
+    L.pa_read_status.restype = I
+    L.pa_read_status.argtypes = [P, P, P]
+    L.pa_strerror.restype = c.c_char_p
+    L.pa_strerror.argtypes = [I]
+    L.pa_launch_count.restype = c.c_uint64
+    L.pa_launch_count.argtypes = []
+    L.pa_version.restype = I
+    L.pa_version.argtypes = []
+    return L
+
+
+def lib():
+    """The loaded C library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m paged_kv_attention_34_b200._build` "
+                "(or __graft_entry__.build()); there is no fallback implementation"
+            )
+        _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().pa_strerror(int(code)).decode()
+
+
+def launch_count() -> int:
+    return int(lib().pa_launch_count())
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise PagedAttnError(rc, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None, ndim=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    return t
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def kv_cache_write(k_new, v_new, slot_mapping, key_cache, value_cache, status=None, stream=None):
+    """Scatter k_new/v_new [T, H_kv, d] into the caches [NB, H_kv, 16, d] at slot_mapping [T] (int32)."""
+    _cuda(key_cache, "key_cache", ndim=4)
+    dt = key_cache.dtype
+    _cuda(value_cache, "value_cache", dt, 4)
+    _cuda(k_new, "k_new", dt, 3)
+    _cuda(v_new, "v_new", dt, 3)
+    _cuda(slot_mapping, "slot_mapping", torch.int32, 1)
+    NB, H_kv, bs, d = key_cache.shape
+    T = k_new.shape[0]
+    if bs != 16 or value_cache.shape != key_cache.shape or k_new.shape != (T, H_kv, d) or v_new.shape != k_new.shape:
+        raise ValueError("shape mismatch between k_new/v_new [T,H_kv,d] and caches [NB,H_kv,16,d]")
+    if slot_mapping.shape[0] != T:
+        raise ValueError("slot_mapping must have T entries")
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    rc = lib().pa_kv_cache_write(
+        _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T, _ptr(key_cache), _ptr(value_cache), NB, H_kv, d,
+        _dtype_code(key_cache), _ptr(status), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_kv_cache_write")
+
+
+def kv_block_copy(key_cache, value_cache, pairs, status=None, stream=None):
+    """Copy-on-write: copy block pairs[i,0] to pairs[i,1] in both caches (pairs: int32 [n, 2])."""
+    _cuda(key_cache, "key_cache", ndim=4)
+    _cuda(value_cache, "value_cache", key_cache.dtype, 4)
+    _cuda(pairs, "pairs", torch.int32, 2)
+    NB, H_kv, _, d = key_cache.shape
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    rc = lib().pa_kv_block_copy(
+        _ptr(key_cache), _ptr(value_cache), NB, H_kv, d, _dtype_code(key_cache), _ptr(pairs), pairs.shape[0],
+        _ptr(status), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_kv_block_copy")
+
+
+def decode_workspace_bytes(T: int, B: int, H_q: int, H_kv: int, d: int, max_ctx: int) -> int:
+    n = lib().pa_decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx)
+    if n == 0:
+        raise ValueError("invalid sizes for pa_decode_workspace_bytes")
+    return int(n)
+
+
+def prefill_workspace_bytes(B: int, H_q: int, H_kv: int, d: int, max_q_len: int) -> int:
+    n = lib().pa_prefill_workspace_bytes(B, H_q, H_kv, d, max_q_len)
+    if n == 0:
+        raise ValueError("invalid sizes for pa_prefill_workspace_bytes")
+    return int(n)
+
+
+def _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, out):
+    _cuda(q, "q", ndim=3)
+    dt = q.dtype
+    _cuda(key_cache, "key_cache", dt, 4)
+    _cuda(value_cache, "value_cache", dt, 4)
+    _cuda(block_tables, "block_tables", torch.int32, 2)
+    _cuda(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _cuda(context_lens, "context_lens", torch.int32, 1)
+    T, H_q, d = q.shape
+    NB, H_kv, bs, dk = key_cache.shape
+    if bs != 16 or dk != d or value_cache.shape != key_cache.shape:
+        raise ValueError("caches must be [NB, H_kv, 16, d] with d matching q")
+    B = context_lens.shape[0]
+    if cu_seqlens_q.shape[0] != B + 1 or block_tables.shape[0] != B:
+        raise ValueError("cu_seqlens_q must have B+1 entries and block_tables B rows")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _cuda(out, "out", dt, 3)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    return out, T, H_q, d, NB, H_kv, B
+
+
+def _workspace(ws, nbytes, device):
+    if ws is None:
+        return torch.empty(nbytes, dtype=torch.uint8, device=device)
+    _cuda(ws, "workspace", torch.uint8, 1)
+    if ws.numel() < nbytes:
+        raise ValueError(f"workspace too small: {ws.numel()} < {nbytes}")
+    return ws
+
+
+def paged_attn_decode(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, max_ctx: int,
+                      scale: float, out=None, workspace=None, stream=None):
+    """Split-KV decode for 1..8 query tokens per sequence; returns out [T, H_q, d]."""
+    out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
+                                               context_lens, out)
+    nbytes = decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx)
+    ws = _workspace(workspace, nbytes, q.device)
+    rc = lib().pa_paged_attn_decode(
+        _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
+        _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_ctx), T, H_q, H_kv, d, float(scale),
+        _dtype_code(q), _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_paged_attn_decode")
+    paged_attn_decode.last_workspace = ws
+    return out
+
+
+def paged_attn_prefill(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, max_q_len: int,
+                       max_ctx: int, scale: float, out=None, workspace=None, stream=None):
+    """Causal varlen prefill over the paged cache; returns out [T, H_q, d]."""
+    out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
+                                               context_lens, out)
+    nbytes = prefill_workspace_bytes(B, H_q, H_kv, d, max_q_len)
+    ws = _workspace(workspace, nbytes, q.device)
+    rc = lib().pa_paged_attn_prefill(
+        _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
+        _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_q_len), int(max_ctx), T, H_q, H_kv, d, float(scale),
+        _dtype_code(q), _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_paged_attn_prefill")
+    paged_attn_prefill.last_workspace = ws
+    return out
+
+
+def read_status(workspace: torch.Tensor, stream=None) -> int:
+    """Device status word at the start of a workspace (or a status tensor); synchronises the stream."""
+    _cuda(workspace, "workspace")
+    val = ctypes.c_int32(0)
+    rc = lib().pa_read_status(_ptr(workspace), ctypes.byref(val), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "pa_read_status")
+    return int(val.value)

@@ -1,0 +1,630 @@
+// Paged attention for groups of up to 64 query rows that share one KV head.
+//
+// Decode ("FlashDecoding" answer of the interview Q&A page): the rows of a
+// CTA are the G query heads x q_b new tokens of one (sequence, KV head); the
+// sequence's pages are split into ranges of `split_pages` pages handled by
+// different CTAs; each split keeps its own running max m and sum l (online
+// softmax, iopencloud "大模型推理加速技术全景" section 2.2) and writes a
+// normalised partial O_s with its log-sum-exp; pa_split_merge_kernel then
+// combines the splits ("cross-block reduction").  A sequence short enough
+// for one split is written straight to `out`.
+//
+// Data movement: one thread issues TMA box loads (64 elements x 16 rows,
+// 128-byte swizzle) of whole (block, head) pages straight from the block pool
+// into a ring of shared-memory stages; completion is tracked by mbarriers with
+// bounded waits.  The page ids come from the block table (iopencloud section
+// 3.2), prefetched into shared memory.  K/V bytes are read once per CTA.
+//
+// Compute: four warps; each owns a 16-row m-tile and a subset of the pages of
+// every stage (several warps on different pages when there are <= 32 rows,
+// merged at the end like splits).  S = Q K^T and O += P V run on mma.sync
+// m16n8k16 with fp32 accumulators; P is rounded to the input type for P V.
+#include <cmath>
+
+#include "pa_device.cuh"
+#include "pa_internal.h"
+
+namespace pa {
+
+constexpr int kRowsPerCta = 64;
+constexpr int kPagesPerStage = 4;
+constexpr int kMaxTablePages = 1024;  // page ids cached in shared memory per CTA
+constexpr int kThreads = 128;
+
+struct RowsParams {
+    const void *q;
+    void *out;
+    const int32_t *block_tables;
+    const int32_t *cu_seqlens;
+    const int32_t *context_lens;
+    float *ws_o;    // [max_splits][T][H_q][D] normalised partial outputs
+    float *ws_lse;  // [max_splits][T][H_q] log2-sum-exp of the scaled scores
+    int32_t *status;
+    int64_t num_blocks;
+    int64_t T;
+    int max_blocks;
+    int B, H_q, H_kv, G;
+    int max_ctx;
+    int max_q_len;
+    int n_rg;         // row groups of 64 rows per (sequence, KV head)
+    int split_pages;  // pages per split (decode); >= all pages for prefill
+    float scale_log2;  // scale * log2(e)
+    int decode;        // 1: split-KV decode grid, 0: prefill grid
+};
+
+template <int D, int STAGES>
+struct RowsSmem {
+    static constexpr int kPageBytes = 16 * D * 2;
+    static constexpr int kStageBytes = 2 * kPagesPerStage * kPageBytes;  // K pages then V pages
+    static constexpr int kQBytes = kRowsPerCta * D * 2;
+    static constexpr int kEpiStride = D + 8;  // floats per row of the epilogue buffer
+    static constexpr int kEpiBytes = (4 * 16 * kEpiStride + 2 * 64) * 4;
+    static_assert(kEpiBytes <= STAGES * kStageBytes, "epilogue must fit in the stage ring");
+    static constexpr int kStageOff = 0;
+    static constexpr int kQOff = STAGES * kStageBytes;
+    static constexpr int kBarOff = kQOff + kQBytes;
+    static constexpr int kTableOff = kBarOff + 8 * STAGES;
+    static constexpr int kFlagOff = kTableOff + 4 * kMaxTablePages;
+    static constexpr int kBytes = kFlagOff + 16;
+    static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (swizzle atoms)
+};
+
+__device__ __forceinline__ int seq_of_token(const int32_t *cu, int B, int64_t t)
+{
+    int lo = 0, hi = B;  // cu[lo] <= t < cu[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(cu + mid) <= t)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Sequence checks shared by the attention and merge kernels.
+__device__ __forceinline__ bool seq_ok(int qb, int ctx, const RowsParams &p, int64_t q1)
+{
+    return qb >= 1 && ctx >= qb && qb <= p.max_q_len && ctx <= p.max_ctx && ctx <= p.max_blocks * 16 && q1 <= p.T;
+}
+
+template <int D, bool BF16, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    pa_attn_rows_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                        const RowsParams p)
+{
+    using L = RowsSmem<D, STAGES>;
+    constexpr int CH = D / 8;       // 16-byte chunks per row
+    constexpr int BOXES = D / 64;   // TMA boxes per page
+    constexpr int KSTEPS = D / 16;  // k-steps of S = Q K^T
+    constexpr int NT = D / 8;       // n-tiles of O
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *s_stage = smem + L::kStageOff;
+    uint8_t *s_q = smem + L::kQOff;
+    uint64_t *s_bar = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    int32_t *s_pages = reinterpret_cast<int32_t *>(smem + L::kTableOff);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- which (sequence, KV head, row group, split) --------------------------------
+    const int b = blockIdx.z;
+    int g, rg, split;
+    if (p.decode) {
+        split = blockIdx.x;
+        g = blockIdx.y / p.n_rg;
+        rg = blockIdx.y % p.n_rg;
+    } else {
+        split = 0;
+        g = blockIdx.y;
+        rg = p.n_rg - 1 - blockIdx.x;  // later row groups see more keys: launch them first
+    }
+    const int q0 = __ldg(p.cu_seqlens + b), q1 = __ldg(p.cu_seqlens + b + 1);
+    const int qb = q1 - q0, ctx = __ldg(p.context_lens + b);
+    if (!seq_ok(qb, ctx, p, q1)) {
+        if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+            set_status(p.status, PA_ERR_SEQ);
+        return;
+    }
+    const int G = p.G;
+    const int R = G * qb;
+    const int row0 = rg * kRowsPerCta;
+    if (row0 >= R)
+        return;
+    const int rows_here = min(kRowsPerCta, R - row0);
+    const int lim_cta = ctx - qb + (row0 + rows_here - 1) / G;  // last key any row here sees
+    const int pages_need = lim_cta / 16 + 1;
+    const int pages_ctx = (ctx + 15) / 16;
+    int n_splits = 1, page_lo = 0, page_hi = pages_need;
+    if (p.decode) {
+        n_splits = (pages_ctx + p.split_pages - 1) / p.split_pages;
+        if (split >= n_splits)
+            return;
+        page_lo = split * p.split_pages;
+        page_hi = min(page_lo + p.split_pages, pages_need);
+    }
+    const int n_pages = max(0, page_hi - page_lo);
+    const int n_stages = (n_pages + kPagesPerStage - 1) / kPagesPerStage;
+
+    // warp roles: MT m-tiles of 16 rows, KG warps per m-tile on different pages
+    const int MT = rows_here <= 16 ? 1 : (rows_here <= 32 ? 2 : 4);
+    const int KG = 4 / MT;
+    const int mt = warp / KG, kg = warp % KG;
+    const bool has_rows = mt * 16 < rows_here;
+
+    // ---- set-up: barriers, page ids, Q tile ---------------------------------------------
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s)
+            mbar_init(&s_bar[s], 1);
+        *s_abort = 0;
+        fence_barrier_init();
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+    }
+    const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
+    for (int i = tid; i < min(n_pages, kMaxTablePages); i += kThreads) {
+        int pg = __ldg(table + page_lo + i);
+        if (pg < 0 || pg >= p.num_blocks) {
+            set_status(p.status, PA_ERR_BOUNDS);
+            pg = static_cast<int>(p.num_blocks);  // past the pool: TMA fills zeros
+        }
+        s_pages[i] = pg;
+    }
+    for (int i = tid; i < kRowsPerCta * CH; i += kThreads) {
+        const int r = i / CH, c = i % CH;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < rows_here) {
+            const int ridx = row0 + r;
+            const int64_t t = q0 + ridx / G;
+            const int h = g * G + ridx % G;
+            v = __ldg(reinterpret_cast<const uint4 *>(p.q) + (t * p.H_q + h) * CH + c);
+        }
+        *reinterpret_cast<uint4 *>(s_q + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
+    }
+    __syncthreads();
+
+    auto page_id = [&](int i) -> int {
+        if (i < kMaxTablePages)
+            return s_pages[i];
+        int pg = __ldg(table + page_lo + i);
+        if (pg < 0 || pg >= p.num_blocks) {
+            set_status(p.status, PA_ERR_BOUNDS);
+            pg = static_cast<int>(p.num_blocks);
+        }
+        return pg;
+    };
+    auto issue = [&](int st) {  // thread 0 only
+        const int slot = st % STAGES;
+        uint8_t *kb = s_stage + slot * L::kStageBytes;
+        uint8_t *vb = kb + kPagesPerStage * L::kPageBytes;
+        const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&s_bar[slot], np * 2 * L::kPageBytes);
+        for (int k = 0; k < np; ++k) {
+            const int y = (page_id(st * kPagesPerStage + k) * p.H_kv + g) * 16;
+#pragma unroll
+            for (int bx = 0; bx < BOXES; ++bx) {
+                tma_load_2d(kb + k * L::kPageBytes + bx * 2048, &tmap_k, bx * 64, y, &s_bar[slot]);
+                tma_load_2d(vb + k * L::kPageBytes + bx * 2048, &tmap_v, bx * 64, y, &s_bar[slot]);
+            }
+        }
+    };
+    if (tid == 0)
+        for (int st = 0; st < min(STAGES, n_stages); ++st)
+            issue(st);
+
+    // ---- per-thread row state --------------------------------------------------------------
+    // This thread holds rows ra = lane/4 and rb = ra + 8 of its warp's m-tile.
+    const int ra = mt * 16 + (lane >> 2), rb = ra + 8;
+    const int lim_a = ra < rows_here ? ctx - qb + (row0 + ra) / G : -1;
+    const int lim_b = rb < rows_here ? ctx - qb + (row0 + rb) / G : -1;
+    const int lim_warp = has_rows ? ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G : -1;
+
+    uint32_t qa[KSTEPS][4];
+    if (has_rows) {
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+            const int mi = lane >> 3, rr = lane & 7;
+            const int r = mt * 16 + (mi & 1) * 8 + rr;
+            const int c = 2 * ks + (mi >> 1);
+            ldsm_x4(smem_u32(s_q + r * (D * 2) + ((c ^ (r & 7)) << 4)), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+        }
+    }
+    float o[NT][4];
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+        o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    const float sl2 = p.scale_log2;
+    const int kq = lane & 3;
+
+    // ---- main loop over stages ---------------------------------------------------------------
+    int it = 0;
+    for (; it < n_stages; ++it) {
+        const int slot = it % STAGES;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_bar[slot], (it / STAGES) & 1));
+        if (!ok) {
+            *s_abort = 1;
+            set_status(p.status, PA_ERR_TIMEOUT);
+        }
+        if (ok && has_rows) {
+            const uint8_t *kst = s_stage + slot * L::kStageBytes;
+            const uint8_t *vst = kst + kPagesPerStage * L::kPageBytes;
+            for (int k = kg; k < kPagesPerStage; k += KG) {
+                const int pidx = it * kPagesPerStage + k;
+                if (pidx >= n_pages)
+                    break;
+                const int j0 = (page_lo + pidx) * 16;
+                if (j0 > lim_warp)
+                    continue;  // every row of this warp is causally masked on this page
+                const uint32_t kbase = smem_u32(kst + k * L::kPageBytes);
+                const uint32_t vbase = smem_u32(vst + k * L::kPageBytes);
+
+                // S (16 rows x 16 keys) = Q K^T
+                float s[2][4];
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const int mi = lane >> 3, rr = lane & 7;
+                    const int key = (mi >> 1) * 8 + rr;
+                    const int c = 2 * ks + (mi & 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kbase + (c >> 3) * 2048 + key * 128 + (((c & 7) ^ (key & 7)) << 4), b0, b1, b2, b3);
+                    mma16816<BF16>(s[0], qa[ks], b0, b1);
+                    mma16816<BF16>(s[1], qa[ks], b2, b3);
+                }
+                // mask (causal / context end), scale to log2 units, online softmax
+                float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const int key = j0 + nt * 8 + 2 * kq + c;
+                        s[nt][c] = key <= lim_a ? s[nt][c] * sl2 : -INFINITY;
+                        s[nt][2 + c] = key <= lim_b ? s[nt][2 + c] * sl2 : -INFINITY;
+                        mx_a = fmaxf(mx_a, s[nt][c]);
+                        mx_b = fmaxf(mx_b, s[nt][2 + c]);
+                    }
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+                const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
+                const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
+                const float al_a = fast_exp2(m_a - base_a), al_b = fast_exp2(m_b - base_b);
+                m_a = mn_a;
+                m_b = mn_b;
+                float ps_a = 0.f, ps_b = 0.f;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    s[nt][0] = fast_exp2(s[nt][0] - base_a);
+                    s[nt][1] = fast_exp2(s[nt][1] - base_a);
+                    s[nt][2] = fast_exp2(s[nt][2] - base_b);
+                    s[nt][3] = fast_exp2(s[nt][3] - base_b);
+                    ps_a += s[nt][0] + s[nt][1];
+                    ps_b += s[nt][2] + s[nt][3];
+                }
+                l_a = l_a * al_a + ps_a;
+                l_b = l_b * al_b + ps_b;
+                if (__any_sync(0xffffffffu, al_a != 1.f || al_b != 1.f)) {
+#pragma unroll
+                    for (int nd = 0; nd < NT; ++nd) {
+                        o[nd][0] *= al_a;
+                        o[nd][1] *= al_a;
+                        o[nd][2] *= al_b;
+                        o[nd][3] *= al_b;
+                    }
+                }
+                uint32_t pa_[4];
+                pa_[0] = pack2<BF16>(s[0][0], s[0][1]);
+                pa_[1] = pack2<BF16>(s[0][2], s[0][3]);
+                pa_[2] = pack2<BF16>(s[1][0], s[1][1]);
+                pa_[3] = pack2<BF16>(s[1][2], s[1][3]);
+
+                // keys past the context end may hold anything (NaN): zero their V
+                uint32_t vm_lo = 0xffffffffu, vm_hi = 0xffffffffu;
+                if (j0 + 16 > ctx) {
+                    const int valid = ctx - j0;
+                    const int k0 = 2 * kq;
+                    vm_lo = (k0 < valid ? 0x0000ffffu : 0u) | (k0 + 1 < valid ? 0xffff0000u : 0u);
+                    vm_hi = (k0 + 8 < valid ? 0x0000ffffu : 0u) | (k0 + 9 < valid ? 0xffff0000u : 0u);
+                }
+                // O (16 x D) += P (16 x 16 keys) V (16 keys x D)
+#pragma unroll
+                for (int ndp = 0; ndp < NT / 2; ++ndp) {
+                    const int mi = lane >> 3, rr = lane & 7;
+                    const int key = (mi & 1) * 8 + rr;
+                    const int c = 2 * ndp + (mi >> 1);
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4_t(vbase + (c >> 3) * 2048 + key * 128 + (((c & 7) ^ (key & 7)) << 4), r0, r1, r2, r3);
+                    r0 &= vm_lo;
+                    r1 &= vm_hi;
+                    r2 &= vm_lo;
+                    r3 &= vm_hi;
+                    mma16816<BF16>(o[2 * ndp], pa_, r0, r1);
+                    mma16816<BF16>(o[2 * ndp + 1], pa_, r2, r3);
+                }
+            }
+        }
+        __syncthreads();  // every warp is done with this slot
+        if (*s_abort)
+            break;
+        if (tid == 0 && it + STAGES < n_stages)
+            issue(it + STAGES);
+    }
+    if (*s_abort) {
+        // let the copies still in flight land (bounded) before the CTA releases its shared memory
+        if (tid == 0)
+            for (int st = it; st < min(it + STAGES, n_stages); ++st)
+                mbar_wait(&s_bar[st % STAGES], (st / STAGES) & 1, kWaitTimeoutNs / 10);
+        return;
+    }
+
+    // ---- epilogue: merge the warps of each m-tile, normalise, store --------------------------
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    float *e_o = reinterpret_cast<float *>(s_stage);  // [4 warps][16 rows][kEpiStride]
+    float *e_m = e_o + 4 * 16 * L::kEpiStride;        // [4][16]
+    float *e_l = e_m + 64;                            // [4][16]
+    if (has_rows) {
+        const int la = lane >> 2, lb = la + 8;
+#pragma unroll
+        for (int nd = 0; nd < NT; ++nd) {
+            const int col = nd * 8 + 2 * kq;
+            *reinterpret_cast<float2 *>(e_o + (warp * 16 + la) * L::kEpiStride + col) = make_float2(o[nd][0], o[nd][1]);
+            *reinterpret_cast<float2 *>(e_o + (warp * 16 + lb) * L::kEpiStride + col) = make_float2(o[nd][2], o[nd][3]);
+        }
+        if (kq == 0) {
+            e_m[warp * 16 + la] = m_a;
+            e_m[warp * 16 + lb] = m_b;
+            e_l[warp * 16 + la] = l_a;
+            e_l[warp * 16 + lb] = l_b;
+        }
+    }
+    __syncthreads();
+    const bool final_out = n_splits == 1;
+    for (int i = tid; i < rows_here * (D / 4); i += kThreads) {
+        const int r = i / (D / 4), c4 = i % (D / 4);
+        const int mtr = r >> 4, lr = r & 15;
+        float M = -INFINITY;
+        for (int k = 0; k < KG; ++k)
+            M = fmaxf(M, e_m[(mtr * KG + k) * 16 + lr]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float Lsum = 0.f;
+        for (int k = 0; k < KG; ++k) {
+            const int w = mtr * KG + k;
+            const float mk = e_m[w * 16 + lr];
+            const float wt = mk == -INFINITY ? 0.f : fast_exp2(mk - M);
+            Lsum += wt * e_l[w * 16 + lr];
+            const float4 v = *reinterpret_cast<const float4 *>(e_o + (w * 16 + lr) * L::kEpiStride + c4 * 4);
+            acc.x += wt * v.x;
+            acc.y += wt * v.y;
+            acc.z += wt * v.z;
+            acc.w += wt * v.w;
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        const int ridx = row0 + r;
+        const int64_t t = q0 + ridx / G;
+        const int h = g * G + ridx % G;
+        const int64_t orow = t * p.H_q + h;
+        if (final_out) {
+            store4<BF16>(static_cast<uint8_t *>(p.out) + (orow * D + c4 * 4) * 2, acc.x * inv, acc.y * inv,
+                         acc.z * inv, acc.w * inv);
+        } else {
+            const int64_t prow = (int64_t)split * p.T * p.H_q + orow;
+            *reinterpret_cast<float4 *>(p.ws_o + prow * D + c4 * 4) =
+                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            if (c4 == 0)
+                p.ws_lse[prow] = Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
+        }
+    }
+}
+
+// One warp per (token, query head) row of a sequence with more than one split:
+// O = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+    if (row >= p.T * p.H_q)
+        return;
+    const int64_t t = row / p.H_q;
+    const int b = seq_of_token(p.cu_seqlens, p.B, t);
+    const int q0 = __ldg(p.cu_seqlens + b), q1 = __ldg(p.cu_seqlens + b + 1);
+    const int ctx = __ldg(p.context_lens + b);
+    if (!seq_ok(q1 - q0, ctx, p, q1))
+        return;
+    const int pages_ctx = (ctx + 15) / 16;
+    const int ns = (pages_ctx + p.split_pages - 1) / p.split_pages;
+    if (ns <= 1)
+        return;
+    const int64_t stride = p.T * p.H_q;
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32)
+        M = fmaxf(M, p.ws_lse[s * stride + row]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Z = 0.f;
+    for (int s = lane; s < ns; s += 32) {
+        const float l = p.ws_lse[s * stride + row];
+        Z += l == -INFINITY ? 0.f : fast_exp2(l - M);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        Z += __shfl_xor_sync(0xffffffffu, Z, o);
+    const float invZ = Z > 0.f ? 1.f / Z : 0.f;
+    constexpr int LANES = D / 4;
+    if (lane < LANES) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s = 0; s < ns; ++s) {
+            const float l = p.ws_lse[s * stride + row];
+            if (l == -INFINITY)
+                continue;
+            const float w = fast_exp2(l - M) * invZ;
+            const float4 v = *reinterpret_cast<const float4 *>(p.ws_o + (s * stride + row) * D + lane * 4);
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+        }
+        store4<BF16>(static_cast<uint8_t *>(p.out) + (row * D + lane * 4) * 2, acc.x, acc.y, acc.z, acc.w);
+    }
+}
+
+// ---- host side ------------------------------------------------------------------------------
+
+constexpr int kStages = 2;
+
+template <int D, bool BF16>
+static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
+                       cudaStream_t stream)
+{
+    using L = RowsSmem<D, kStages>;
+    auto kern = pa_attn_rows_kernel<D, BF16, kStages>;
+    static uint64_t configured = 0;  // one bit per device, per template instance
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return PA_ERR_CUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (!bit || !(configured & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured |= bit;
+    }
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(tk, tv, rp);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+static int launch_merge(const RowsParams &rp, cudaStream_t stream)
+{
+    const int64_t rows = rp.T * rp.H_q;
+    const int64_t blocks = (rows + 7) / 8;
+    pa_split_merge_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(rp);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+static int split_pages_override()
+{
+    static int v = -2;
+    if (v == -2) {
+        const char *e = getenv("PA_DECODE_SPLIT_PAGES");
+        v = e ? atoi(e) : -1;
+    }
+    return v;
+}
+
+DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
+{
+    (void)d;
+    DecodePlan pl;
+    const int G = H_q / H_kv;
+    pl.row_groups = (8 * G + kRowsPerCta - 1) / kRowsPerCta;
+    const int64_t pages = (int64_t)(max_ctx + 15) / 16;
+    // Aim for about 8 waves of CTAs over the SMs (2 resident per SM), never
+    // fewer than 16 pages (256 keys) per split; a multiple of the stage size.
+    const int64_t units = (int64_t)B * H_kv * pl.row_groups;
+    const int64_t slots = (int64_t)sm_count() * 2 * 8;
+    int64_t sp = units > 0 ? (units * pages + slots - 1) / slots : pages;
+    sp = sp < 16 ? 16 : sp;
+    sp = (sp + kPagesPerStage - 1) / kPagesPerStage * kPagesPerStage;
+    if (sp > kMaxTablePages)
+        sp = kMaxTablePages;
+    const int ov = split_pages_override();
+    if (ov > 0)
+        sp = ov;
+    pl.split_pages = static_cast<int>(sp);
+    pl.max_splits = pages > 0 ? static_cast<int>((pages + sp - 1) / sp) : 1;
+    return pl;
+}
+
+size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx)
+{
+    const DecodePlan pl = decode_plan(B, H_q, H_kv, d, max_ctx);
+    size_t bytes = PA_STATUS_BYTES;
+    if (pl.max_splits > 1) {
+        const size_t rows = static_cast<size_t>(pl.max_splits) * static_cast<size_t>(T) * H_q;
+        bytes += rows * d * sizeof(float);
+        bytes += rows * sizeof(float);
+        bytes += 256;
+    }
+    return bytes;
+}
+
+template <int D, bool BF16>
+static int run(const AttnArgs &a, bool decode)
+{
+    CUtensorMap tk, tv;
+    int rc = make_cache_tmap(&tk, a.key_cache, a.num_blocks, a.H_kv, D, a.dtype);
+    if (rc == PA_OK)
+        rc = make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
+    if (rc != PA_OK)
+        return rc;
+    RowsParams rp{};
+    rp.q = a.q;
+    rp.out = a.out;
+    rp.block_tables = a.block_tables;
+    rp.cu_seqlens = a.cu_seqlens_q;
+    rp.context_lens = a.context_lens;
+    rp.status = static_cast<int32_t *>(a.workspace);
+    rp.num_blocks = a.num_blocks;
+    rp.T = a.T;
+    rp.max_blocks = a.max_blocks;
+    rp.B = a.B;
+    rp.H_q = a.H_q;
+    rp.H_kv = a.H_kv;
+    rp.G = a.H_q / a.H_kv;
+    rp.max_ctx = a.max_ctx;
+    rp.max_q_len = a.max_q_len;
+    rp.scale_log2 = a.scale * 1.4426950408889634f;
+    rp.decode = decode ? 1 : 0;
+    if (decode) {
+        const DecodePlan pl = decode_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx);
+        rp.n_rg = pl.row_groups;
+        rp.split_pages = pl.split_pages;
+        if (pl.max_splits > 1) {
+            const size_t rows = static_cast<size_t>(pl.max_splits) * static_cast<size_t>(a.T) * a.H_q;
+            uint8_t *ws = static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES;
+            rp.ws_o = reinterpret_cast<float *>(ws);
+            rp.ws_lse = reinterpret_cast<float *>(ws + rows * D * sizeof(float));
+        }
+        if (a.B > 65535 || (int64_t)a.H_kv * pl.row_groups > 65535)
+            return PA_ERR_UNSUPPORTED;
+        dim3 grid(pl.max_splits, a.H_kv * pl.row_groups, a.B);
+        rc = launch_rows<D, BF16>(rp, tk, tv, grid, a.stream);
+        if (rc == PA_OK && pl.max_splits > 1)
+            rc = launch_merge<D, BF16>(rp, a.stream);
+        return rc;
+    }
+    const int G = a.H_q / a.H_kv;
+    rp.n_rg = static_cast<int>(((int64_t)a.max_q_len * G + kRowsPerCta - 1) / kRowsPerCta);
+    rp.split_pages = 1 << 30;
+    if (a.B > 65535 || a.H_kv > 65535)
+        return PA_ERR_UNSUPPORTED;
+    dim3 grid(rp.n_rg, a.H_kv, a.B);
+    return launch_rows<D, BF16>(rp, tk, tv, grid, a.stream);
+}
+
+static int dispatch(const AttnArgs &a, bool decode)
+{
+    if (a.d == 128)
+        return a.dtype == PA_BF16 ? run<128, true>(a, decode) : run<128, false>(a, decode);
+    return a.dtype == PA_BF16 ? run<64, true>(a, decode) : run<64, false>(a, decode);
+}
+
+int launch_decode(const AttnArgs &a) { return dispatch(a, true); }
+
+int launch_prefill(const AttnArgs &a) { return dispatch(a, false); }
+
+}  // namespace pa

@@ -1,0 +1,67 @@
+// Host-side internals of libpagedattn shared between translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/paged_attn.h"
+
+namespace pa {
+
+// Counts every kernel launch of the library (pa_launch_count).
+void count_launch(uint64_t n = 1);
+
+// True when p is non-null and 16-byte aligned.
+inline bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// 2-D tensor map over a paged cache [num_blocks][H_kv][16][d] viewed as
+// rows of d elements; box = 64 elements x 16 rows, 128-byte swizzle.
+// Returns PA_OK or PA_ERR_CUDA / PA_ERR_ARG.
+int make_cache_tmap(CUtensorMap *map, const void *cache, int64_t num_blocks, int H_kv, int d, pa_dtype dtype);
+
+// Reset the status word at the start of a workspace on `stream`.
+int reset_status(void *workspace, cudaStream_t stream);
+
+int sm_count();
+
+// ---- launchers (one per translation unit) --------------------------------------------
+
+struct AttnArgs {
+    void *out;
+    const void *q;
+    const void *key_cache;
+    const void *value_cache;
+    int64_t num_blocks;
+    const int32_t *block_tables;
+    int max_blocks;
+    const int32_t *cu_seqlens_q;
+    const int32_t *context_lens;
+    int B;
+    int max_q_len;
+    int max_ctx;
+    int64_t T;
+    int H_q;
+    int H_kv;
+    int d;
+    float scale;
+    pa_dtype dtype;
+    void *workspace;
+    size_t workspace_bytes;
+    cudaStream_t stream;
+};
+
+// Split-KV decode plan: pages per split and the number of splits.
+struct DecodePlan {
+    int split_pages;
+    int max_splits;
+    int row_groups;
+};
+DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx);
+size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx);
+
+int launch_decode(const AttnArgs &a);
+int launch_prefill(const AttnArgs &a);
+
+}  // namespace pa

@@ -1,0 +1,145 @@
+"""The C-ABI library on the CPU: it builds, loads, exports every declared entry
+point, and rejects bad arguments on the host before touching the device.
+
+Only host-side paths run here (no GPU): every call below returns from its
+argument checks before any CUDA runtime call.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_attention_34_b200 as pa
+from paged_kv_attention_34_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "paged_attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if _build.needs_build():
+        _build.build()
+    return pa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for n in ("pa_kv_cache_write", "pa_paged_attn_decode", "pa_paged_attn_prefill", "pa_kv_block_copy"):
+        assert n in names
+
+
+def test_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r"\bT (pa_[a-z_0-9]+)", out.stdout))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(L, n)
+
+
+def test_version_and_strerror(L):
+    assert L.pa_version() == 100
+    for code, name in pa.STATUS_NAMES.items():
+        assert pa.strerror(code) and pa.strerror(code) != "unknown status", name
+    assert pa.strerror(12345) == "unknown status"
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_write_rejects_bad_args(L):
+    f = L.pa_kv_cache_write
+    ok = dict(T=4, NB=8, H=2, d=128, dt=0)
+
+    def call(T=4, NB=8, H=2, d=128, dt=0, kn=_fake(), slot=_fake(), status=None):
+        return f(kn, _fake(), slot, T, _fake(), _fake(), NB, H, d, dt, status, None)
+
+    assert call(d=96) == -2
+    assert call(d=32) == -2
+    assert call(T=-1) == -1
+    assert call(NB=0) == -1
+    assert call(H=0) == -1
+    assert call(dt=7) == -1
+    assert call(kn=_fake(0x10008)) == -3  # not 16-byte aligned
+    assert call(slot=_fake(0x10002)) == -3
+    assert call(T=0) == 0  # nothing to do, nothing launched
+    del ok
+
+
+def test_block_copy_rejects_bad_args(L):
+    f = L.pa_kv_block_copy
+    assert f(_fake(), _fake(), 8, 2, 80, 0, _fake(), 3, None, None) == -2
+    assert f(_fake(), _fake(), 8, 2, 64, 0, _fake(), -1, None, None) == -1
+    assert f(_fake(0x10004), _fake(), 8, 2, 64, 0, _fake(), 3, None, None) == -3
+    assert f(_fake(), _fake(), 8, 2, 64, 0, _fake(), 0, None, None) == 0
+
+
+def _decode(L, *, B=2, T=2, H_q=8, H_kv=2, d=128, max_ctx=100, NB=16, ws=_fake(), wsb=1 << 20, q=_fake(),
+            scale=0.1, dt=1):
+    return L.pa_paged_attn_decode(_fake(), q, _fake(), _fake(), NB, _fake(), 8, _fake(), _fake(), B, max_ctx, T,
+                                  H_q, H_kv, d, scale, dt, ws, wsb, None)
+
+
+def test_decode_rejects_bad_args(L):
+    assert _decode(L, H_q=6, H_kv=4) == -2  # H_q % H_kv
+    assert _decode(L, d=96) == -2
+    assert _decode(L, B=-1) == -1
+    assert _decode(L, ws=None) == -4
+    assert _decode(L, wsb=16) == -4
+    assert _decode(L, ws=_fake(0x10008)) == -3
+    assert _decode(L, q=_fake(0x10001)) == -3
+    assert _decode(L, scale=float("nan")) == -1
+    assert _decode(L, NB=(1 << 31) // 32) == -2  # TMA row coordinate would overflow
+    assert _decode(L, dt=3) == -1
+
+
+def test_prefill_rejects_bad_args(L):
+    f = L.pa_paged_attn_prefill
+
+    def call(max_q_len=16, H_q=4, H_kv=4, d=64, wsb=256):
+        return f(_fake(), _fake(), _fake(), _fake(), 4, _fake(), 4, _fake(), _fake(), 1, max_q_len, 64, 16, H_q,
+                 H_kv, d, 0.1, 0, _fake(), wsb, None)
+
+    assert call(max_q_len=0) == -1
+    assert call(H_q=5, H_kv=2) == -2
+    assert call(d=256) == -2
+    assert call(wsb=8) == -4
+
+
+def test_workspace_queries(L):
+    # one split needs only the status word; long contexts need partials
+    small = pa.decode_workspace_bytes(3, 3, 4, 4, 64, 50)
+    assert small == pa.PA_STATUS_BYTES
+    big = pa.decode_workspace_bytes(16, 16, 64, 8, 128, 32768)
+    assert big > pa.PA_STATUS_BYTES
+    # monotone in T and max_ctx
+    assert pa.decode_workspace_bytes(32, 16, 64, 8, 128, 32768) >= big
+    assert pa.decode_workspace_bytes(16, 16, 64, 8, 128, 65536) >= big
+    assert L.pa_decode_workspace_bytes(1, 1, 6, 4, 128, 10) == 0  # invalid GQA ratio
+    assert pa.prefill_workspace_bytes(8, 40, 40, 128, 2048) >= pa.PA_STATUS_BYTES
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+
+    q = torch.zeros((1, 1, 64), dtype=torch.float16)
+    with pytest.raises(ValueError, match="CUDA"):
+        pa.paged_attn_decode(q, q.view(1, 1, 1, 64), q.view(1, 1, 1, 64), torch.zeros((1, 1), dtype=torch.int32),
+                             torch.zeros(2, dtype=torch.int32), torch.ones(1, dtype=torch.int32), 1, 0.1)
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(pa, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(pa, "_lib", None)
+    with pytest.raises(ImportError, match="no fallback"):
+        pa.lib()

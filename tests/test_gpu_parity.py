@@ -1,0 +1,228 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Tolerances (max-abs error against fp64, N(0,1) inputs): 3e-3 for fp16
+outputs, 1.6e-2 for bf16 outputs.  Cache writes and block copies must match
+the oracle's caches byte for byte.  Caches are filled with NaN outside every
+sequence's context, so any read past a context end shows up as a NaN.
+
+Small seeded cases are checked on every output row; the five full-size
+configurations are checked on sampled rows (all rows of the shortest and the
+longest sequence of each call, plus random rows), in the same launch
+configuration the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_attention_34_b200 as pa
+from oracle_pins import oracle_step
+from paged_kv_attention_34_b200 import workloads as W
+from paged_kv_attention_34_b200.step import DeviceStep
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.float16: 3e-3, torch.bfloat16: 1.6e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    pa.lib()
+
+
+def _u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def sample_rows(w: W.Workload, n_random: int, seed: int = 0) -> np.ndarray:
+    rows = set()
+    cu = w.cu_seqlens_q.tolist()
+    for c in w.calls:
+        seqs = list(range(c.seq_lo, c.seq_hi))
+        by_ctx = sorted(seqs, key=lambda b: w.ctx_lens[b])
+        for b in {by_ctx[0], by_ctx[-1]}:
+            toks = range(cu[b], cu[b + 1])
+            if len(toks) > 64:  # long prompts: first, last and a spread of tokens
+                toks = sorted(set(list(toks[:4]) + list(toks[-4:]) + list(toks[:: max(1, len(toks) // 16)])))
+            for t in toks:
+                for h in range(w.H_q):
+                    rows.add(t * w.H_q + h)
+    g = np.random.default_rng(seed)
+    rows.update(g.integers(0, w.T * w.H_q, size=n_random).tolist())
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def run_and_compare(w: W.Workload, rows=None, check_cache=True):
+    st = DeviceStep(w)
+    out = st.run()
+    torch.cuda.synchronize()
+    assert st.statuses() == [0] * (1 + len(st.calls)), st.statuses()
+    ref, kc_ref, vc_ref = oracle_step(w, oracle.lib(), rows=rows)
+    if check_cache:
+        # bit-exact caches (compared on the device to keep host memory small)
+        dev = st.key_cache.device
+        assert torch.equal(st.key_cache.view(torch.int16), torch.from_numpy(kc_ref.view(np.int16)).to(dev))
+        assert torch.equal(st.value_cache.view(torch.int16), torch.from_numpy(vc_ref.view(np.int16)).to(dev))
+    got = out.double().cpu().numpy().reshape(w.T * w.H_q, w.d)
+    if rows is not None:
+        got = got[rows]
+    else:
+        ref = ref.reshape(-1, w.d)
+    assert np.isfinite(got).all(), "non-finite output"
+    err = np.abs(got - ref).max()
+    assert err <= TOL[w.dtype], f"{w.name}: max abs err {err:.3e} > {TOL[w.dtype]}"
+    return err
+
+
+# ---- small seeded sweeps (every row) -----------------------------------------------------
+
+DECODE_CASES = [
+    # (B, q_max, ctx_max, H_kv, G, d, dtype)
+    (5, 1, 300, 2, 1, 64, W.F16),
+    (5, 1, 700, 3, 1, 128, W.F16),
+    (4, 4, 500, 2, 4, 128, W.BF16),
+    (3, 8, 900, 1, 8, 128, W.BF16),  # 64 rows per CTA
+    (3, 8, 400, 2, 8, 64, W.F16),
+    (2, 8, 300, 1, 16, 128, W.BF16),  # two row groups per KV head
+    (6, 6, 2000, 2, 4, 128, W.BF16),  # many splits, verify-like rows
+    (4, 3, 33, 2, 2, 64, W.BF16),     # tiny contexts, partial blocks
+]
+
+
+def _case_id(c):
+    return "B{}q{}c{}h{}g{}d{}{}".format(*c[:6], "bf16" if c[6] == W.BF16 else "f16")
+
+
+@pytest.mark.parametrize("idx", range(len(DECODE_CASES)), ids=lambda i: _case_id(DECODE_CASES[i]))
+@pytest.mark.parametrize("seed", [1, 2])
+def test_decode_small(idx, seed):
+    B, q_max, ctx_max, H_kv, G, d, dt = DECODE_CASES[idx]
+    w = W.random_workload(1000 * seed + 17 * idx, B=B, q_max=q_max, ctx_max=ctx_max, H_kv=H_kv, G=G, d=d,
+                          dtype=dt, kind="decode")
+    run_and_compare(w)
+
+
+PREFILL_CASES = [
+    (3, 200, 300, 2, 1, 128, W.BF16),
+    (2, 130, 260, 2, 4, 128, W.BF16),  # chunks with earlier context, GQA
+    (3, 90, 90, 2, 1, 64, W.F16),
+    (4, 17, 40, 1, 8, 128, W.F16),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(PREFILL_CASES)), ids=lambda i: _case_id(PREFILL_CASES[i]))
+def test_prefill_small(idx):
+    B, q_max, ctx_max, H_kv, G, d, dt = PREFILL_CASES[idx]
+    w = W.random_workload(77 + 31 * idx, B=B, q_max=q_max, ctx_max=ctx_max, H_kv=H_kv, G=G, d=d, dtype=dt,
+                          kind="prefill")
+    run_and_compare(w)
+
+
+def test_prefill_fresh_prompts_exact_lengths():
+    # prompts of 1, 15, 16, 17, 127, 128, 129 tokens with no earlier context
+    L = [1, 15, 16, 17, 127, 128, 129]
+    w = W.build_workload("fresh", q_lens=L, ctx_lens=L, H_q=4, H_kv=2, d=128, dtype=W.BF16, seed=9,
+                         calls=[W.AttnCall("prefill", 0, len(L))], pool_extra=5)
+    run_and_compare(w)
+
+
+# ---- the five configurations ----------------------------------------------------------------
+
+def test_config1_tiny_decode_all_rows():
+    run_and_compare(W.config1())
+
+
+def test_config2_13b_decode_sampled():
+    w = W.config2()
+    run_and_compare(w, rows=sample_rows(w, 512))
+
+
+def test_config3_prefill_sampled():
+    w = W.config3()
+    run_and_compare(w, rows=sample_rows(w, 512))
+
+
+def test_config4_gqa_shared_prefix_sampled():
+    w = W.config4()
+    run_and_compare(w, rows=sample_rows(w, 256))
+
+
+def test_config5_mixed_step_sampled():
+    w = W.config5()
+    run_and_compare(w, rows=sample_rows(w, 1024))
+
+
+# ---- edge cases and device-side error reporting -------------------------------------------------
+
+def test_empty_batch_launches_nothing():
+    dev = "cuda"
+    q = torch.empty((0, 4, 64), dtype=torch.float16, device=dev)
+    kc = torch.zeros((2, 4, 16, 64), dtype=torch.float16, device=dev)
+    n0 = pa.launch_count()
+    out = pa.paged_attn_decode(q, kc, kc, torch.zeros((0, 1), dtype=torch.int32, device=dev),
+                               torch.zeros(1, dtype=torch.int32, device=dev),
+                               torch.zeros(0, dtype=torch.int32, device=dev), 0, 0.125)
+    assert out.shape == (0, 4, 64) and pa.launch_count() == n0
+    assert pa.read_status(pa.paged_attn_decode.last_workspace) == 0
+
+
+def test_bad_block_id_is_reported_not_faulted():
+    w = W.random_workload(5, B=2, q_max=1, ctx_max=40, H_kv=2, G=1, d=64, dtype=W.F16, kind="decode")
+    w.block_tables[1, 0] = w.num_blocks + 3  # out of the pool
+    st = DeviceStep(w)
+    st.run()
+    torch.cuda.synchronize()
+    assert st.statuses()[1] == -7  # PA_ERR_BOUNDS
+    # sequence 0 is untouched by the bad entry and still exact
+    ref, _, _ = oracle_step(W.random_workload(5, B=2, q_max=1, ctx_max=40, H_kv=2, G=1, d=64, dtype=W.F16,
+                                              kind="decode"), oracle.lib())
+    got = st.out[:1].double().cpu().numpy()
+    assert np.abs(got - ref[:1]).max() <= TOL[torch.float16]
+
+
+def test_bad_slot_is_reported_and_skipped():
+    w = W.random_workload(6, B=2, q_max=2, ctx_max=30, H_kv=2, G=1, d=64, dtype=W.F16, kind="decode")
+    st = DeviceStep(w)
+    before = st.key_cache.clone()
+    bad = st.slot_mapping.clone()
+    bad[:] = -1
+    bad[0] = w.num_blocks * 16 + 5
+    pa.kv_cache_write(st.k_new, st.v_new, bad, st.key_cache, st.value_cache, status=st.status)
+    assert pa.read_status(st.status) == -7
+    assert torch.equal(before.view(torch.int16), st.key_cache.view(torch.int16))
+
+
+def test_inconsistent_sequence_is_reported():
+    w = W.random_workload(7, B=3, q_max=2, ctx_max=30, H_kv=1, G=2, d=128, dtype=W.BF16, kind="decode")
+    st = DeviceStep(w)
+    st.calls[0].ctx[1] = 0  # ctx < q_len
+    st.run()
+    torch.cuda.synchronize()
+    assert st.statuses()[1] == -8  # PA_ERR_SEQ
+
+
+def test_block_copy_bitexact_random():
+    g = torch.Generator().manual_seed(3)
+    NB, H, d = 40, 4, 128
+    kc = torch.randn((NB, H, 16, d), generator=g).bfloat16()
+    vc = torch.randn((NB, H, 16, d), generator=g).bfloat16()
+    pairs = torch.tensor([[3, 10], [3, 11], [17, 2], [39, 0]], dtype=torch.int32)
+    k16, v16 = _u16(kc).copy(), _u16(vc).copy()
+    assert oracle.kv_block_copy(k16, v16, pairs) == 0
+    kd, vd = kc.cuda(), vc.cuda()
+    pa.kv_block_copy(kd, vd, pairs.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(_u16(kd), k16) and np.array_equal(_u16(vd), v16)
+
+
+def test_repeat_runs_identical():
+    w = W.random_workload(8, B=4, q_max=3, ctx_max=600, H_kv=2, G=4, d=128, dtype=W.BF16, kind="decode")
+    st = DeviceStep(w)
+    a = st.run().clone()
+    b = st.run().clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
