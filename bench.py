@@ -248,7 +248,7 @@ def run_ours(args):
     stream = torch.cuda.Stream(device=device)
 
     # ---- headline: 13B-shaped decode step ----
-    w = W.config2(seed=shard_seed(34_002, rank))
+    w = W.config2(seed=shard_seed(34_002, rank), B=args.batch)
     with torch.cuda.stream(stream):
         st = DeviceStep(w, device=device)
     call = st.calls[0]
@@ -294,12 +294,12 @@ def run_ours(args):
         "dtype": "f16",
         "data": "synthetic: seeded N(0,1) fp16 Q/K/V, uniform context lengths, shuffled 16-token blocks (no dataset)",
         "config": {
-            "workload": HEADLINE,
-            "global_batch": 64 * world,
+            "workload": HEADLINE if args.batch == 64 else HEADLINE.replace("B 64", f"B {args.batch}"),
+            "global_batch": args.batch * world,
             "seq_len": "context U[128,4096] (sum %d per rank 0)" % sum(w.ctx_lens),
             "parallelism": f"dp{world} (independent sequences per rank, no data-path collective)",
-            "step": "kv_cache_write(64 new tokens) + paged_attn_decode (split kernel + merge)",
-            "l2": "no flush: the KV read per step (2.8 GB) is larger than the 126 MB L2",
+            "step": f"kv_cache_write({args.batch} new tokens) + paged_attn_decode (split kernel + merge)",
+            "l2": "no flush: the KV read per step (%.2f GB) is larger than the 126 MB L2" % (attn_bytes(w) / 1e9),
         },
         "roofline": {
             "kernel": "paged_attn_decode (split-KV kernel + LSE merge kernel, timed together)",
@@ -542,6 +542,8 @@ def main(argv=None):
     ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
+    ap.add_argument("--batch", type=int, default=64,
+                    help="sequences of the headline decode workload (64 = the 13B-shaped layer; smaller for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
