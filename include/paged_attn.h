@@ -63,7 +63,8 @@ typedef enum {
     PA_ERR_CUDA = -5,        /* a CUDA runtime call failed (launch, attribute, driver entry point) */
     PA_ERR_TIMEOUT = -6,     /* device: a bounded wait on an asynchronous copy ran out */
     PA_ERR_BOUNDS = -7,      /* device: a block id, slot or length was out of range; item skipped */
-    PA_ERR_SEQ = -8          /* device: cu_seqlens_q / context_lens inconsistent (q_b < 1, ctx_b < q_b, ...) */
+    PA_ERR_SEQ = -8,         /* device: cu_seqlens_q / context_lens inconsistent (q_b < 1, ctx_b < q_b, ...) */
+    PA_ERR_TOO_LARGE = -9    /* pa_paged_attn_decode_noalloc: the sizes need more than its fixed scratch */
 } pa_status;
 
 /* Size of the device status word area at the start of every workspace, bytes. */
@@ -129,6 +130,36 @@ int pa_paged_attn_decode(void *out, const void *q, const void *key_cache, const 
                          const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int max_ctx, int64_t T,
                          int H_q, int H_kv, int d, float scale, pa_dtype dtype, void *workspace,
                          size_t workspace_bytes, void *stream);
+
+/*
+ * pa_paged_attn_decode_noalloc -- pa_paged_attn_decode without a caller workspace.
+ * The pages have no counterpart: this is an interface for callers that may not
+ * allocate device memory when they call, such as plugins inside an engine that
+ * owns all device memory and forbids allocation while work is enqueued, or
+ * latency-critical code that cannot take cudaMalloc's implicit synchronisation
+ * or a possible allocation failure mid-step.  Same arguments and results as
+ * pa_paged_attn_decode, except:
+ *   - the scratch (status word + split partials) is a fixed array of
+ *     PA_DECODE_NOALLOC_SCRATCH_BYTES inside the library; every GPU that loads
+ *     it holds that memory until the process exits;
+ *   - sizes whose pa_decode_workspace_bytes(...) exceeds that maximum are
+ *     rejected with PA_ERR_TOO_LARGE before anything is launched;
+ *   - the first call on each device (with that device current) looks up the
+ *     array's device address (cudaGetSymbolAddress) and keeps it: make that
+ *     first call before any stream capture;
+ *   - all calls on a device share the array and it keeps the last call's
+ *     contents; the status word is cleared on `stream` before each launch.
+ *     Calls that overlap on the GPU (different streams without ordering) race;
+ *   - status: optional device int32 (may be NULL) that receives the call's
+ *     device status word (copied on `stream` after the kernels).
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES (32u << 20)
+int pa_paged_attn_decode_noalloc(void *out, const void *q, const void *key_cache, const void *value_cache,
+                                 int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
+                                 const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int max_ctx,
+                                 int64_t T, int H_q, int H_kv, int d, float scale, pa_dtype dtype, int32_t *status,
+                                 void *stream);
 
 /*
  * pa_prefill_workspace_bytes -- device workspace of pa_paged_attn_prefill

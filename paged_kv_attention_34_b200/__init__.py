@@ -37,6 +37,7 @@ STATUS_NAMES = {
     -6: "PA_ERR_TIMEOUT",
     -7: "PA_ERR_BOUNDS",
     -8: "PA_ERR_SEQ",
+    -9: "PA_ERR_TOO_LARGE",
 }
 
 _lib = None

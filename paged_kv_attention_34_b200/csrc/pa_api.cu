@@ -179,6 +179,7 @@ extern "C" const char *pa_strerror(int code)
     case PA_ERR_TIMEOUT: return "device wait on an asynchronous copy timed out";
     case PA_ERR_BOUNDS: return "block id, slot or length out of range (item skipped)";
     case PA_ERR_SEQ: return "inconsistent cu_seqlens_q / context_lens (sequence skipped)";
+    case PA_ERR_TOO_LARGE: return "sizes need more scratch than the allocation-free decode entry point holds";
     default: return "unknown status";
     }
 }
