@@ -625,6 +625,4 @@ static int dispatch(const AttnArgs &a, bool decode)
 
 int launch_decode(const AttnArgs &a) { return dispatch(a, true); }
 
-int launch_prefill(const AttnArgs &a) { return dispatch(a, false); }
-
 }  // namespace pa

@@ -62,6 +62,24 @@ int make_cache_tmap(CUtensorMap *map, const void *cache, int64_t num_blocks, int
     return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+int make_q_tmap(CUtensorMap *map, const void *q, int64_t T, int H_q, int d, int G, int tok, pa_dtype dtype)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return PA_ERR_CUDA;
+    if (G < 1 || G > 256 || tok < 1 || tok > 256)
+        return PA_ERR_UNSUPPORTED;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H_q), static_cast<cuuint64_t>(T)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H_q) * d * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(tok)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                    const_cast<void *>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
 int reset_status(void *workspace, cudaStream_t stream)
 {
     return cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream) == cudaSuccess ? PA_OK : PA_ERR_CUDA;

@@ -21,6 +21,10 @@ inline bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p
 // Returns PA_OK or PA_ERR_CUDA / PA_ERR_ARG.
 int make_cache_tmap(CUtensorMap *map, const void *cache, int64_t num_blocks, int H_kv, int d, pa_dtype dtype);
 
+// 3-D tensor map over Q [T][H_q][d] for query tiles of `tok` tokens x G heads of one
+// KV head: dims (d, H_q, T), box (64, G, tok), 128-byte swizzle.
+int make_q_tmap(CUtensorMap *map, const void *q, int64_t T, int H_q, int d, int G, int tok, pa_dtype dtype);
+
 // Reset the status word at the start of a workspace on `stream`.
 int reset_status(void *workspace, cudaStream_t stream);
 
