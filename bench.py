@@ -533,6 +533,28 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def run_one_leg(args):
+    """One leg alone on cuda:LOCAL_RANK (for profiling); prints the leg's JSON object."""
+    import torch
+
+    import paged_kv_attention_34_b200 as pa
+
+    _, local_rank, _ = dist_env()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    pa.lib()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.Stream(device=device)
+    hbm, bf16 = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"])
+    if args.only == "prefill":
+        res = leg_prefill(args, stream, device, bf16, peak_src, 0)
+    elif args.only == "gqa":
+        res = leg_gqa(args, stream, device, hbm, 0)
+    else:
+        res = leg_mixed(args, stream, device, hbm, bf16, 0)
+    print(json.dumps({"leg": args.only, **res}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -542,6 +564,8 @@ def main(argv=None):
     ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
+    ap.add_argument("--only", choices=["prefill", "gqa", "mixed"], default=None,
+                    help="run one leg alone and print its JSON object (profiling runs)")
     ap.add_argument("--batch", type=int, default=64,
                     help="sequences of the headline decode workload (64 = the 13B-shaped layer; smaller for profiling)")
     args = ap.parse_args(argv)
@@ -549,6 +573,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_one_leg(args)
     else:
         run_ours(args)
 
