@@ -8,24 +8,31 @@
 // Q&A page); a chunk with earlier context sees it (chunked prefill).
 //
 // Tiling (the online softmax of iopencloud section 2.2, on Blackwell units):
-//   * a work item = (sequence, KV head, query tile).  A query tile holds
-//     128 rows = 128/G tokens x the G query heads of the KV head, so every K/V
-//     tile is shared by the whole GQA group;
+//   * a query tile holds 128 rows = 128/G tokens x the G query heads of one KV
+//     head, so every K/V tile is shared by the whole GQA group.  A work item is
+//     a PAIR of consecutive query tiles (A, B) of one (sequence, KV head): both
+//     tiles read the same K/V tiles, and while one softmax warpgroup works on
+//     its scores the tensor core runs the other tile's products;
 //   * K/V tiles of 128 keys = 8 pages of 16 keys, each page fetched by TMA
-//     (64-element x 16-row boxes, 128-byte swizzle) straight from its block;
-//   * S = Q K^T: tcgen05.mma M=128 N=128, both operands in shared memory
-//     (K-major), fp32 accumulator in TMEM (two S buffers);
-//   * softmax: 4 warps, one thread per row (= TMEM lane) read S with
-//     tcgen05.ld, keep the running max m and sum l in registers, write
-//     P (16-bit) back over S in TMEM;
-//   * O += P V: tcgen05.mma with A = P from TMEM, B = V in shared memory
-//     (MN-major), fp32 accumulator in TMEM (two O buffers, one per item in
-//     flight).  O is rescaled only when a row's max grows by more than 2^8
-//     (exact: the same stale max is used for P and for l, and O / l is taken
-//     once at the end);
-//   * warp roles: warp 0 issues TMA (Q, K, V), warp 1 allocates TMEM and issues
-//     the MMAs, warps 2-5 run the softmax and the epilogue.  Persistent CTAs,
-//     one per SM, walk the items heaviest first (later query tiles see more keys).
+//     (64-element x 16-row boxes, 128-byte swizzle) straight from its block,
+//     on separate K and V rings;
+//   * S_X = Q_X K^T (X = A, B): tcgen05.mma M=128 N=128, K-major operands in
+//     shared memory, fp32 accumulator in TMEM;
+//   * softmax warpgroup X (one thread per row = TMEM lane) reads S_X with
+//     tcgen05.ld, keeps the running max m and sum l in registers and writes
+//     P_X (16-bit) back over S_X in TMEM;
+//   * O_X += P_X V: tcgen05.mma with A = P_X from TMEM and B = V (MN-major) in
+//     shared memory, fp32 accumulator in TMEM.  O_X is rescaled only when a
+//     row's max grows by more than 2^8 (exact: the same stale max is used for
+//     P and for l, and O / l is taken once at the end);
+//   * tensor-core issue order per K/V tile j: S_A(j), O_B += P_B(j-1) V(j-1),
+//     S_B(j), O_A += P_A(j) V(j).  Each S_X(j+1) is issued after the P_X(j) V
+//     product that reads the same TMEM columns; tcgen05.mma operations of one
+//     thread execute in issue order, which makes that reuse safe;
+//   * warp 0 issues TMA and hands out work items from a global counter,
+//     heaviest first (later query tiles see more keys); warp 1 allocates TMEM
+//     and issues the MMAs; warps 2-5 and 6-9 are the two softmax warpgroups
+//     (rescale and epilogue included).  One persistent CTA per SM.
 // All waits are bounded; a wait that runs out records PA_ERR_TIMEOUT and the
 // CTA winds down (its copies and MMAs in flight are waited for, TMEM freed).
 #include <cmath>
@@ -39,10 +46,13 @@ namespace tcp {
 
 constexpr int kRows = 128;     // query rows per tile (TMEM lanes)
 constexpr int kKeys = 128;     // keys per K/V tile
-constexpr int kStages = 2;     // K/V ring depth
-constexpr int kThreads = 192;  // 6 warps
+constexpr int kStages = 2;     // depth of the K ring and of the V ring
+constexpr int kThreads = 320;  // 10 warps
 constexpr int kMaxTable = 1024;
+constexpr int kItemSlots = 2;
+constexpr int kItemReaders = 9;  // warp 1 and warps 2-9 each acknowledge a work item
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr size_t kCounterOffset = 64;      // work counter inside the status area of the workspace
 
 struct Params {
     const int32_t *block_tables;
@@ -50,6 +60,7 @@ struct Params {
     const int32_t *context_lens;
     void *out;
     int32_t *status;
+    int *counter;
     int64_t num_blocks;
     int64_t T;
     int max_blocks;
@@ -57,36 +68,57 @@ struct Params {
     int max_q_len, max_ctx;
     int tok_per_tile;   // 128 / G (floor)
     int rows_per_tile;  // tok_per_tile * G
-    int n_qt_max;       // ceil(max_q_len / tok_per_tile)
-    int n_items;        // n_qt_max * B * H_kv
+    int n_pairs_max;    // ceil(ceil(max_q_len / tok_per_tile) / 2)
+    int n_items;        // n_pairs_max * B * H_kv
     int oob_row;        // first row past the pool in the cache tensor map
     float scale_log2;
 };
 
 template <int D>
 struct Smem {
-    static constexpr int kKB = D / 64;                 // 128-byte column blocks
-    static constexpr int kTile = kKB * kRows * 128;    // one 128-row x D tile (Q, K or V)
-    static constexpr int kQ = 0;                       // 2 Q buffers
-    static constexpr int kKV = 2 * kTile;              // kStages x (K tile, V tile)
-    static constexpr int kTable = kKV + kStages * 2 * kTile;
+    static constexpr int kKB = D / 64;               // 128-byte column blocks
+    static constexpr int kTile = kKB * kRows * 128;  // one 128-row x D tile
+    static constexpr int kQ = 0;                     // Q_A, Q_B
+    static constexpr int kK = 2 * kTile;             // K ring
+    static constexpr int kV = kK + kStages * kTile;  // V ring
+    static constexpr int kTable = kV + kStages * kTile;
     static constexpr int kBars = kTable + 4 * kMaxTable;
-    // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] s_free[2] p_full[2] o_full[2] o_free[2] drain
-    static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 1;
-    static constexpr int kTmemSlot = kBars + 8 * kNumBars;
+    static constexpr int kNumBars = 2 * 2 + 4 * kStages + 5 * 2 + 2 * kItemSlots + 1;
+    static constexpr int kItems = kBars + 8 * kNumBars;
+    static constexpr int kTmemSlot = kItems + 4 * kItemSlots;
     static constexpr int kAbort = kTmemSlot + 8;
     static constexpr int kBytes = kAbort + 8;
     static constexpr int kAlloc = kBytes + 1024;
 };
 
-struct Item {
-    int b, g, t_begin, n_tok, q0, qb, ctx, lim_hi, n_pages, n_kv;
+// One query tile of a work item.
+struct Tile {
+    bool on;      // the tile has at least one query token
+    int t_begin;  // first token (within the sequence) of the tile
+    int n_tok;    // tokens in the tile
+    int n_kv;     // K/V tiles it needs (causal)
 };
 
+struct Item {
+    int b, g, q0, qb, ctx;
+    Tile A, Bt;
+    int n_kv;     // K/V tiles of the item (= the larger of the two)
+    int n_pages;  // pages of the item
+};
+
+__device__ __forceinline__ void make_tile(const Params &p, const Item &I, int qt, Tile &t)
+{
+    t.t_begin = qt * p.tok_per_tile;
+    t.on = t.t_begin < I.qb;
+    t.n_tok = t.on ? min(p.tok_per_tile, I.qb - t.t_begin) : 0;
+    t.n_kv = t.on ? (I.ctx - I.qb + t.t_begin + t.n_tok - 1) / kKeys + 1 : 0;
+}
+
+// Decode work item `it`; false when it has no query token (or its sequence is invalid).
 __device__ __forceinline__ bool get_item(const Params &p, int it, Item &I, bool report)
 {
     const int per = p.B * p.H_kv;
-    const int qt = p.n_qt_max - 1 - it / per;
+    const int pair = p.n_pairs_max - 1 - it / per;  // heaviest first
     const int rem = it % per;
     I.b = rem / p.H_kv;
     I.g = rem % p.H_kv;
@@ -97,17 +129,17 @@ __device__ __forceinline__ bool get_item(const Params &p, int it, Item &I, bool 
     const bool ok = I.qb >= 1 && I.ctx >= I.qb && I.qb <= p.max_q_len && I.ctx <= p.max_ctx &&
                     I.ctx <= p.max_blocks * 16 && q1 <= p.T && I.q0 >= 0;
     if (!ok) {
-        if (report && qt == 0 && I.g == 0)
+        if (report && pair == 0 && I.g == 0)
             set_status(p.status, PA_ERR_SEQ);
         return false;
     }
-    I.t_begin = qt * p.tok_per_tile;
-    if (I.t_begin >= I.qb)
+    make_tile(p, I, 2 * pair, I.A);
+    make_tile(p, I, 2 * pair + 1, I.Bt);
+    if (!I.A.on)
         return false;
-    I.n_tok = min(p.tok_per_tile, I.qb - I.t_begin);
-    I.lim_hi = I.ctx - I.qb + I.t_begin + I.n_tok - 1;
-    I.n_pages = I.lim_hi / 16 + 1;
-    I.n_kv = I.lim_hi / kKeys + 1;
+    I.n_kv = max(I.A.n_kv, I.Bt.n_kv);
+    const int lim_hi = I.ctx - I.qb + (I.Bt.on ? I.Bt.t_begin + I.Bt.n_tok : I.A.t_begin + I.A.n_tok) - 1;
+    I.n_pages = lim_hi / 16 + 1;
     return true;
 }
 
@@ -132,6 +164,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     }
 }
 
+// Parity to wait for the k-th completion (0-based) of a barrier; and for the k-th
+// "slot is free again" wait on a barrier whose slot starts out free.
+__device__ __forceinline__ uint32_t full_par(int k) { return static_cast<uint32_t>(k & 1); }
+__device__ __forceinline__ uint32_t free_par(int k) { return static_cast<uint32_t>((k & 1) ^ 1); }
+
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     pa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
@@ -140,15 +177,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     using L = Smem<D>;
     constexpr int KB = L::kKB;
     constexpr uint32_t kTmemCols = 512;
-    constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + 128;
+    // TMEM columns: S_A, S_B (P written over their first 64 columns), O_A, O_B
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBars);
-    uint64_t *q_full = bars, *q_empty = bars + 2;
-    uint64_t *kv_full = bars + 4, *kv_empty = bars + 4 + kStages;
-    uint64_t *s_full = bars + 4 + 2 * kStages, *s_free = s_full + 2, *p_full = s_full + 4;
-    uint64_t *o_full = s_full + 6, *o_free = s_full + 8, *drain = s_full + 10;
+    uint64_t *q_full = bars;                    // [2] Q_X landed
+    uint64_t *q_empty = bars + 2;               // [2] Q_X no longer read
+    uint64_t *k_full = bars + 4;                // [kStages]
+    uint64_t *k_empty = k_full + kStages;       // [kStages]
+    uint64_t *v_full = k_empty + kStages;       // [kStages]
+    uint64_t *v_empty = v_full + kStages;       // [kStages]
+    uint64_t *s_full = v_empty + kStages;       // [2] S_X computed
+    uint64_t *p_full = s_full + 2;              // [2] P_X written (128 arrivals)
+    uint64_t *pv_done = p_full + 2;             // [2] O_X += P_X V completed
+    uint64_t *o_full = pv_done + 2;             // [2] O_X final for the item
+    uint64_t *o_free = o_full + 2;              // [2] epilogue of X has read O_X (128 arrivals)
+    uint64_t *item_full = o_free + 2;           // [kItemSlots]
+    uint64_t *item_empty = item_full + kItemSlots;
+    uint64_t *drain = item_empty + kItemSlots;  // [1]
+    int *item_slot = reinterpret_cast<int *>(smem + L::kItems);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kAbort);
     int32_t *s_table = reinterpret_cast<int32_t *>(smem + L::kTable);
@@ -156,18 +204,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&q_full[i], 1);
-            mbar_init(&q_empty[i], 1);
-            mbar_init(&s_full[i], 1);
-            mbar_init(&s_free[i], 1);
-            mbar_init(&p_full[i], 128);
-            mbar_init(&o_full[i], 1);
-            mbar_init(&o_free[i], 128);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&q_full[x], 1);
+            mbar_init(&q_empty[x], 1);
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 128);
+            mbar_init(&pv_done[x], 1);
+            mbar_init(&o_full[x], 1);
+            mbar_init(&o_free[x], 128);
         }
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&kv_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+        }
+        for (int i = 0; i < kItemSlots; ++i) {
+            mbar_init(&item_full[i], 1);
+            mbar_init(&item_empty[i], kItemReaders);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -184,15 +238,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // TMEM columns of tile X: S_X at 128 X, O_X at 256 + 128 X
 
     if (warp == 0) {
-        // ===================== TMA producer =====================
-        int kv_n = 0, n_it = 0, kv_issued = 0;
+        // ===================== scheduler + TMA producer =====================
+        int n_pub = 0, k_n = 0, v_n = 0, q_n[2] = {0, 0};
         bool ok = true;
-        for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+        for (;;) {
+            // next work item that has query tokens (lane 0 draws, the warp follows)
+            int it = -1;
             Item I;
-            if (!get_item(p, it, I, lane == 0))
-                continue;
+            for (;;) {
+                // lane 0 decides for the whole warp (the abort flag may change between lanes' reads)
+                int cand = -1;
+                if (lane == 0 && ok && !*abort_flag)
+                    cand = atomicAdd(p.counter, 1);
+                cand = __shfl_sync(0xffffffffu, cand, 0);
+                if (cand < 0 || cand >= p.n_items)
+                    break;
+                if (get_item(p, cand, I, lane == 0)) {
+                    it = cand;
+                    break;
+                }
+            }
+            // publish it (or the end marker -1) to the other roles
+            if (lane == 0) {
+                const int slot = n_pub % kItemSlots;
+                const bool got = wait_bar(&item_empty[slot], free_par(n_pub / kItemSlots), abort_flag, p.status);
+                ok = ok && got;
+                item_slot[slot] = ok ? it : -1;
+                mbar_arrive(&item_full[slot]);
+            }
+            ++n_pub;
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (it < 0 || !ok)
+                break;
+            // page ids of the item into shared memory
             const int32_t *table = p.block_tables + (int64_t)I.b * p.max_blocks;
             for (int i = lane; i < min(I.n_pages, kMaxTable); i += 32) {
                 int pg = __ldg(table + i);
@@ -204,169 +285,273 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncwarp();
             if (lane == 0) {
-                const int qbuf = n_it & 1;
-                ok = wait_bar(&q_empty[qbuf], ((n_it >> 1) & 1) ^ 1, abort_flag, p.status);
-                if (ok) {
-                    uint8_t *qs = smem + L::kQ + qbuf * L::kTile;
-                    mbar_arrive_expect_tx(&q_full[qbuf], KB * p.rows_per_tile * 128);
-                    for (int kb = 0; kb < KB; ++kb)
-                        tc::tma_load_3d(qs + kb * kRows * 128, &tmap_q, kb * 64, I.g * p.G, I.q0 + I.t_begin,
-                                        &q_full[qbuf]);
-                }
-                for (int j = 0; j < I.n_kv && ok; ++j) {
-                    const int n = kv_n + j, s = n % kStages;
-                    ok = wait_bar(&kv_empty[s], ((n / kStages) & 1) ^ 1, abort_flag, p.status);
+                // Q tiles
+                const Tile *tl[2] = {&I.A, &I.Bt};
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (!ok || !tl[x]->on)
+                        continue;
+                    ok = wait_bar(&q_empty[x], free_par(q_n[x]), abort_flag, p.status);
                     if (!ok)
                         break;
-                    uint8_t *ks = smem + L::kKV + s * 2 * L::kTile;
-                    uint8_t *vs = ks + L::kTile;
-                    mbar_arrive_expect_tx(&kv_full[s], 2 * L::kTile);
-                    ++kv_issued;
+                    uint8_t *qs = smem + L::kQ + x * L::kTile;
+                    mbar_arrive_expect_tx(&q_full[x], KB * p.rows_per_tile * 128);
+                    for (int kb = 0; kb < KB; ++kb)
+                        tc::tma_load_3d(qs + kb * kRows * 128, &tmap_q, kb * 64, I.g * p.G, I.q0 + tl[x]->t_begin,
+                                        &q_full[x]);
+                    ++q_n[x];
+                }
+                // K and V tiles, interleaved
+                for (int j = 0; j < I.n_kv && ok; ++j) {
+                    int y[8];
+#pragma unroll
                     for (int pg = 0; pg < 8; ++pg) {
                         const int pidx = j * 8 + pg;
-                        int y = p.oob_row;  // pages past this item's range: zero-filled by TMA
+                        y[pg] = p.oob_row;  // pages past the item's range: zero-filled by TMA
                         if (pidx < I.n_pages) {
                             int id = pidx < kMaxTable ? s_table[pidx] : __ldg(table + pidx);
-                            if (id < 0 || id >= p.num_blocks) {
-                                set_status(p.status, PA_ERR_BOUNDS);
+                            if (id >= p.num_blocks)
                                 id = -1;
-                            }
                             if (id >= 0)
-                                y = (id * p.H_kv + I.g) * 16;
-                        }
-#pragma unroll
-                        for (int kb = 0; kb < KB; ++kb) {
-                            tma_load_2d(ks + kb * kRows * 128 + pg * 2048, &tmap_k, kb * 64, y, &kv_full[s]);
-                            tma_load_2d(vs + kb * kRows * 128 + pg * 2048, &tmap_v, kb * 64, y, &kv_full[s]);
+                                y[pg] = (id * p.H_kv + I.g) * 16;
+                            else
+                                set_status(p.status, PA_ERR_BOUNDS);
                         }
                     }
+                    const int ks = k_n % kStages;
+                    ok = wait_bar(&k_empty[ks], free_par(k_n / kStages), abort_flag, p.status);
+                    if (!ok)
+                        break;
+                    uint8_t *kdst = smem + L::kK + ks * L::kTile;
+                    mbar_arrive_expect_tx(&k_full[ks], L::kTile);
+                    ++k_n;
+#pragma unroll
+                    for (int pg = 0; pg < 8; ++pg)
+#pragma unroll
+                        for (int kb = 0; kb < KB; ++kb)
+                            tma_load_2d(kdst + kb * kRows * 128 + pg * 2048, &tmap_k, kb * 64, y[pg], &k_full[ks]);
+                    const int vs = v_n % kStages;
+                    ok = wait_bar(&v_empty[vs], free_par(v_n / kStages), abort_flag, p.status);
+                    if (!ok)
+                        break;
+                    uint8_t *vdst = smem + L::kV + vs * L::kTile;
+                    mbar_arrive_expect_tx(&v_full[vs], L::kTile);
+                    ++v_n;
+#pragma unroll
+                    for (int pg = 0; pg < 8; ++pg)
+#pragma unroll
+                        for (int kb = 0; kb < KB; ++kb)
+                            tma_load_2d(vdst + kb * kRows * 128 + pg * 2048, &tmap_v, kb * 64, y[pg], &v_full[vs]);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            kv_issued = __shfl_sync(0xffffffffu, kv_issued, 0);
+            k_n = __shfl_sync(0xffffffffu, k_n, 0);
+            v_n = __shfl_sync(0xffffffffu, v_n, 0);
+            q_n[0] = __shfl_sync(0xffffffffu, q_n[0], 0);
+            q_n[1] = __shfl_sync(0xffffffffu, q_n[1], 0);
             __syncwarp();
-            kv_n += I.n_kv;
-            ++n_it;
         }
         if (lane == 0 && *abort_flag) {
-            // let the copies already issued land before shared memory is released: the
-            // last arming of stage s was its ((issued_s - 1))-th use
+            // let the copies already issued land before shared memory is released
             for (int s = 0; s < kStages; ++s) {
-                const int issued_s = kv_issued / kStages + (s < kv_issued % kStages ? 1 : 0);
-                if (issued_s > 0)
-                    mbar_wait(&kv_full[s], (issued_s - 1) & 1, kWaitTimeoutNs / 10);
+                const int k_uses = k_n / kStages + (s < k_n % kStages ? 1 : 0);
+                const int v_uses = v_n / kStages + (s < v_n % kStages ? 1 : 0);
+                if (k_uses > 0)
+                    mbar_wait(&k_full[s], full_par(k_uses - 1), kWaitTimeoutNs / 10);
+                if (v_uses > 0)
+                    mbar_wait(&v_full[s], full_par(v_uses - 1), kWaitTimeoutNs / 10);
             }
         }
     } else if (warp == 1) {
         // ===================== MMA issuer =====================
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = tc::idesc_f16(BF16, kRows, kKeys, false);
-            constexpr uint32_t idesc_pv = tc::idesc_f16(BF16, kRows, D, true);
-            int kv_n = 0, n_it = 0;
-            bool ok = true;
-            for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
-                Item I;
-                if (!get_item(p, it, I, false))
-                    continue;
-                const int qbuf = n_it & 1, ob = n_it & 1;
-                const uint32_t o_tmem = tmem + (ob ? kColO1 : kColO0);
-                ok = wait_bar(&q_full[qbuf], (n_it >> 1) & 1, abort_flag, p.status);
-                const uint32_t q_addr = smem_u32(smem + L::kQ + qbuf * L::kTile);
-                for (int j = 0; j <= I.n_kv && ok; ++j) {
-                    if (j < I.n_kv) {
-                        const int n = kv_n + j, s = n % kStages, sb = n & 1;
-                        ok = wait_bar(&kv_full[s], (n / kStages) & 1, abort_flag, p.status) &&
-                             wait_bar(&s_free[sb], ((n >> 1) & 1) ^ 1, abort_flag, p.status);
+        constexpr uint32_t idesc_qk = tc::idesc_f16(BF16, kRows, kKeys, false);
+        constexpr uint32_t idesc_pv = tc::idesc_f16(BF16, kRows, D, true);
+        int n_item = 0, k_n = 0, v_n = 0, q_n[2] = {0, 0}, pv_n[2] = {0, 0}, o_n[2] = {0, 0};
+        bool ok = true;
+        for (;;) {
+            const int slot = n_item % kItemSlots;
+            ok = wait_bar(&item_full[slot], full_par(n_item / kItemSlots), abort_flag, p.status);
+            ok = __all_sync(0xffffffffu, ok);
+            const int it = ok ? item_slot[slot] : -1;
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&item_empty[slot]);
+            ++n_item;
+            if (it < 0)
+                break;
+            Item I;
+            get_item(p, it, I, false);
+            if (lane == 0) {
+                const Tile *tl[2] = {&I.A, &I.Bt};
+                uint32_t q_addr[2];
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+                    q_addr[x] = smem_u32(smem + L::kQ + x * L::kTile);
+#pragma unroll
+                for (int x = 0; x < 2; ++x)
+                    if (ok && tl[x]->on) {
+                        ok = wait_bar(&q_full[x], full_par(q_n[x]), abort_flag, p.status);
+                        ++q_n[x];
+                    }
+                // S_X(j) = Q_X K_j^T
+                auto qk = [&](int x, int j, int kstage) {
+                    const uint32_t k_addr = smem_u32(smem + L::kK + kstage * L::kTile);
+                    const uint32_t d = tmem + 128u * x;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
+                        tc::mma_ss(d, tc::desc_k_sw128(q_addr[x] + off), tc::desc_k_sw128(k_addr + off), idesc_qk,
+                                   ks > 0 ? 1u : 0u);
+                    }
+                    tc::commit(&s_full[x]);
+                    if (j == tl[x]->n_kv - 1)
+                        tc::commit(&q_empty[x]);  // Q_X no longer needed
+                };
+                // O_X += P_X(j) V_j (waits for P_X(j); on the first tile also for the last epilogue of X)
+                auto pv = [&](int x, int j, int vstage) -> bool {
+                    if (!wait_bar(&p_full[x], full_par(pv_n[x]), abort_flag, p.status))
+                        return false;
+                    if (j == 0 && !wait_bar(&o_free[x], free_par(o_n[x]), abort_flag, p.status))
+                        return false;
+                    tc::fence_after_sync();
+                    const uint32_t v_addr = smem_u32(smem + L::kV + vstage * L::kTile);
+                    const uint32_t d = tmem + 256u + 128u * x;
+                    const uint32_t a = tmem + 128u * x;
+#pragma unroll
+                    for (int ks = 0; ks < kKeys / 16; ++ks)
+                        tc::mma_ts(d, a + ks * 8, tc::desc_mn_sw128(v_addr + ks * 2048, kRows * 128), idesc_pv,
+                                   (j > 0 || ks > 0) ? 1u : 0u);
+                    tc::commit(&pv_done[x]);
+                    ++pv_n[x];
+                    if (j == tl[x]->n_kv - 1) {
+                        tc::commit(&o_full[x]);
+                        ++o_n[x];
+                    }
+                    return true;
+                };
+                const int n = I.n_kv;
+                int vst_prev = 0;
+                for (int j = 0; j <= n && ok; ++j) {
+                    int kst = 0, vst = 0;
+                    if (j < n) {
+                        kst = k_n % kStages;
+                        ok = wait_bar(&k_full[kst], full_par(k_n / kStages), abort_flag, p.status);
+                        ++k_n;
                         if (!ok)
                             break;
                         tc::fence_after_sync();
-                        const uint32_t k_addr = smem_u32(smem + L::kKV + s * 2 * L::kTile);
-                        const uint32_t s_tmem = tmem + (sb ? kColS1 : kColS0);
-#pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint32_t off = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
-                            tc::mma_ss(s_tmem, tc::desc_k_sw128(q_addr + off), tc::desc_k_sw128(k_addr + off),
-                                       idesc_qk, ks > 0 ? 1u : 0u);
-                        }
-                        tc::commit(&s_full[sb]);
-                        if (j == I.n_kv - 1)
-                            tc::commit(&q_empty[qbuf]);
+                        if (j < I.A.n_kv)
+                            qk(0, j, kst);
                     }
                     if (j >= 1) {
-                        const int n = kv_n + j - 1, s = n % kStages, sb = n & 1;
-                        ok = wait_bar(&p_full[sb], (n >> 1) & 1, abort_flag, p.status);
-                        if (ok && j == 1)
-                            ok = wait_bar(&o_free[ob], ((n_it >> 1) & 1) ^ 1, abort_flag, p.status);
+                        // O_B += P_B(j-1) V(j-1); after it the V tile j-1 is free
+                        if (j - 1 < I.Bt.n_kv) {
+                            ok = pv(1, j - 1, vst_prev);
+                            if (!ok)
+                                break;
+                        }
+                        tc::commit(&v_empty[vst_prev]);
+                    }
+                    if (j < n) {
+                        if (j < I.Bt.n_kv)
+                            qk(1, j, kst);
+                        tc::commit(&k_empty[kst]);
+                        vst = v_n % kStages;
+                        ok = wait_bar(&v_full[vst], full_par(v_n / kStages), abort_flag, p.status);
+                        ++v_n;
                         if (!ok)
                             break;
-                        tc::fence_after_sync();
-                        const uint32_t v_addr = smem_u32(smem + L::kKV + s * 2 * L::kTile + L::kTile);
-                        const uint32_t p_tmem = tmem + (sb ? kColS1 : kColS0);
-#pragma unroll
-                        for (int ks = 0; ks < kKeys / 16; ++ks)
-                            tc::mma_ts(o_tmem, p_tmem + ks * 8, tc::desc_mn_sw128(v_addr + ks * 2048, kRows * 128),
-                                       idesc_pv, (j > 1 || ks > 0) ? 1u : 0u);
-                        tc::commit(&kv_empty[s]);
-                        tc::commit(&s_free[sb]);
-                        if (j == I.n_kv)
-                            tc::commit(&o_full[ob]);
+                        if (j < I.A.n_kv) {
+                            ok = pv(0, j, vst);
+                            if (!ok)
+                                break;
+                        }
                     }
+                    vst_prev = vst;
                 }
-                kv_n += I.n_kv;
-                ++n_it;
             }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            k_n = __shfl_sync(0xffffffffu, k_n, 0);
+            v_n = __shfl_sync(0xffffffffu, v_n, 0);
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                q_n[x] = __shfl_sync(0xffffffffu, q_n[x], 0);
+                pv_n[x] = __shfl_sync(0xffffffffu, pv_n[x], 0);
+                o_n[x] = __shfl_sync(0xffffffffu, o_n[x], 0);
+            }
+            if (!ok)
+                break;
+        }
+        if (lane == 0) {
             // every MMA issued so far must be complete before TMEM is released
             tc::commit(drain);
             mbar_wait(drain, 0, kWaitTimeoutNs / 10);
         }
         __syncwarp();
     } else {
-        // ===================== softmax + epilogue (warps 2-5) =====================
-        const int sub = warp & 3;        // TMEM sub-partition of this warp
-        const int r = sub * 32 + lane;   // query row of this thread in the tile
+        // ===================== softmax warpgroups: warps 2-5 -> tile A, 6-9 -> tile B =====================
+        const int x = (warp - 2) >> 2;  // 0 = A, 1 = B
+        const int sub = warp & 3;       // TMEM sub-partition of this warp
+        const int r = sub * 32 + lane;  // query row of this thread in its tile
         const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
+        const uint32_t s_tmem = tmem + lane_addr + 128u * x;
+        const uint32_t o_tmem = tmem + lane_addr + 256u + 128u * x;
         const float sl2 = p.scale_log2;
-        int kv_n = 0, n_it = 0;
+        int n_item = 0, s_n = 0, pv_n = 0, o_n = 0, kv_base = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+        for (;;) {
+            const int slot = n_item % kItemSlots;
+            ok = wait_bar(&item_full[slot], full_par(n_item / kItemSlots), abort_flag, p.status);
+            ok = __all_sync(0xffffffffu, ok);
+            const int it = ok ? item_slot[slot] : -1;
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&item_empty[slot]);
+            ++n_item;
+            if (it < 0)
+                break;
             Item I;
-            if (!get_item(p, it, I, false))
+            get_item(p, it, I, false);
+            const int kv_first = kv_base;  // index of this item's first K/V tile in the producer's order
+            kv_base += I.n_kv;
+            const Tile &t = x == 0 ? I.A : I.Bt;
+            if (!t.on)
                 continue;
-            const int ob = n_it & 1;
-            const uint32_t o_tmem = tmem + lane_addr + (ob ? kColO1 : kColO0);
             const int tl = r / p.G, gi = r % p.G;
-            const bool row_valid = r < p.rows_per_tile && tl < I.n_tok;
-            const int lim = row_valid ? I.ctx - I.qb + I.t_begin + tl : -1;
+            const bool row_valid = r < p.rows_per_tile && tl < t.n_tok;
+            const int lim = row_valid ? I.ctx - I.qb + t.t_begin + tl : -1;
+            // the warpgroup whose P V first reads the item's last V tile clears the keys past the
+            // context end in it (P is 0 there, but 0 * NaN is NaN)
+            const bool zero_owner = (x == 0) == (I.A.n_kv == I.n_kv);
             float m = -INFINITY, l = 0.f;
-            for (int j = 0; j < I.n_kv; ++j) {
-                const int n = kv_n + j, sb = n & 1;
-                ok = wait_bar(&s_full[sb], (n >> 1) & 1, abort_flag, p.status);
+            for (int j = 0; j < t.n_kv; ++j) {
+                ok = wait_bar(&s_full[x], full_par(s_n), abort_flag, p.status);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok)
                     break;
+                ++s_n;
                 tc::fence_after_sync();
-                const uint32_t s_tmem = tmem + lane_addr + (sb ? kColS1 : kColS0);
-                float s[kKeys];
-                {
-                    uint32_t raw[kKeys];
-                    tc::ld128(s_tmem, raw);
-#pragma unroll
-                    for (int i = 0; i < kKeys; ++i)
-                        s[i] = __uint_as_float(raw[i]);
-                }
+                // pass 1: row max of the (masked) scores, 64 columns at a time
                 const int key0 = j * kKeys;
-                float mx = -INFINITY;
-                if (key0 + kKeys - 1 <= lim) {
+                const bool need_mask = key0 + kKeys - 1 > lim;
+                float mx8[8];
 #pragma unroll
-                    for (int c = 0; c < kKeys; ++c)
-                        mx = fmaxf(mx, s[c]);
-                } else {
+                for (int i = 0; i < 8; ++i)
+                    mx8[i] = -INFINITY;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t raw[64];
+                    tc::ld64(s_tmem + h * 64, raw);
 #pragma unroll
-                    for (int c = 0; c < kKeys; ++c) {
-                        s[c] = (key0 + c <= lim) ? s[c] : -INFINITY;
-                        mx = fmaxf(mx, s[c]);
+                    for (int c = 0; c < 64; ++c) {
+                        float v = __uint_as_float(raw[c]);
+                        if (need_mask && key0 + h * 64 + c > lim)
+                            v = -INFINITY;
+                        mx8[c & 7] = fmaxf(mx8[c & 7], v);
                     }
                 }
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
                 const float mx_s = mx * sl2;  // scaled max (-inf stays -inf)
                 float factor = 1.f;
                 bool grow = false;
@@ -379,8 +564,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     grow = true;
                 }
                 if (__any_sync(0xffffffffu, grow)) {
-                    // O must hold P_(n-1) V_(n-1) before it is rescaled
-                    ok = wait_bar(&s_free[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, p.status);
+                    // O_X must hold every earlier P V product before it is rescaled
+                    ok = wait_bar(&pv_done[x], full_par(pv_n - 1), abort_flag, p.status);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok)
                         break;
@@ -394,63 +579,74 @@ __global__ void __launch_bounds__(kThreads, 1)
                             o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
                         tc::st32(o_tmem + c * 32, o);
                     }
-                    tc::wait_st();
                 }
-                const float base = m == -INFINITY ? 0.f : m;
-                uint32_t pk[kKeys / 2];
-                float rs = 0.f;
+                // pass 2: P = 2^(s * scale * log2 e - m), packed to 16 bits over the first 64 columns
+                // (half h reads columns 64h..64h+63 and writes 32h..32h+31: never ahead of its reads)
+                const float nb = m == -INFINITY ? 0.f : -m;
+                float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t raw[64];
+                    tc::ld64(s_tmem + h * 64, raw);
+                    uint32_t pk[32];
 #pragma unroll
-                for (int c = 0; c < kKeys; c += 2) {
-                    const float p0 = fast_exp2(fmaf(s[c], sl2, -base));
-                    const float p1 = fast_exp2(fmaf(s[c + 1], sl2, -base));
-                    rs += p0 + p1;
-                    pk[c / 2] = pack2<BF16>(p0, p1);
+                    for (int c = 0; c < 64; c += 2) {
+                        float v0 = __uint_as_float(raw[c]), v1 = __uint_as_float(raw[c + 1]);
+                        if (need_mask) {
+                            v0 = key0 + h * 64 + c <= lim ? v0 : -INFINITY;
+                            v1 = key0 + h * 64 + c + 1 <= lim ? v1 : -INFINITY;
+                        }
+                        const float p0 = fast_exp2(fmaf(v0, sl2, nb));
+                        const float p1 = fast_exp2(fmaf(v1, sl2, nb));
+                        rs[(c >> 1) & 3] += p0 + p1;
+                        pk[c >> 1] = pack2<BF16>(p0, p1);
+                    }
+                    tc::st32(s_tmem + h * 32, pk);
                 }
-                l += rs;
-                tc::st32(s_tmem, pk);
-                tc::st32(s_tmem + 32, pk + 32);
+                l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
                 tc::wait_st();
-                // keys past the context end in the sequence's last page may hold anything:
-                // zero their V rows before P V reads them (P is 0 there, but 0 * NaN is NaN)
-                if (j == I.n_kv - 1 && warp == 2) {
+                ++pv_n;  // the P V product of this tile
+                if (j == I.n_kv - 1 && zero_owner && sub == 0) {
                     const int last_page = (I.ctx + 15) / 16 - 1;
                     const int pg = last_page - 8 * j;
                     if ((I.ctx & 15) && I.n_pages == last_page + 1 && pg >= 0 && pg < 8) {
-                        const int s = n % kStages;
-                        ok = wait_bar(&kv_full[s], (n / kStages) & 1, abort_flag, p.status);
-                        if (ok) {
-                            uint8_t *vs = smem + L::kKV + s * 2 * L::kTile + L::kTile;
+                        const int vn = kv_first + j;  // V load index of this K/V step
+                        const int vstage = vn % kStages;
+                        bool landed = wait_bar(&v_full[vstage], full_par(vn / kStages), abort_flag, p.status);
+                        landed = __all_sync(0xffffffffu, landed);
+                        if (landed) {
+                            uint8_t *vsm = smem + L::kV + vstage * L::kTile;
                             const int r0 = I.ctx & 15;
-                            const int nz = (16 - r0) * 8 * KB;  // 16-byte chunks to clear
-                            for (int i = lane; i < nz; i += 32) {
-                                const int kb = i / ((16 - r0) * 8);
-                                const int rem = i % ((16 - r0) * 8);
+                            const int per_kb = (16 - r0) * 8;  // 16-byte chunks to clear per column block
+                            for (int i = lane; i < per_kb * KB; i += 32) {
+                                const int kb = i / per_kb, rem = i % per_kb;
                                 const int row = pg * 16 + r0 + rem / 8;
-                                *reinterpret_cast<uint4 *>(vs + kb * kRows * 128 + row * 128 + (rem & 7) * 16) =
+                                *reinterpret_cast<uint4 *>(vsm + kb * kRows * 128 + row * 128 + (rem & 7) * 16) =
                                     make_uint4(0, 0, 0, 0);
                             }
                             fence_proxy_async_smem();
                         }
-                        ok = __all_sync(0xffffffffu, ok);
                         __syncwarp();
+                        ok = landed;
                     }
                 }
                 tc::fence_before_sync();
-                mbar_arrive(&p_full[sb]);
+                mbar_arrive(&p_full[x]);
                 if (!ok)
                     break;
             }
             if (!ok)
                 break;
-            // epilogue: O / l -> out
-            ok = wait_bar(&o_full[ob], (n_it >> 1) & 1, abort_flag, p.status);
+            // epilogue: O_X / l -> out
+            ok = wait_bar(&o_full[x], full_par(o_n), abort_flag, p.status);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok)
                 break;
+            ++o_n;
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             uint8_t *orow = static_cast<uint8_t *>(p.out) +
-                            ((int64_t)(I.q0 + I.t_begin + tl) * p.H_q + I.g * p.G + gi) * (D * 2);
+                            ((int64_t)(I.q0 + t.t_begin + tl) * p.H_q + I.g * p.G + gi) * (D * 2);
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -468,9 +664,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc::fence_before_sync();
-            mbar_arrive(&o_free[ob]);
-            kv_n += I.n_kv;
-            ++n_it;
+            mbar_arrive(&o_free[x]);
         }
     }
 
@@ -496,6 +690,7 @@ static int run(const AttnArgs &a)
     p.context_lens = a.context_lens;
     p.out = a.out;
     p.status = static_cast<int32_t *>(a.workspace);
+    p.counter = reinterpret_cast<int *>(static_cast<uint8_t *>(a.workspace) + kCounterOffset);
     p.num_blocks = a.num_blocks;
     p.T = a.T;
     p.max_blocks = a.max_blocks;
@@ -507,8 +702,9 @@ static int run(const AttnArgs &a)
     p.max_ctx = a.max_ctx;
     p.tok_per_tile = kRows / G;
     p.rows_per_tile = p.tok_per_tile * G;
-    p.n_qt_max = (a.max_q_len + p.tok_per_tile - 1) / p.tok_per_tile;
-    const int64_t items = (int64_t)p.n_qt_max * a.B * a.H_kv;
+    const int n_qt = (a.max_q_len + p.tok_per_tile - 1) / p.tok_per_tile;
+    p.n_pairs_max = (n_qt + 1) / 2;
+    const int64_t items = (int64_t)p.n_pairs_max * a.B * a.H_kv;
     if (items > (int64_t(1) << 30) || a.T > (int64_t(1) << 31) - 256)
         return PA_ERR_UNSUPPORTED;
     p.n_items = static_cast<int>(items);
@@ -523,6 +719,8 @@ static int run(const AttnArgs &a)
         rc = make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
     if (rc != PA_OK)
         return rc;
+    if (cudaMemsetAsync(p.counter, 0, sizeof(int), a.stream) != cudaSuccess)
+        return PA_ERR_CUDA;
 
     auto kern = pa_prefill_tc_kernel<D, BF16>;
     static uint64_t configured = 0;
