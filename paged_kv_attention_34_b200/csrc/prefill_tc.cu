@@ -31,8 +31,9 @@
 //     thread execute in issue order, which makes that reuse safe;
 //   * warp 0 issues TMA and hands out work items from a global counter,
 //     heaviest first (later query tiles see more keys); warp 1 allocates TMEM
-//     and issues the MMAs; warps 2-5 and 6-9 are the two softmax warpgroups
-//     (rescale and epilogue included).  One persistent CTA per SM.
+//     and issues the MMAs (warps 2-3 idle; the first warpgroup shrinks its register
+//     budget so the softmax warpgroups can grow theirs); warps 4-7 and 8-11 are the
+//     two softmax warpgroups (rescale and epilogue included).  One persistent CTA per SM.
 // All waits are bounded; a wait that runs out records PA_ERR_TIMEOUT and the
 // CTA winds down (its copies and MMAs in flight are waited for, TMEM freed).
 #include <cmath>
@@ -47,10 +48,16 @@ namespace tcp {
 constexpr int kRows = 128;     // query rows per tile (TMEM lanes)
 constexpr int kKeys = 128;     // keys per K/V tile
 constexpr int kStages = 2;     // depth of the K ring and of the V ring
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 384;  // 3 warpgroups: scheduler/TMA/MMA, softmax A, softmax B
+// Register budgets: launched at 168 per thread (65536 / 384, rounded to 8); the first warpgroup
+// gives registers back, the softmax warpgroups take them: 128 * 80 + 256 * 208 <= 384 * 168.
+constexpr int kLaunchRegs = 168;
+constexpr uint32_t kRegsControl = 88;
+constexpr uint32_t kRegsSoftmax = 208;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split over budget");
 constexpr int kMaxTable = 1024;
 constexpr int kItemSlots = 2;
-constexpr int kItemReaders = 9;  // warp 1 and warps 2-9 each acknowledge a work item
+constexpr int kItemReaders = 9;  // warp 1 and warps 4-11 each acknowledge a work item
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr size_t kCounterOffset = 64;      // work counter inside the status area of the workspace
 
@@ -71,24 +78,8 @@ struct Params {
     int n_pairs_max;    // ceil(ceil(max_q_len / tok_per_tile) / 2)
     int n_items;        // n_pairs_max * B * H_kv
     int oob_row;        // first row past the pool in the cache tensor map
+    int out_align32;    // out is 32-byte aligned: 32-byte stores in the epilogue
     float scale_log2;
-};
-
-template <int D>
-struct Smem {
-    static constexpr int kKB = D / 64;               // 128-byte column blocks
-    static constexpr int kTile = kKB * kRows * 128;  // one 128-row x D tile
-    static constexpr int kQ = 0;                     // Q_A, Q_B
-    static constexpr int kK = 2 * kTile;             // K ring
-    static constexpr int kV = kK + kStages * kTile;  // V ring
-    static constexpr int kTable = kV + kStages * kTile;
-    static constexpr int kBars = kTable + 4 * kMaxTable;
-    static constexpr int kNumBars = 2 * 2 + 4 * kStages + 5 * 2 + 2 * kItemSlots + 1;
-    static constexpr int kItems = kBars + 8 * kNumBars;
-    static constexpr int kTmemSlot = kItems + 4 * kItemSlots;
-    static constexpr int kAbort = kTmemSlot + 8;
-    static constexpr int kBytes = kAbort + 8;
-    static constexpr int kAlloc = kBytes + 1024;
 };
 
 // One query tile of a work item.
@@ -104,6 +95,30 @@ struct Item {
     Tile A, Bt;
     int n_kv;     // K/V tiles of the item (= the larger of the two)
     int n_pages;  // pages of the item
+};
+
+// What the scheduler hands to the other roles: the item index (-1 = no more work) and the
+// decoded item, so that no role re-reads the sequence metadata from global memory.
+struct ItemSlot {
+    int it;
+    Item I;
+};
+
+template <int D>
+struct Smem {
+    static constexpr int kKB = D / 64;               // 128-byte column blocks
+    static constexpr int kTile = kKB * kRows * 128;  // one 128-row x D tile
+    static constexpr int kQ = 0;                     // Q_A, Q_B
+    static constexpr int kK = 2 * kTile;             // K ring
+    static constexpr int kV = kK + kStages * kTile;  // V ring
+    static constexpr int kTable = kV + kStages * kTile;
+    static constexpr int kBars = kTable + 4 * kMaxTable;
+    static constexpr int kNumBars = 2 * 2 + 4 * kStages + 5 * 2 + 2 * kItemSlots + 1;
+    static constexpr int kItems = kBars + 8 * kNumBars;
+    static constexpr int kTmemSlot = kItems + ((int(sizeof(ItemSlot)) * kItemSlots + 15) / 16) * 16;
+    static constexpr int kAbort = kTmemSlot + 8;
+    static constexpr int kBytes = kAbort + 8;
+    static constexpr int kAlloc = kBytes + 1024;
 };
 
 __device__ __forceinline__ void make_tile(const Params &p, const Item &I, int qt, Tile &t)
@@ -196,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *item_full = o_free + 2;           // [kItemSlots]
     uint64_t *item_empty = item_full + kItemSlots;
     uint64_t *drain = item_empty + kItemSlots;  // [1]
-    int *item_slot = reinterpret_cast<int *>(smem + L::kItems);
+    ItemSlot *item_slot = reinterpret_cast<ItemSlot *>(smem + L::kItems);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kAbort);
     int32_t *s_table = reinterpret_cast<int32_t *>(smem + L::kTable);
@@ -240,6 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     // TMEM columns of tile X: S_X at 128 X, O_X at 256 + 128 X
 
+    if (warp < 4) {
+    // first warpgroup: give registers back (all four warps), then split into roles
+    tc::regs_shrink<kRegsControl>();
     if (warp == 0) {
         // ===================== scheduler + TMA producer =====================
         int n_pub = 0, k_n = 0, v_n = 0, q_n[2] = {0, 0};
@@ -266,26 +284,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int slot = n_pub % kItemSlots;
                 const bool got = wait_bar(&item_empty[slot], free_par(n_pub / kItemSlots), abort_flag, p.status);
                 ok = ok && got;
-                item_slot[slot] = ok ? it : -1;
+                item_slot[slot].it = ok ? it : -1;
+                item_slot[slot].I = I;
                 mbar_arrive(&item_full[slot]);
             }
             ++n_pub;
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (it < 0 || !ok)
                 break;
-            // page ids of the item into shared memory
             const int32_t *table = p.block_tables + (int64_t)I.b * p.max_blocks;
-            for (int i = lane; i < min(I.n_pages, kMaxTable); i += 32) {
-                int pg = __ldg(table + i);
-                if (pg < 0 || pg >= p.num_blocks) {
-                    set_status(p.status, PA_ERR_BOUNDS);
-                    pg = -1;
-                }
-                s_table[i] = pg;
-            }
-            __syncwarp();
             if (lane == 0) {
-                // Q tiles
+                // Q tiles first: they do not need the page table
                 const Tile *tl[2] = {&I.A, &I.Bt};
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
@@ -301,6 +310,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &q_full[x]);
                     ++q_n[x];
                 }
+            }
+            // page ids of the item into shared memory
+            for (int i = lane; i < min(I.n_pages, kMaxTable); i += 32) {
+                int pg = __ldg(table + i);
+                if (pg < 0 || pg >= p.num_blocks) {
+                    set_status(p.status, PA_ERR_BOUNDS);
+                    pg = -1;
+                }
+                s_table[i] = pg;
+            }
+            __syncwarp();
+            if (lane == 0) {
                 // K and V tiles, interleaved
                 for (int j = 0; j < I.n_kv && ok; ++j) {
                     int y[8];
@@ -364,115 +385,121 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // ===================== MMA issuer =====================
+        // Event driven: every product is issued as soon as its inputs are ready, so one slow
+        // softmax tile does not hold back the other tile's products.  Per tile, S_X(j+1) is
+        // issued only after P_X(j) V (in-order execution keeps the TMEM reuse safe); a K (V) tile
+        // is released once every S (P V) product that reads it has been issued.
         constexpr uint32_t idesc_qk = tc::idesc_f16(BF16, kRows, kKeys, false);
         constexpr uint32_t idesc_pv = tc::idesc_f16(BF16, kRows, D, true);
-        int n_item = 0, k_n = 0, v_n = 0, q_n[2] = {0, 0}, pv_n[2] = {0, 0}, o_n[2] = {0, 0};
+        int n_item = 0, k_base = 0, q_n[2] = {0, 0}, pv_n[2] = {0, 0}, o_n[2] = {0, 0};
         bool ok = true;
         for (;;) {
             const int slot = n_item % kItemSlots;
             ok = wait_bar(&item_full[slot], full_par(n_item / kItemSlots), abort_flag, p.status);
             ok = __all_sync(0xffffffffu, ok);
-            const int it = ok ? item_slot[slot] : -1;
+            const int it = ok ? item_slot[slot].it : -1;
+            Item I;
+            if (it >= 0)
+                I = item_slot[slot].I;
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&item_empty[slot]);
             ++n_item;
             if (it < 0)
                 break;
-            Item I;
-            get_item(p, it, I, false);
             if (lane == 0) {
-                const Tile *tl[2] = {&I.A, &I.Bt};
-                uint32_t q_addr[2];
+                const int nt[2] = {I.A.n_kv, I.Bt.n_kv};  // 0 for a tile without tokens
+                const int n = I.n_kv;
+                const uint32_t q_addr[2] = {smem_u32(smem + L::kQ), smem_u32(smem + L::kQ + L::kTile)};
 #pragma unroll
                 for (int x = 0; x < 2; ++x)
-                    q_addr[x] = smem_u32(smem + L::kQ + x * L::kTile);
-#pragma unroll
-                for (int x = 0; x < 2; ++x)
-                    if (ok && tl[x]->on) {
+                    if (ok && nt[x] > 0) {
                         ok = wait_bar(&q_full[x], full_par(q_n[x]), abort_flag, p.status);
                         ++q_n[x];
                     }
-                // S_X(j) = Q_X K_j^T
-                auto qk = [&](int x, int j, int kstage) {
-                    const uint32_t k_addr = smem_u32(smem + L::kK + kstage * L::kTile);
-                    const uint32_t d = tmem + 128u * x;
+                int qk_i[2] = {0, 0}, pv_i[2] = {0, 0};  // next S / next P V product per tile
+                int k_rel = 0, v_rel = 0;                // K / V tiles of this item released
+                uint64_t t_last = globaltimer();
+                while (ok) {
+                    bool progress = false;
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
-                        tc::mma_ss(d, tc::desc_k_sw128(q_addr[x] + off), tc::desc_k_sw128(k_addr + off), idesc_qk,
-                                   ks > 0 ? 1u : 0u);
-                    }
-                    tc::commit(&s_full[x]);
-                    if (j == tl[x]->n_kv - 1)
-                        tc::commit(&q_empty[x]);  // Q_X no longer needed
-                };
-                // O_X += P_X(j) V_j (waits for P_X(j); on the first tile also for the last epilogue of X)
-                auto pv = [&](int x, int j, int vstage) -> bool {
-                    if (!wait_bar(&p_full[x], full_par(pv_n[x]), abort_flag, p.status))
-                        return false;
-                    if (j == 0 && !wait_bar(&o_free[x], free_par(o_n[x]), abort_flag, p.status))
-                        return false;
-                    tc::fence_after_sync();
-                    const uint32_t v_addr = smem_u32(smem + L::kV + vstage * L::kTile);
-                    const uint32_t d = tmem + 256u + 128u * x;
-                    const uint32_t a = tmem + 128u * x;
+                    for (int x = 0; x < 2; ++x) {
+                        // O_X += P_X(j) V_j
+                        const int j = pv_i[x];
+                        // on the item's last V tile, tile A goes first (it clears the tail rows)
+                        const bool order_ok = !(x == 1 && j == n - 1 && nt[0] == n && pv_i[0] < n);
+                        if (j < qk_i[x] && order_ok) {
+                            const int vg = k_base + j;
+                            if (mbar_test(&p_full[x], full_par(pv_n[x])) &&
+                                mbar_test(&v_full[vg % kStages], full_par(vg / kStages)) &&
+                                (j > 0 || mbar_test(&o_free[x], free_par(o_n[x])))) {
+                                tc::fence_after_sync();
+                                const uint32_t v_addr = smem_u32(smem + L::kV + (vg % kStages) * L::kTile);
+                                const uint32_t d = tmem + 256u + 128u * x;
+                                const uint32_t a = tmem + 128u * x;
 #pragma unroll
-                    for (int ks = 0; ks < kKeys / 16; ++ks)
-                        tc::mma_ts(d, a + ks * 8, tc::desc_mn_sw128(v_addr + ks * 2048, kRows * 128), idesc_pv,
-                                   (j > 0 || ks > 0) ? 1u : 0u);
-                    tc::commit(&pv_done[x]);
-                    ++pv_n[x];
-                    if (j == tl[x]->n_kv - 1) {
-                        tc::commit(&o_full[x]);
-                        ++o_n[x];
-                    }
-                    return true;
-                };
-                const int n = I.n_kv;
-                int vst_prev = 0;
-                for (int j = 0; j <= n && ok; ++j) {
-                    int kst = 0, vst = 0;
-                    if (j < n) {
-                        kst = k_n % kStages;
-                        ok = wait_bar(&k_full[kst], full_par(k_n / kStages), abort_flag, p.status);
-                        ++k_n;
-                        if (!ok)
-                            break;
-                        tc::fence_after_sync();
-                        if (j < I.A.n_kv)
-                            qk(0, j, kst);
-                    }
-                    if (j >= 1) {
-                        // O_B += P_B(j-1) V(j-1); after it the V tile j-1 is free
-                        if (j - 1 < I.Bt.n_kv) {
-                            ok = pv(1, j - 1, vst_prev);
-                            if (!ok)
-                                break;
+                                for (int ks = 0; ks < kKeys / 16; ++ks)
+                                    tc::mma_ts(d, a + ks * 8, tc::desc_mn_sw128(v_addr + ks * 2048, kRows * 128),
+                                               idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+                                tc::commit(&pv_done[x]);
+                                ++pv_n[x];
+                                ++pv_i[x];
+                                if (pv_i[x] == nt[x]) {
+                                    tc::commit(&o_full[x]);
+                                    ++o_n[x];
+                                }
+                                progress = true;
+                            }
                         }
-                        tc::commit(&v_empty[vst_prev]);
-                    }
-                    if (j < n) {
-                        if (j < I.Bt.n_kv)
-                            qk(1, j, kst);
-                        tc::commit(&k_empty[kst]);
-                        vst = v_n % kStages;
-                        ok = wait_bar(&v_full[vst], full_par(v_n / kStages), abort_flag, p.status);
-                        ++v_n;
-                        if (!ok)
-                            break;
-                        if (j < I.A.n_kv) {
-                            ok = pv(0, j, vst);
-                            if (!ok)
-                                break;
+                        // S_X(j) = Q_X K_j^T, once P_X(j-1) V has been issued
+                        const int jq = qk_i[x];
+                        if (jq < nt[x] && pv_i[x] == jq) {
+                            const int kg = k_base + jq;
+                            if (mbar_test(&k_full[kg % kStages], full_par(kg / kStages))) {
+                                tc::fence_after_sync();
+                                const uint32_t k_addr = smem_u32(smem + L::kK + (kg % kStages) * L::kTile);
+                                const uint32_t d = tmem + 128u * x;
+#pragma unroll
+                                for (int ks = 0; ks < D / 16; ++ks) {
+                                    const uint32_t off = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
+                                    tc::mma_ss(d, tc::desc_k_sw128(q_addr[x] + off), tc::desc_k_sw128(k_addr + off),
+                                               idesc_qk, ks > 0 ? 1u : 0u);
+                                }
+                                tc::commit(&s_full[x]);
+                                ++qk_i[x];
+                                if (qk_i[x] == nt[x])
+                                    tc::commit(&q_empty[x]);  // Q_X no longer needed
+                                progress = true;
+                            }
                         }
                     }
-                    vst_prev = vst;
+                    // release the K and V tiles that no further product of this item reads
+                    while (k_rel < n && (k_rel >= nt[0] || qk_i[0] > k_rel) && (k_rel >= nt[1] || qk_i[1] > k_rel)) {
+                        tc::commit(&k_empty[(k_base + k_rel) % kStages]);
+                        ++k_rel;
+                    }
+                    while (v_rel < n && (v_rel >= nt[0] || pv_i[0] > v_rel) && (v_rel >= nt[1] || pv_i[1] > v_rel)) {
+                        tc::commit(&v_empty[(k_base + v_rel) % kStages]);
+                        ++v_rel;
+                    }
+                    if (pv_i[0] == nt[0] && pv_i[1] == nt[1])
+                        break;  // every product of the item is issued
+                    if (progress) {
+                        t_last = globaltimer();
+                    } else {
+                        if (*abort_flag) {
+                            ok = false;
+                        } else if (globaltimer() - t_last > kWaitTimeoutNs) {
+                            *abort_flag = 1;
+                            set_status(p.status, PA_ERR_TIMEOUT);
+                            ok = false;
+                        }
+                    }
                 }
+                k_base += n;
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            k_n = __shfl_sync(0xffffffffu, k_n, 0);
-            v_n = __shfl_sync(0xffffffffu, v_n, 0);
+            k_base = __shfl_sync(0xffffffffu, k_base, 0);
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 q_n[x] = __shfl_sync(0xffffffffu, q_n[x], 0);
@@ -488,9 +515,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(drain, 0, kWaitTimeoutNs / 10);
         }
         __syncwarp();
+    }
     } else {
-        // ===================== softmax warpgroups: warps 2-5 -> tile A, 6-9 -> tile B =====================
-        const int x = (warp - 2) >> 2;  // 0 = A, 1 = B
+        tc::regs_grow<kRegsSoftmax>();
+        // ===================== softmax warpgroups: warps 4-7 -> tile A, 8-11 -> tile B =====================
+        const int x = (warp - 4) >> 2;  // 0 = A, 1 = B
         const int sub = warp & 3;       // TMEM sub-partition of this warp
         const int r = sub * 32 + lane;  // query row of this thread in its tile
         const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
@@ -503,15 +532,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int slot = n_item % kItemSlots;
             ok = wait_bar(&item_full[slot], full_par(n_item / kItemSlots), abort_flag, p.status);
             ok = __all_sync(0xffffffffu, ok);
-            const int it = ok ? item_slot[slot] : -1;
+            const int it = ok ? item_slot[slot].it : -1;
+            Item I;
+            if (it >= 0)
+                I = item_slot[slot].I;
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&item_empty[slot]);
             ++n_item;
             if (it < 0)
                 break;
-            Item I;
-            get_item(p, it, I, false);
             const int kv_first = kv_base;  // index of this item's first K/V tile in the producer's order
             kv_base += I.n_kv;
             const Tile &t = x == 0 ? I.A : I.Bt;
@@ -521,37 +551,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_valid = r < p.rows_per_tile && tl < t.n_tok;
             const int lim = row_valid ? I.ctx - I.qb + t.t_begin + tl : -1;
             // the warpgroup whose P V first reads the item's last V tile clears the keys past the
-            // context end in it (P is 0 there, but 0 * NaN is NaN)
-            const bool zero_owner = (x == 0) == (I.A.n_kv == I.n_kv);
+            // context end in it (P is 0 there, but 0 * NaN is NaN); everything it needs is fixed here
+            const int last_page = (I.ctx + 15) / 16 - 1;
+            const int zpg = last_page - 8 * (I.n_kv - 1);
+            const bool do_zero = ((x == 0) == (I.A.n_kv == I.n_kv)) && sub == 0 && (I.ctx & 15) &&
+                                 I.n_pages == last_page + 1 && zpg >= 0 && zpg < 8;
+            const int zr0 = I.ctx & 15;
+            const int zvn = kv_first + I.n_kv - 1;  // V load index of the item's last K/V step
+            const int n_kv_t = t.n_kv;
+            uint8_t *orow = static_cast<uint8_t *>(p.out) +
+                            ((int64_t)(I.q0 + t.t_begin + tl) * p.H_q + I.g * p.G + gi) * (D * 2);
             float m = -INFINITY, l = 0.f;
-            for (int j = 0; j < t.n_kv; ++j) {
+            for (int j = 0; j < n_kv_t; ++j) {
                 ok = wait_bar(&s_full[x], full_par(s_n), abort_flag, p.status);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok)
                     break;
                 ++s_n;
                 tc::fence_after_sync();
-                // pass 1: row max of the (masked) scores, 64 columns at a time
+                // the whole S row in one TMEM load; masked keys (causal / context end) become -inf
                 const int key0 = j * kKeys;
-                const bool need_mask = key0 + kKeys - 1 > lim;
-                float mx8[8];
+                uint32_t raw[kKeys];
+                tc::ld128(s_tmem, raw);
+                if (key0 + kKeys - 1 > lim) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    mx8[i] = -INFINITY;
-#pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t raw[64];
-                    tc::ld64(s_tmem + h * 64, raw);
-#pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        float v = __uint_as_float(raw[c]);
-                        if (need_mask && key0 + h * 64 + c > lim)
-                            v = -INFINITY;
-                        mx8[c & 7] = fmaxf(mx8[c & 7], v);
-                    }
+                    for (int c = 0; c < kKeys; ++c)
+                        if (key0 + c > lim)
+                            raw[c] = 0xff800000u;  // -inf
                 }
-                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                float mx4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    mx4[i] = fmaxf(__uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1]));
+#pragma unroll
+                for (int c = 8; c < kKeys; c += 2)
+                    mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
+                const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
                 const float mx_s = mx * sl2;  // scaled max (-inf stays -inf)
                 float factor = 1.f;
                 bool grow = false;
@@ -571,64 +606,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     tc::fence_after_sync();
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tc::ld32(o_tmem + c * 32, o);
+                    for (int c = 0; c < D / 16; ++c) {
+                        uint32_t o[16];
+                        tc::ld16(o_tmem + c * 16, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
+                        for (int i = 0; i < 16; ++i)
                             o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-                        tc::st32(o_tmem + c * 32, o);
+                        tc::st16(o_tmem + c * 16, o);
                     }
                 }
-                // pass 2: P = 2^(s * scale * log2 e - m), packed to 16 bits over the first 64 columns
-                // (half h reads columns 64h..64h+63 and writes 32h..32h+31: never ahead of its reads)
+                // P = 2^(s * scale * log2 e - m), packed to 16 bits in place and stored over the
+                // first 64 columns of S
+                // P = 2^(s * scale * log2 e - m) (masked keys: 2^-inf = 0), packed to 16 bits in place
                 const float nb = m == -INFINITY ? 0.f : -m;
-                float rs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t raw[64];
-                    tc::ld64(s_tmem + h * 64, raw);
-                    uint32_t pk[32];
+                const uint64_t sl2_2 = f2_pack(sl2, sl2), nb_2 = f2_pack(nb, nb);
+                uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        float v0 = __uint_as_float(raw[c]), v1 = __uint_as_float(raw[c + 1]);
-                        if (need_mask) {
-                            v0 = key0 + h * 64 + c <= lim ? v0 : -INFINITY;
-                            v1 = key0 + h * 64 + c + 1 <= lim ? v1 : -INFINITY;
-                        }
-                        const float p0 = fast_exp2(fmaf(v0, sl2, nb));
-                        const float p1 = fast_exp2(fmaf(v1, sl2, nb));
-                        rs[(c >> 1) & 3] += p0 + p1;
-                        pk[c >> 1] = pack2<BF16>(p0, p1);
-                    }
-                    tc::st32(s_tmem + h * 32, pk);
+                for (int q = 0; q < kKeys / 2; ++q) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(raw[2 * q]), __uint_as_float(raw[2 * q + 1])), sl2_2, nb_2),
+                              x0, x1);
+                    const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+                    acc[q & 1] = f2_add(acc[q & 1], f2_pack(p0, p1));
+                    raw[q] = pack2<BF16>(p0, p1);
                 }
-                l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+                {
+                    float a0, a1, b0, b1;
+                    f2_unpack(acc[0], a0, a1);
+                    f2_unpack(acc[1], b0, b1);
+                    l += (a0 + a1) + (b0 + b1);
+                }
+                tc::st32(s_tmem, raw);
+                tc::st32(s_tmem + 32, raw + 32);
                 tc::wait_st();
                 ++pv_n;  // the P V product of this tile
-                if (j == I.n_kv - 1 && zero_owner && sub == 0) {
-                    const int last_page = (I.ctx + 15) / 16 - 1;
-                    const int pg = last_page - 8 * j;
-                    if ((I.ctx & 15) && I.n_pages == last_page + 1 && pg >= 0 && pg < 8) {
-                        const int vn = kv_first + j;  // V load index of this K/V step
-                        const int vstage = vn % kStages;
-                        bool landed = wait_bar(&v_full[vstage], full_par(vn / kStages), abort_flag, p.status);
-                        landed = __all_sync(0xffffffffu, landed);
-                        if (landed) {
-                            uint8_t *vsm = smem + L::kV + vstage * L::kTile;
-                            const int r0 = I.ctx & 15;
-                            const int per_kb = (16 - r0) * 8;  // 16-byte chunks to clear per column block
-                            for (int i = lane; i < per_kb * KB; i += 32) {
-                                const int kb = i / per_kb, rem = i % per_kb;
-                                const int row = pg * 16 + r0 + rem / 8;
-                                *reinterpret_cast<uint4 *>(vsm + kb * kRows * 128 + row * 128 + (rem & 7) * 16) =
-                                    make_uint4(0, 0, 0, 0);
-                            }
-                            fence_proxy_async_smem();
+                if (do_zero && j == n_kv_t - 1) {
+                    const int vstage = zvn % kStages;
+                    bool landed = wait_bar(&v_full[vstage], full_par(zvn / kStages), abort_flag, p.status);
+                    landed = __all_sync(0xffffffffu, landed);
+                    if (landed) {
+                        uint8_t *vsm = smem + L::kV + vstage * L::kTile;
+                        const int per_kb = (16 - zr0) * 8;  // 16-byte chunks to clear per column block
+                        for (int i = lane; i < per_kb * KB; i += 32) {
+                            const int kb = i / per_kb, rem = i % per_kb;
+                            const int row = zpg * 16 + zr0 + rem / 8;
+                            *reinterpret_cast<uint4 *>(vsm + kb * kRows * 128 + row * 128 + (rem & 7) * 16) =
+                                make_uint4(0, 0, 0, 0);
                         }
-                        __syncwarp();
-                        ok = landed;
+                        fence_proxy_async_smem();
                     }
+                    __syncwarp();
+                    ok = landed;
                 }
                 tc::fence_before_sync();
                 mbar_arrive(&p_full[x]);
@@ -645,21 +673,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++o_n;
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint8_t *orow = static_cast<uint8_t *>(p.out) +
-                            ((int64_t)(I.q0 + t.t_begin + tl) * p.H_q + I.g * p.G + gi) * (D * 2);
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tc::ld32(o_tmem + c * 32, o);
-                if (row_valid) {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 v;
-                        v.x = pack2<BF16>(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
-                        v.y = pack2<BF16>(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-                        v.z = pack2<BF16>(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-                        v.w = pack2<BF16>(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(orow + (c * 32 + i) * 2) = v;
+                for (int i = 0; i < 32; i += 2)
+                    o[i >> 1] = pack2<BF16>(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+                if (row_valid) {
+                    uint8_t *dst = orow + c * 64;
+                    if (p.out_align32) {
+                        st_global_v8(dst, o);
+                        st_global_v8(dst + 32, o + 8);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4)
+                            *reinterpret_cast<uint4 *>(dst + i * 4) = make_uint4(o[i], o[i + 1], o[i + 2], o[i + 3]);
                     }
                 }
             }
@@ -709,6 +738,7 @@ static int run(const AttnArgs &a)
         return PA_ERR_UNSUPPORTED;
     p.n_items = static_cast<int>(items);
     p.oob_row = static_cast<int>(a.num_blocks * a.H_kv * 16);
+    p.out_align32 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     p.scale_log2 = a.scale * 1.4426950408889634f;
 
     CUtensorMap tq, tk, tv;
@@ -729,6 +759,13 @@ static int run(const AttnArgs &a)
         return PA_ERR_CUDA;
     const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
     if (!bit || !(configured & bit)) {
+        // the per-warpgroup register split assumes exactly kLaunchRegs registers per thread at
+        // launch; with any other count the growing warpgroups could wait forever, so refuse
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+            return PA_ERR_CUDA;
+        if (fa.numRegs != kLaunchRegs)
+            return PA_ERR_UNSUPPORTED;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
             return PA_ERR_CUDA;
         configured |= bit;

@@ -116,8 +116,21 @@ __device__ __forceinline__ void commit(uint64_t *bar)
 
 // ---- TMEM <-> registers (32 lanes x 32-bit, consecutive columns per thread) ---------------
 
-// Load 32, 64 or 128 consecutive 32-bit columns of this thread's TMEM lane and wait for
+// Load 16, 32, 64 or 128 consecutive 32-bit columns of this thread's TMEM lane and wait for
 // them in the same statement, so no register is read before the data has arrived.
+__device__ __forceinline__ void ld16(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15"
+        "}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
 __device__ __forceinline__ void ld32(uint32_t taddr, uint32_t *r)
 {
     asm volatile(
@@ -190,6 +203,17 @@ __device__ __forceinline__ void ld128(uint32_t taddr, uint32_t *r)
         : "memory");
 }
 
+__device__ __forceinline__ void st16(uint32_t taddr, const uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {"
+        "%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16"
+        "};" ::"r"(taddr),
+          "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void st32(uint32_t taddr, const uint32_t *r)
 {
     asm volatile(
@@ -203,6 +227,22 @@ __device__ __forceinline__ void st32(uint32_t taddr, const uint32_t *r)
 }
 
 __device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---- per-warpgroup register budget (setmaxnreg) ---------------------------------------------
+// All four warps of a warpgroup execute the same call.  The budgets of all warpgroups must add
+// up to no more than the CTA's launch allocation (threads x registers per thread at launch).
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_grow()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <uint32_t N>
+__device__ __forceinline__ void regs_shrink()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 // ---- TMA 3-D tile load -----------------------------------------------------------------------
 
