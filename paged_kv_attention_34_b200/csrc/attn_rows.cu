@@ -9,11 +9,15 @@
 // combines the splits ("cross-block reduction").  A sequence short enough
 // for one split is written straight to `out`.
 //
-// Data movement: one thread issues TMA box loads (64 elements x 16 rows,
-// 128-byte swizzle) of whole (block, head) pages straight from the block pool
-// into a ring of shared-memory stages; completion is tracked by mbarriers with
-// bounded waits.  The page ids come from the block table (iopencloud section
-// 3.2), prefetched into shared memory.  K/V bytes are read once per CTA.
+// Data movement: TMA box loads (64 elements x 16 rows, 128-byte swizzle) of
+// whole (block, head) pages straight from the block pool into a ring of three
+// shared-memory stages; completion is tracked by mbarriers with bounded waits.
+// The page ids come from the block table (iopencloud section 3.2): the first
+// stages are issued at once from the table in global memory, the rest from a
+// copy in shared memory.  A stage is refilled by the last warp to finish with
+// it, so no warp waits for the others between stages.  Q is staged through the
+// last stage's buffer before that buffer's first load.  K/V bytes are read
+// once per CTA.
 //
 // Compute: four warps; each owns a 16-row m-tile and a subset of the pages of
 // every stage (several warps on different pages when there are <= 32 rows,
@@ -28,7 +32,7 @@ namespace pa {
 
 constexpr int kRowsPerCta = 64;
 constexpr int kPagesPerStage = 4;
-constexpr int kMaxTablePages = 1024;  // page ids cached in shared memory per CTA
+constexpr int kMaxTablePages = 256;  // page ids of one split (split_pages <= this)
 constexpr int kThreads = 128;
 
 struct RowsParams {
@@ -47,9 +51,8 @@ struct RowsParams {
     int max_ctx;
     int max_q_len;
     int n_rg;         // row groups of 64 rows per (sequence, KV head)
-    int split_pages;  // pages per split (decode); >= all pages for prefill
+    int split_pages;  // pages per split
     float scale_log2;  // scale * log2(e)
-    int decode;        // 1: split-KV decode grid, 0: prefill grid
 };
 
 template <int D, int STAGES>
@@ -60,10 +63,13 @@ struct RowsSmem {
     static constexpr int kEpiStride = D + 8;  // floats per row of the epilogue buffer
     static constexpr int kEpiBytes = (4 * 16 * kEpiStride + 2 * 64) * 4;
     static_assert(kEpiBytes <= STAGES * kStageBytes, "epilogue must fit in the stage ring");
+    static_assert(kQBytes <= kStageBytes, "Q is staged through one stage buffer");
     static constexpr int kStageOff = 0;
-    static constexpr int kQOff = STAGES * kStageBytes;
-    static constexpr int kBarOff = kQOff + kQBytes;
-    static constexpr int kTableOff = kBarOff + 8 * STAGES;
+    static constexpr int kQOff = (STAGES - 1) * kStageBytes;  // aliases the last stage during set-up
+    static constexpr int kBarOff = STAGES * kStageBytes;
+    static constexpr int kCountOff = kBarOff + 8 * STAGES;    // warps done with each stage
+    static constexpr int kIssuedOff = kCountOff + 4 * STAGES; // loads issued into each stage
+    static constexpr int kTableOff = kIssuedOff + 4 * STAGES;
     static constexpr int kFlagOff = kTableOff + 4 * kMaxTablePages;
     static constexpr int kBytes = kFlagOff + 16;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (swizzle atoms)
@@ -104,6 +110,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *s_stage = smem + L::kStageOff;
     uint8_t *s_q = smem + L::kQOff;
     uint64_t *s_bar = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    int *s_count = reinterpret_cast<int *>(smem + L::kCountOff);
+    int *s_issued = reinterpret_cast<int *>(smem + L::kIssuedOff);
     int32_t *s_pages = reinterpret_cast<int32_t *>(smem + L::kTableOff);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
 
@@ -111,16 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- which (sequence, KV head, row group, split) --------------------------------
     const int b = blockIdx.z;
-    int g, rg, split;
-    if (p.decode) {
-        split = blockIdx.x;
-        g = blockIdx.y / p.n_rg;
-        rg = blockIdx.y % p.n_rg;
-    } else {
-        split = 0;
-        g = blockIdx.y;
-        rg = p.n_rg - 1 - blockIdx.x;  // later row groups see more keys: launch them first
-    }
+    const int split = blockIdx.x;
+    const int g = blockIdx.y / p.n_rg, rg = blockIdx.y % p.n_rg;
     const int q0 = __ldg(p.cu_seqlens + b), q1 = __ldg(p.cu_seqlens + b + 1);
     const int qb = q1 - q0, ctx = __ldg(p.context_lens + b);
     if (!seq_ok(qb, ctx, p, q1)) {
@@ -137,14 +137,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lim_cta = ctx - qb + (row0 + rows_here - 1) / G;  // last key any row here sees
     const int pages_need = lim_cta / 16 + 1;
     const int pages_ctx = (ctx + 15) / 16;
-    int n_splits = 1, page_lo = 0, page_hi = pages_need;
-    if (p.decode) {
-        n_splits = (pages_ctx + p.split_pages - 1) / p.split_pages;
-        if (split >= n_splits)
-            return;
-        page_lo = split * p.split_pages;
-        page_hi = min(page_lo + p.split_pages, pages_need);
-    }
+    const int n_splits = (pages_ctx + p.split_pages - 1) / p.split_pages;
+    if (split >= n_splits)
+        return;
+    const int page_lo = split * p.split_pages;
+    const int page_hi = min(page_lo + p.split_pages, pages_need);
     const int n_pages = max(0, page_hi - page_lo);
     const int n_stages = (n_pages + kPagesPerStage - 1) / kPagesPerStage;
 
@@ -154,24 +151,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int mt = warp / KG, kg = warp % KG;
     const bool has_rows = mt * 16 < rows_here;
 
-    // ---- set-up: barriers, page ids, Q tile ---------------------------------------------
-    if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s)
-            mbar_init(&s_bar[s], 1);
-        *s_abort = 0;
-        fence_barrier_init();
-        prefetch_tmap(&tmap_k);
-        prefetch_tmap(&tmap_v);
-    }
+    // ---- set-up: barriers and the first loads, page ids, Q tile ---------------------------
     const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
-    for (int i = tid; i < min(n_pages, kMaxTablePages); i += kThreads) {
-        int pg = __ldg(table + page_lo + i);
+    auto checked = [&](int pg) -> int {
         if (pg < 0 || pg >= p.num_blocks) {
             set_status(p.status, PA_ERR_BOUNDS);
             pg = static_cast<int>(p.num_blocks);  // past the pool: TMA fills zeros
         }
-        s_pages[i] = pg;
+        return pg;
+    };
+    auto issue = [&](int st, bool from_global) {  // one thread
+        const int slot = st % STAGES;
+        uint8_t *kb = s_stage + slot * L::kStageBytes;
+        uint8_t *vb = kb + kPagesPerStage * L::kPageBytes;
+        const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&s_bar[slot], np * 2 * L::kPageBytes);
+        s_issued[slot] += 1;
+        for (int k = 0; k < np; ++k) {
+            const int i = st * kPagesPerStage + k;
+            const int pg = from_global ? checked(__ldg(table + page_lo + i)) : s_pages[i];
+            const int y = (pg * p.H_kv + g) * 16;
+#pragma unroll
+            for (int bx = 0; bx < BOXES; ++bx) {
+                tma_load_2d(kb + k * L::kPageBytes + bx * 2048, &tmap_k, bx * 64, y, &s_bar[slot]);
+                tma_load_2d(vb + k * L::kPageBytes + bx * 2048, &tmap_v, bx * 64, y, &s_bar[slot]);
+            }
+        }
+    };
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&s_bar[s], 1);
+            s_count[s] = 0;
+            s_issued[s] = 0;
+        }
+        *s_abort = 0;
+        fence_barrier_init();
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+        // the first stages go out before anything else (their page ids straight from global)
+        for (int st = 0; st < min(STAGES - 1, n_stages); ++st)
+            issue(st, true);
     }
+    for (int i = tid; i < n_pages; i += kThreads)
+        s_pages[i] = checked(__ldg(table + page_lo + i));
     for (int i = tid; i < kRowsPerCta * CH; i += kThreads) {
         const int r = i / CH, c = i % CH;
         uint4 v = make_uint4(0, 0, 0, 0);
@@ -184,36 +207,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4 *>(s_q + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
     }
     __syncthreads();
-
-    auto page_id = [&](int i) -> int {
-        if (i < kMaxTablePages)
-            return s_pages[i];
-        int pg = __ldg(table + page_lo + i);
-        if (pg < 0 || pg >= p.num_blocks) {
-            set_status(p.status, PA_ERR_BOUNDS);
-            pg = static_cast<int>(p.num_blocks);
-        }
-        return pg;
-    };
-    auto issue = [&](int st) {  // thread 0 only
-        const int slot = st % STAGES;
-        uint8_t *kb = s_stage + slot * L::kStageBytes;
-        uint8_t *vb = kb + kPagesPerStage * L::kPageBytes;
-        const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&s_bar[slot], np * 2 * L::kPageBytes);
-        for (int k = 0; k < np; ++k) {
-            const int y = (page_id(st * kPagesPerStage + k) * p.H_kv + g) * 16;
-#pragma unroll
-            for (int bx = 0; bx < BOXES; ++bx) {
-                tma_load_2d(kb + k * L::kPageBytes + bx * 2048, &tmap_k, bx * 64, y, &s_bar[slot]);
-                tma_load_2d(vb + k * L::kPageBytes + bx * 2048, &tmap_v, bx * 64, y, &s_bar[slot]);
-            }
-        }
-    };
-    if (tid == 0)
-        for (int st = 0; st < min(STAGES, n_stages); ++st)
-            issue(st);
 
     // ---- per-thread row state --------------------------------------------------------------
     // This thread holds rows ra = lane/4 and rb = ra + 8 of its warp's m-tile.
@@ -232,6 +225,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ldsm_x4(smem_u32(s_q + r * (D * 2) + ((c ^ (r & 7)) << 4)), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
         }
     }
+    __syncthreads();  // Q is in registers: the last stage buffer can be loaded
+    if (tid == 0 && STAGES - 1 < n_stages)
+        issue(STAGES - 1, false);
     float o[NT][4];
 #pragma unroll
     for (int i = 0; i < NT; ++i)
@@ -351,17 +347,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-        __syncthreads();  // every warp is done with this slot
+        // the last warp done with this slot refills it
+        __syncwarp();
+        if (lane == 0 && atomicAdd(&s_count[slot], 1) == 3) {
+            s_count[slot] = 0;
+            if (it + STAGES < n_stages && !*s_abort)
+                issue(it + STAGES, false);
+        }
         if (*s_abort)
             break;
-        if (tid == 0 && it + STAGES < n_stages)
-            issue(it + STAGES);
     }
+    __syncthreads();
     if (*s_abort) {
         // let the copies still in flight land (bounded) before the CTA releases its shared memory
         if (tid == 0)
-            for (int st = it; st < min(it + STAGES, n_stages); ++st)
-                mbar_wait(&s_bar[st % STAGES], (st / STAGES) & 1, kWaitTimeoutNs / 10);
+            for (int s = 0; s < STAGES; ++s)
+                if (s_issued[s] > 0)
+                    mbar_wait(&s_bar[s], (s_issued[s] - 1) & 1, kWaitTimeoutNs / 10);
         return;
     }
 
@@ -482,7 +484,7 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
 
 // ---- host side ------------------------------------------------------------------------------
 
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 
 template <int D, bool BF16>
 static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
@@ -543,7 +545,7 @@ DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
         sp = kMaxTablePages;
     const int ov = split_pages_override();
     if (ov > 0)
-        sp = ov;
+        sp = ov < kMaxTablePages ? ov : kMaxTablePages;
     pl.split_pages = static_cast<int>(sp);
     pl.max_splits = pages > 0 ? static_cast<int>((pages + sp - 1) / sp) : 1;
     return pl;
@@ -563,7 +565,7 @@ size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
 }
 
 template <int D, bool BF16>
-static int run(const AttnArgs &a, bool decode)
+static int run(const AttnArgs &a)
 {
     CUtensorMap tk, tv;
     int rc = make_cache_tmap(&tk, a.key_cache, a.num_blocks, a.H_kv, D, a.dtype);
@@ -588,8 +590,7 @@ static int run(const AttnArgs &a, bool decode)
     rp.max_ctx = a.max_ctx;
     rp.max_q_len = a.max_q_len;
     rp.scale_log2 = a.scale * 1.4426950408889634f;
-    rp.decode = decode ? 1 : 0;
-    if (decode) {
+    {
         const DecodePlan pl = decode_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx);
         rp.n_rg = pl.row_groups;
         rp.split_pages = pl.split_pages;
@@ -607,22 +608,13 @@ static int run(const AttnArgs &a, bool decode)
             rc = launch_merge<D, BF16>(rp, a.stream);
         return rc;
     }
-    const int G = a.H_q / a.H_kv;
-    rp.n_rg = static_cast<int>(((int64_t)a.max_q_len * G + kRowsPerCta - 1) / kRowsPerCta);
-    rp.split_pages = 1 << 30;
-    if (a.B > 65535 || a.H_kv > 65535)
-        return PA_ERR_UNSUPPORTED;
-    dim3 grid(rp.n_rg, a.H_kv, a.B);
-    return launch_rows<D, BF16>(rp, tk, tv, grid, a.stream);
 }
 
-static int dispatch(const AttnArgs &a, bool decode)
+int launch_decode(const AttnArgs &a)
 {
     if (a.d == 128)
-        return a.dtype == PA_BF16 ? run<128, true>(a, decode) : run<128, false>(a, decode);
-    return a.dtype == PA_BF16 ? run<64, true>(a, decode) : run<64, false>(a, decode);
+        return a.dtype == PA_BF16 ? run<128, true>(a) : run<128, false>(a);
+    return a.dtype == PA_BF16 ? run<64, true>(a) : run<64, false>(a);
 }
-
-int launch_decode(const AttnArgs &a) { return dispatch(a, true); }
 
 }  // namespace pa
