@@ -293,23 +293,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (it < 0 || !ok)
                 break;
             const int32_t *table = p.block_tables + (int64_t)I.b * p.max_blocks;
-            if (lane == 0) {
-                // Q tiles first: they do not need the page table
-                const Tile *tl[2] = {&I.A, &I.Bt};
-#pragma unroll
-                for (int x = 0; x < 2; ++x) {
-                    if (!ok || !tl[x]->on)
-                        continue;
-                    ok = wait_bar(&q_empty[x], free_par(q_n[x]), abort_flag, p.status);
-                    if (!ok)
-                        break;
-                    uint8_t *qs = smem + L::kQ + x * L::kTile;
-                    mbar_arrive_expect_tx(&q_full[x], KB * p.rows_per_tile * 128);
-                    for (int kb = 0; kb < KB; ++kb)
-                        tc::tma_load_3d(qs + kb * kRows * 128, &tmap_q, kb * 64, I.g * p.G, I.q0 + tl[x]->t_begin,
-                                        &q_full[x]);
-                    ++q_n[x];
-                }
+            // Q_A goes out first (its buffer frees early: the previous item's last S_A comes before
+            // its last S_B); Q_B is slipped in between K/V tiles as soon as its buffer is free, so
+            // the next item's K/V loads do not wait for the current item's last S_B
+            auto load_q = [&](int x, const Tile &tq) {
+                uint8_t *qs = smem + L::kQ + x * L::kTile;
+                mbar_arrive_expect_tx(&q_full[x], KB * p.rows_per_tile * 128);
+                for (int kb = 0; kb < KB; ++kb)
+                    tc::tma_load_3d(qs + kb * kRows * 128, &tmap_q, kb * 64, I.g * p.G, I.q0 + tq.t_begin, &q_full[x]);
+                ++q_n[x];
+            };
+            bool qb_pending = I.Bt.on;
+            if (lane == 0 && ok) {
+                ok = wait_bar(&q_empty[0], free_par(q_n[0]), abort_flag, p.status);
+                if (ok)
+                    load_q(0, I.A);
             }
             // page ids of the item into shared memory
             for (int i = lane; i < min(I.n_pages, kMaxTable); i += 32) {
@@ -324,6 +322,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) {
                 // K and V tiles, interleaved
                 for (int j = 0; j < I.n_kv && ok; ++j) {
+                    if (qb_pending && mbar_test(&q_empty[1], free_par(q_n[1]))) {
+                        load_q(1, I.Bt);
+                        qb_pending = false;
+                    }
                     int y[8];
 #pragma unroll
                     for (int pg = 0; pg < 8; ++pg) {
@@ -363,6 +365,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kb = 0; kb < KB; ++kb)
                             tma_load_2d(vdst + kb * kRows * 128 + pg * 2048, &tmap_v, kb * 64, y[pg], &v_full[vs]);
+                }
+                if (ok && qb_pending) {
+                    ok = wait_bar(&q_empty[1], free_par(q_n[1]), abort_flag, p.status);
+                    if (ok)
+                        load_q(1, I.Bt);
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -411,12 +418,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nt[2] = {I.A.n_kv, I.Bt.n_kv};  // 0 for a tile without tokens
                 const int n = I.n_kv;
                 const uint32_t q_addr[2] = {smem_u32(smem + L::kQ), smem_u32(smem + L::kQ + L::kTile)};
-#pragma unroll
-                for (int x = 0; x < 2; ++x)
-                    if (ok && nt[x] > 0) {
-                        ok = wait_bar(&q_full[x], full_par(q_n[x]), abort_flag, p.status);
-                        ++q_n[x];
-                    }
                 int qk_i[2] = {0, 0}, pv_i[2] = {0, 0};  // next S / next P V product per tile
                 int k_rel = 0, v_rel = 0;                // K / V tiles of this item released
                 uint64_t t_last = globaltimer();
@@ -455,7 +456,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int jq = qk_i[x];
                         if (jq < nt[x] && pv_i[x] == jq) {
                             const int kg = k_base + jq;
-                            if (mbar_test(&k_full[kg % kStages], full_par(kg / kStages))) {
+                            if (mbar_test(&k_full[kg % kStages], full_par(kg / kStages)) &&
+                                (jq > 0 || mbar_test(&q_full[x], full_par(q_n[x])))) {
+                                if (jq == 0)
+                                    ++q_n[x];
                                 tc::fence_after_sync();
                                 const uint32_t k_addr = smem_u32(smem + L::kK + (kg % kStages) * L::kTile);
                                 const uint32_t d = tmem + 128u * x;
