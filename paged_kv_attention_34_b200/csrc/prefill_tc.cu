@@ -25,15 +25,18 @@
 //     shared memory, fp32 accumulator in TMEM.  O_X is rescaled only when a
 //     row's max grows by more than 2^8 (exact: the same stale max is used for
 //     P and for l, and O / l is taken once at the end);
-//   * tensor-core issue order per K/V tile j: S_A(j), O_B += P_B(j-1) V(j-1),
-//     S_B(j), O_A += P_A(j) V(j).  Each S_X(j+1) is issued after the P_X(j) V
-//     product that reads the same TMEM columns; tcgen05.mma operations of one
-//     thread execute in issue order, which makes that reuse safe;
-//   * warp 0 issues TMA and hands out work items from a global counter,
-//     heaviest first (later query tiles see more keys); warp 1 allocates TMEM
-//     and issues the MMAs (warps 2-3 idle; the first warpgroup shrinks its register
-//     budget so the softmax warpgroups can grow theirs); warps 4-7 and 8-11 are the
-//     two softmax warpgroups (rescale and epilogue included).  One persistent CTA per SM.
+//   * the MMAs of tile X are issued by one thread of their own (warp 0 for A, warp 1 for B), in
+//     the order S_X(j), O_X += P_X(j) V_j, S_X(j+1), ...; S_X(j+1) goes after the product that
+//     reads the TMEM columns it overwrites (tcgen05.mma operations of one thread execute in issue
+//     order), and the two threads feed the tensor core independently, so one tile's products run
+//     while the other tile's softmax runs;
+//   * warp 2 hands out work items from a global counter, heaviest first (later query tiles see
+//     more keys), loads the Q tiles and feeds the K ring; warp 3 feeds the V ring and clears the
+//     V rows past the context end in the tile that holds it (P is 0 there, but 0 * NaN is NaN);
+//     lanes 0-7 each fetch one page of a tile (one thread issuing all boxes of a tile is limited
+//     by the per-instruction issue cost of TMA).  The first warpgroup shrinks its register budget
+//     so the softmax warpgroups can grow theirs; warps 4-7 and 8-11 are the two softmax
+//     warpgroups (rescale and epilogue included).  One persistent CTA per SM.
 // All waits are bounded; a wait that runs out records PA_ERR_TIMEOUT and the
 // CTA winds down (its copies and MMAs in flight are waited for, TMEM freed).
 #include <cmath>
@@ -48,16 +51,15 @@ namespace tcp {
 constexpr int kRows = 128;     // query rows per tile (TMEM lanes)
 constexpr int kKeys = 128;     // keys per K/V tile
 constexpr int kStages = 2;     // depth of the K ring and of the V ring
-constexpr int kThreads = 384;  // 3 warpgroups: scheduler/TMA/MMA, softmax A, softmax B
+constexpr int kThreads = 384;  // 3 warpgroups: MMA/TMA/scheduling, softmax A, softmax B
 // Register budgets: launched at 168 per thread (65536 / 384, rounded to 8); the first warpgroup
-// gives registers back, the softmax warpgroups take them: 128 * 80 + 256 * 208 <= 384 * 168.
+// gives registers back, the softmax warpgroups take them: 128 * 104 + 256 * 200 <= 384 * 168.
 constexpr int kLaunchRegs = 168;
-constexpr uint32_t kRegsControl = 88;
-constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsControl = 104;
+constexpr uint32_t kRegsSoftmax = 200;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split over budget");
-constexpr int kMaxTable = 1024;
 constexpr int kItemSlots = 2;
-constexpr int kItemReaders = 9;  // warp 1 and warps 4-11 each acknowledge a work item
+constexpr int kItemReaders = 11;  // warps 0, 1, 3 and 4-11 each acknowledge a work item
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr size_t kCounterOffset = 64;      // work counter inside the status area of the workspace
 
@@ -111,9 +113,8 @@ struct Smem {
     static constexpr int kQ = 0;                     // Q_A, Q_B
     static constexpr int kK = 2 * kTile;             // K ring
     static constexpr int kV = kK + kStages * kTile;  // V ring
-    static constexpr int kTable = kV + kStages * kTile;
-    static constexpr int kBars = kTable + 4 * kMaxTable;
-    static constexpr int kNumBars = 2 * 2 + 4 * kStages + 5 * 2 + 2 * kItemSlots + 1;
+    static constexpr int kBars = kV + kStages * kTile;
+    static constexpr int kNumBars = 2 * 2 + 4 * kStages + 4 * 2 + 2 * kItemSlots + 2;
     static constexpr int kItems = kBars + 8 * kNumBars;
     static constexpr int kTmemSlot = kItems + ((int(sizeof(ItemSlot)) * kItemSlots + 15) / 16) * 16;
     static constexpr int kAbort = kTmemSlot + 8;
@@ -200,21 +201,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *q_full = bars;                    // [2] Q_X landed
     uint64_t *q_empty = bars + 2;               // [2] Q_X no longer read
     uint64_t *k_full = bars + 4;                // [kStages]
-    uint64_t *k_empty = k_full + kStages;       // [kStages]
+    uint64_t *k_empty = k_full + kStages;       // [kStages] released by both MMA threads
     uint64_t *v_full = k_empty + kStages;       // [kStages]
-    uint64_t *v_empty = v_full + kStages;       // [kStages]
+    uint64_t *v_empty = v_full + kStages;       // [kStages] released by both MMA threads
     uint64_t *s_full = v_empty + kStages;       // [2] S_X computed
     uint64_t *p_full = s_full + 2;              // [2] P_X written (128 arrivals)
-    uint64_t *pv_done = p_full + 2;             // [2] O_X += P_X V completed
-    uint64_t *o_full = pv_done + 2;             // [2] O_X final for the item
+    uint64_t *o_full = p_full + 2;              // [2] O_X final for the item
     uint64_t *o_free = o_full + 2;              // [2] epilogue of X has read O_X (128 arrivals)
     uint64_t *item_full = o_free + 2;           // [kItemSlots]
     uint64_t *item_empty = item_full + kItemSlots;
-    uint64_t *drain = item_empty + kItemSlots;  // [1]
+    uint64_t *drain = item_empty + kItemSlots;  // [1] both MMA threads' products complete
+    uint64_t *v_land = drain + 1;               // [1] V tile with a context end landed (before zeroing)
     ItemSlot *item_slot = reinterpret_cast<ItemSlot *>(smem + L::kItems);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kAbort);
-    int32_t *s_table = reinterpret_cast<int32_t *>(smem + L::kTable);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -224,28 +224,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&q_empty[x], 1);
             mbar_init(&s_full[x], 1);
             mbar_init(&p_full[x], 128);
-            mbar_init(&pv_done[x], 1);
             mbar_init(&o_full[x], 1);
             mbar_init(&o_free[x], 128);
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&k_full[i], 1);
-            mbar_init(&k_empty[i], 1);
+            mbar_init(&k_empty[i], 2);
             mbar_init(&v_full[i], 1);
-            mbar_init(&v_empty[i], 1);
+            mbar_init(&v_empty[i], 2);
         }
         for (int i = 0; i < kItemSlots; ++i) {
             mbar_init(&item_full[i], 1);
             mbar_init(&item_empty[i], kItemReaders);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);
+        mbar_init(v_land, 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_q);
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_v);
     }
-    if (warp == 1) {
+    if (warp == 0) {
         tc::tmem_alloc(tmem_slot, kTmemCols);
         tc::tmem_relinquish();
     }
@@ -258,147 +258,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < 4) {
     // first warpgroup: give registers back (all four warps), then split into roles
     tc::regs_shrink<kRegsControl>();
-    if (warp == 0) {
-        // ===================== scheduler + TMA producer =====================
-        int n_pub = 0, k_n = 0, v_n = 0, q_n[2] = {0, 0};
-        bool ok = true;
-        for (;;) {
-            // next work item that has query tokens (lane 0 draws, the warp follows)
-            int it = -1;
-            Item I;
-            for (;;) {
-                // lane 0 decides for the whole warp (the abort flag may change between lanes' reads)
-                int cand = -1;
-                if (lane == 0 && ok && !*abort_flag)
-                    cand = atomicAdd(p.counter, 1);
-                cand = __shfl_sync(0xffffffffu, cand, 0);
-                if (cand < 0 || cand >= p.n_items)
-                    break;
-                if (get_item(p, cand, I, lane == 0)) {
-                    it = cand;
-                    break;
-                }
-            }
-            // publish it (or the end marker -1) to the other roles
-            if (lane == 0) {
-                const int slot = n_pub % kItemSlots;
-                const bool got = wait_bar(&item_empty[slot], free_par(n_pub / kItemSlots), abort_flag, p.status);
-                ok = ok && got;
-                item_slot[slot].it = ok ? it : -1;
-                item_slot[slot].I = I;
-                mbar_arrive(&item_full[slot]);
-            }
-            ++n_pub;
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (it < 0 || !ok)
-                break;
-            const int32_t *table = p.block_tables + (int64_t)I.b * p.max_blocks;
-            // Q_A goes out first (its buffer frees early: the previous item's last S_A comes before
-            // its last S_B); Q_B is slipped in between K/V tiles as soon as its buffer is free, so
-            // the next item's K/V loads do not wait for the current item's last S_B
-            auto load_q = [&](int x, const Tile &tq) {
-                uint8_t *qs = smem + L::kQ + x * L::kTile;
-                mbar_arrive_expect_tx(&q_full[x], KB * p.rows_per_tile * 128);
-                for (int kb = 0; kb < KB; ++kb)
-                    tc::tma_load_3d(qs + kb * kRows * 128, &tmap_q, kb * 64, I.g * p.G, I.q0 + tq.t_begin, &q_full[x]);
-                ++q_n[x];
-            };
-            bool qb_pending = I.Bt.on;
-            if (lane == 0 && ok) {
-                ok = wait_bar(&q_empty[0], free_par(q_n[0]), abort_flag, p.status);
-                if (ok)
-                    load_q(0, I.A);
-            }
-            // page ids of the item into shared memory
-            for (int i = lane; i < min(I.n_pages, kMaxTable); i += 32) {
-                int pg = __ldg(table + i);
-                if (pg < 0 || pg >= p.num_blocks) {
-                    set_status(p.status, PA_ERR_BOUNDS);
-                    pg = -1;
-                }
-                s_table[i] = pg;
-            }
-            __syncwarp();
-            if (lane == 0) {
-                // K and V tiles, interleaved
-                for (int j = 0; j < I.n_kv && ok; ++j) {
-                    if (qb_pending && mbar_test(&q_empty[1], free_par(q_n[1]))) {
-                        load_q(1, I.Bt);
-                        qb_pending = false;
-                    }
-                    int y[8];
-#pragma unroll
-                    for (int pg = 0; pg < 8; ++pg) {
-                        const int pidx = j * 8 + pg;
-                        y[pg] = p.oob_row;  // pages past the item's range: zero-filled by TMA
-                        if (pidx < I.n_pages) {
-                            int id = pidx < kMaxTable ? s_table[pidx] : __ldg(table + pidx);
-                            if (id >= p.num_blocks)
-                                id = -1;
-                            if (id >= 0)
-                                y[pg] = (id * p.H_kv + I.g) * 16;
-                            else
-                                set_status(p.status, PA_ERR_BOUNDS);
-                        }
-                    }
-                    const int ks = k_n % kStages;
-                    ok = wait_bar(&k_empty[ks], free_par(k_n / kStages), abort_flag, p.status);
-                    if (!ok)
-                        break;
-                    uint8_t *kdst = smem + L::kK + ks * L::kTile;
-                    mbar_arrive_expect_tx(&k_full[ks], L::kTile);
-                    ++k_n;
-#pragma unroll
-                    for (int pg = 0; pg < 8; ++pg)
-#pragma unroll
-                        for (int kb = 0; kb < KB; ++kb)
-                            tma_load_2d(kdst + kb * kRows * 128 + pg * 2048, &tmap_k, kb * 64, y[pg], &k_full[ks]);
-                    const int vs = v_n % kStages;
-                    ok = wait_bar(&v_empty[vs], free_par(v_n / kStages), abort_flag, p.status);
-                    if (!ok)
-                        break;
-                    uint8_t *vdst = smem + L::kV + vs * L::kTile;
-                    mbar_arrive_expect_tx(&v_full[vs], L::kTile);
-                    ++v_n;
-#pragma unroll
-                    for (int pg = 0; pg < 8; ++pg)
-#pragma unroll
-                        for (int kb = 0; kb < KB; ++kb)
-                            tma_load_2d(vdst + kb * kRows * 128 + pg * 2048, &tmap_v, kb * 64, y[pg], &v_full[vs]);
-                }
-                if (ok && qb_pending) {
-                    ok = wait_bar(&q_empty[1], free_par(q_n[1]), abort_flag, p.status);
-                    if (ok)
-                        load_q(1, I.Bt);
-                }
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            k_n = __shfl_sync(0xffffffffu, k_n, 0);
-            v_n = __shfl_sync(0xffffffffu, v_n, 0);
-            q_n[0] = __shfl_sync(0xffffffffu, q_n[0], 0);
-            q_n[1] = __shfl_sync(0xffffffffu, q_n[1], 0);
-            __syncwarp();
-        }
-        if (lane == 0 && *abort_flag) {
-            // let the copies already issued land before shared memory is released
-            for (int s = 0; s < kStages; ++s) {
-                const int k_uses = k_n / kStages + (s < k_n % kStages ? 1 : 0);
-                const int v_uses = v_n / kStages + (s < v_n % kStages ? 1 : 0);
-                if (k_uses > 0)
-                    mbar_wait(&k_full[s], full_par(k_uses - 1), kWaitTimeoutNs / 10);
-                if (v_uses > 0)
-                    mbar_wait(&v_full[s], full_par(v_uses - 1), kWaitTimeoutNs / 10);
-            }
-        }
-    } else if (warp == 1) {
-        // ===================== MMA issuer =====================
-        // Event driven: every product is issued as soon as its inputs are ready, so one slow
-        // softmax tile does not hold back the other tile's products.  Per tile, S_X(j+1) is
-        // issued only after P_X(j) V (in-order execution keeps the TMEM reuse safe); a K (V) tile
-        // is released once every S (P V) product that reads it has been issued.
+    if (warp < 2) {
+        // ===================== MMA issuers: warp 0 for tile A, warp 1 for tile B (one thread each) =====================
+        // Per K/V tile j: S_X(j) = Q_X K_j^T, then O_X += P_X(j) V_j once the softmax has written P_X(j);
+        // S_X(j+1) is issued after that product, which reads the TMEM columns S_X(j+1) overwrites
+        // (tcgen05.mma operations of one thread execute in issue order).  The two threads feed the
+        // tensor core independently, so one tile's waits overlap the other tile's products.  Each
+        // thread releases every K and V tile of the item (the empty barriers count two arrivals),
+        // always after waiting for the tile to land, so that neither can arrive twice on a stage
+        // before the other has arrived once.
+        const int x = warp;
         constexpr uint32_t idesc_qk = tc::idesc_f16(BF16, kRows, kKeys, false);
         constexpr uint32_t idesc_pv = tc::idesc_f16(BF16, kRows, D, true);
-        int n_item = 0, k_base = 0, q_n[2] = {0, 0}, pv_n[2] = {0, 0}, o_n[2] = {0, 0};
+        const uint32_t q_addr = smem_u32(smem + L::kQ + x * L::kTile);
+        const uint32_t s_tm = tmem + 128u * x;
+        const uint32_t o_tm = tmem + 256u + 128u * x;
+        int n_item = 0, k_base = 0, q_n = 0, pv_n = 0, o_n = 0;
         bool ok = true;
         for (;;) {
             const int slot = n_item % kItemSlots;
@@ -415,101 +290,83 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (it < 0)
                 break;
             if (lane == 0) {
-                const int nt[2] = {I.A.n_kv, I.Bt.n_kv};  // 0 for a tile without tokens
+                const int nt = x == 0 ? I.A.n_kv : I.Bt.n_kv;  // 0 for a tile without tokens
                 const int n = I.n_kv;
-                const uint32_t q_addr[2] = {smem_u32(smem + L::kQ), smem_u32(smem + L::kQ + L::kTile)};
-                int qk_i[2] = {0, 0}, pv_i[2] = {0, 0};  // next S / next P V product per tile
-                int k_rel = 0, v_rel = 0;                // K / V tiles of this item released
-                uint64_t t_last = globaltimer();
-                while (ok) {
-                    bool progress = false;
+                auto wait_k = [&](int j) {
+                    const int kg = k_base + j;
+                    return wait_bar(&k_full[kg % kStages], full_par(kg / kStages), abort_flag, p.status);
+                };
+                auto wait_v = [&](int j) {
+                    const int vg = k_base + j;
+                    return wait_bar(&v_full[vg % kStages], full_par(vg / kStages), abort_flag, p.status);
+                };
+                // S_X(j) = Q_X K_j^T
+                auto issue_s = [&](int j) {
+                    const uint32_t k_addr = smem_u32(smem + L::kK + ((k_base + j) % kStages) * L::kTile);
 #pragma unroll
-                    for (int x = 0; x < 2; ++x) {
-                        // O_X += P_X(j) V_j
-                        const int j = pv_i[x];
-                        // on the item's last V tile, tile A goes first (it clears the tail rows)
-                        const bool order_ok = !(x == 1 && j == n - 1 && nt[0] == n && pv_i[0] < n);
-                        if (j < qk_i[x] && order_ok) {
-                            const int vg = k_base + j;
-                            if (mbar_test(&p_full[x], full_par(pv_n[x])) &&
-                                mbar_test(&v_full[vg % kStages], full_par(vg / kStages)) &&
-                                (j > 0 || mbar_test(&o_free[x], free_par(o_n[x])))) {
-                                tc::fence_after_sync();
-                                const uint32_t v_addr = smem_u32(smem + L::kV + (vg % kStages) * L::kTile);
-                                const uint32_t d = tmem + 256u + 128u * x;
-                                const uint32_t a = tmem + 128u * x;
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
+                        tc::mma_ss(s_tm, tc::desc_k_sw128(q_addr + off), tc::desc_k_sw128(k_addr + off), idesc_qk,
+                                   ks > 0 ? 1u : 0u);
+                    }
+                    tc::commit(&s_full[x]);
+                    if (j == nt - 1)
+                        tc::commit(&q_empty[x]);  // Q_X no longer needed
+                };
+                // O_X += P_X(j) V_j
+                auto issue_pv = [&](int j) {
+                    const uint32_t v_addr = smem_u32(smem + L::kV + ((k_base + j) % kStages) * L::kTile);
 #pragma unroll
-                                for (int ks = 0; ks < kKeys / 16; ++ks)
-                                    tc::mma_ts(d, a + ks * 8, tc::desc_mn_sw128(v_addr + ks * 2048, kRows * 128),
-                                               idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-                                tc::commit(&pv_done[x]);
-                                ++pv_n[x];
-                                ++pv_i[x];
-                                if (pv_i[x] == nt[x]) {
-                                    tc::commit(&o_full[x]);
-                                    ++o_n[x];
-                                }
-                                progress = true;
-                            }
-                        }
-                        // S_X(j) = Q_X K_j^T, once P_X(j-1) V has been issued
-                        const int jq = qk_i[x];
-                        if (jq < nt[x] && pv_i[x] == jq) {
-                            const int kg = k_base + jq;
-                            if (mbar_test(&k_full[kg % kStages], full_par(kg / kStages)) &&
-                                (jq > 0 || mbar_test(&q_full[x], full_par(q_n[x])))) {
-                                if (jq == 0)
-                                    ++q_n[x];
-                                tc::fence_after_sync();
-                                const uint32_t k_addr = smem_u32(smem + L::kK + (kg % kStages) * L::kTile);
-                                const uint32_t d = tmem + 128u * x;
-#pragma unroll
-                                for (int ks = 0; ks < D / 16; ++ks) {
-                                    const uint32_t off = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
-                                    tc::mma_ss(d, tc::desc_k_sw128(q_addr[x] + off), tc::desc_k_sw128(k_addr + off),
-                                               idesc_qk, ks > 0 ? 1u : 0u);
-                                }
-                                tc::commit(&s_full[x]);
-                                ++qk_i[x];
-                                if (qk_i[x] == nt[x])
-                                    tc::commit(&q_empty[x]);  // Q_X no longer needed
-                                progress = true;
-                            }
+                    for (int ks = 0; ks < kKeys / 16; ++ks)
+                        tc::mma_ts(o_tm, s_tm + ks * 8, tc::desc_mn_sw128(v_addr + ks * 2048, kRows * 128), idesc_pv,
+                                   (j > 0 || ks > 0) ? 1u : 0u);
+                    ++pv_n;
+                    if (j == nt - 1) {
+                        tc::commit(&o_full[x]);
+                        ++o_n;
+                    }
+                };
+                ok = wait_k(0);
+                if (ok && nt > 0) {
+                    ok = wait_bar(&q_full[x], full_par(q_n), abort_flag, p.status);
+                    if (ok) {
+                        ++q_n;
+                        tc::fence_after_sync();
+                        issue_s(0);
+                    }
+                }
+                if (ok)
+                    tc::commit(&k_empty[k_base % kStages]);
+                for (int j = 0; j < n && ok; ++j) {
+                    // V_j and K_(j+1) are normally in place long before P_X(j): check them first
+                    ok = wait_v(j);
+                    if (ok && j + 1 < n)
+                        ok = wait_k(j + 1);
+                    if (ok && j < nt) {
+                        ok = wait_bar(&p_full[x], full_par(pv_n), abort_flag, p.status);
+                        if (ok && j == 0)
+                            ok = wait_bar(&o_free[x], free_par(o_n), abort_flag, p.status);
+                        if (ok) {
+                            tc::fence_after_sync();
+                            issue_pv(j);
                         }
                     }
-                    // release the K and V tiles that no further product of this item reads
-                    while (k_rel < n && (k_rel >= nt[0] || qk_i[0] > k_rel) && (k_rel >= nt[1] || qk_i[1] > k_rel)) {
-                        tc::commit(&k_empty[(k_base + k_rel) % kStages]);
-                        ++k_rel;
-                    }
-                    while (v_rel < n && (v_rel >= nt[0] || pv_i[0] > v_rel) && (v_rel >= nt[1] || pv_i[1] > v_rel)) {
-                        tc::commit(&v_empty[(k_base + v_rel) % kStages]);
-                        ++v_rel;
-                    }
-                    if (pv_i[0] == nt[0] && pv_i[1] == nt[1])
-                        break;  // every product of the item is issued
-                    if (progress) {
-                        t_last = globaltimer();
-                    } else {
-                        if (*abort_flag) {
-                            ok = false;
-                        } else if (globaltimer() - t_last > kWaitTimeoutNs) {
-                            *abort_flag = 1;
-                            set_status(p.status, PA_ERR_TIMEOUT);
-                            ok = false;
-                        }
+                    if (!ok)
+                        break;
+                    tc::commit(&v_empty[(k_base + j) % kStages]);
+                    if (j + 1 < n) {
+                        if (j + 1 < nt)
+                            issue_s(j + 1);
+                        tc::commit(&k_empty[(k_base + j + 1) % kStages]);
                     }
                 }
                 k_base += n;
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             k_base = __shfl_sync(0xffffffffu, k_base, 0);
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                q_n[x] = __shfl_sync(0xffffffffu, q_n[x], 0);
-                pv_n[x] = __shfl_sync(0xffffffffu, pv_n[x], 0);
-                o_n[x] = __shfl_sync(0xffffffffu, o_n[x], 0);
-            }
+            q_n = __shfl_sync(0xffffffffu, q_n, 0);
+            pv_n = __shfl_sync(0xffffffffu, pv_n, 0);
+            o_n = __shfl_sync(0xffffffffu, o_n, 0);
             if (!ok)
                 break;
         }
@@ -519,6 +376,165 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(drain, 0, kWaitTimeoutNs / 10);
         }
         __syncwarp();
+    } else {
+        // ===================== producers: warp 2 = scheduler + Q + K ring, warp 3 = V ring =====================
+        // One TMA box is 16 keys x 64 columns of one page; lanes 0-7 each fetch one page of a tile
+        // (one thread issuing every box of a tile is limited by the per-instruction issue cost).
+        const bool is_v = warp == 3;
+        const CUtensorMap *tmap = is_v ? &tmap_v : &tmap_k;
+        uint64_t *full = is_v ? v_full : k_full;
+        uint64_t *empty = is_v ? v_empty : k_empty;
+        uint8_t *ring = smem + (is_v ? L::kV : L::kK);
+        int n_item = 0, n_tiles = 0, q_n[2] = {0, 0}, z_n = 0;
+        bool ok = true;
+        for (;;) {
+            int it = -1;
+            Item I;
+            if (!is_v) {
+                // next work item that has query tokens (lane 0 draws, the warp follows)
+                for (;;) {
+                    // lane 0 decides for the whole warp (the abort flag may change between lanes' reads)
+                    int cand = -1;
+                    if (lane == 0 && ok && !*abort_flag)
+                        cand = atomicAdd(p.counter, 1);
+                    cand = __shfl_sync(0xffffffffu, cand, 0);
+                    if (cand < 0 || cand >= p.n_items)
+                        break;
+                    if (get_item(p, cand, I, lane == 0)) {
+                        it = cand;
+                        break;
+                    }
+                }
+                // publish it (or the end marker -1) to the other roles
+                if (lane == 0) {
+                    const int slot = n_item % kItemSlots;
+                    const bool got = wait_bar(&item_empty[slot], free_par(n_item / kItemSlots), abort_flag, p.status);
+                    ok = ok && got;
+                    item_slot[slot].it = ok ? it : -1;
+                    item_slot[slot].I = I;
+                    mbar_arrive(&item_full[slot]);
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok)
+                    it = -1;
+            } else {
+                const int slot = n_item % kItemSlots;
+                ok = wait_bar(&item_full[slot], full_par(n_item / kItemSlots), abort_flag, p.status);
+                ok = __all_sync(0xffffffffu, ok);
+                it = ok ? item_slot[slot].it : -1;
+                if (it >= 0)
+                    I = item_slot[slot].I;
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&item_empty[slot]);
+            }
+            ++n_item;
+            if (it < 0)
+                break;
+            const int32_t *table = p.block_tables + (int64_t)I.b * p.max_blocks;
+            // TMA row of page `pidx` of the item (lanes 0-7); pages past the item's range, and bad
+            // block ids, read rows past the pool, which TMA fills with zeros
+            auto page_row = [&](int pidx) -> int {
+                int y = p.oob_row;
+                if (lane < 8 && pidx < I.n_pages) {
+                    const int id = __ldg(table + pidx);
+                    if (id >= 0 && id < p.num_blocks)
+                        y = (id * p.H_kv + I.g) * 16;
+                    else
+                        set_status(p.status, PA_ERR_BOUNDS);
+                }
+                return y;
+            };
+            // The last page of the context may be partly filled: its V rows past the context end can
+            // hold anything (NaN included) and P is 0 there, but 0 * NaN is NaN, so the V warp clears
+            // them before the tile is handed on.  That happens only when this item reads up to the
+            // context end.
+            const int last_page = (I.ctx + 15) / 16 - 1;
+            const int zpg = last_page - 8 * (I.n_kv - 1);  // page of the last tile holding the context end
+            const int zr0 = I.ctx & 15;                   // first row to clear
+            const bool zero_tail = is_v && zr0 != 0 && I.n_pages == last_page + 1 && zpg >= 0 && zpg < 8;
+            int y = page_row(lane);
+            for (int j = 0; j < I.n_kv; ++j) {
+                const int y_next = j + 1 < I.n_kv ? page_row((j + 1) * 8 + lane) : p.oob_row;  // in flight meanwhile
+                const int st = n_tiles % kStages;
+                const bool z = zero_tail && j == I.n_kv - 1;
+                uint64_t *done = z ? v_land : &full[st];
+                if (lane == 0) {
+                    ok = wait_bar(&empty[st], free_par(n_tiles / kStages), abort_flag, p.status);
+                    if (ok)
+                        mbar_arrive_expect_tx(done, L::kTile);
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok)
+                    break;
+                ++n_tiles;
+                uint8_t *dst = ring + st * L::kTile;
+                if (lane < 8) {
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb)
+                        tma_load_2d(dst + lane * 2048 + kb * kRows * 128, tmap, kb * 64, y, done);
+                }
+                y = y_next;
+                if (z) {
+                    ++z_n;
+                    ok = wait_bar(v_land, full_par(z_n - 1), abort_flag, p.status);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok)
+                        break;
+                    const int per_kb = (16 - zr0) * 8;  // 16-byte chunks to clear per column block
+                    for (int i = lane; i < per_kb * KB; i += 32) {
+                        const int kb = i / per_kb, rem = i % per_kb;
+                        const int row = zpg * 16 + zr0 + rem / 8;
+                        *reinterpret_cast<uint4 *>(dst + kb * kRows * 128 + row * 128 + (rem & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();  // generic writes before the tensor core reads the tile
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&full[st]);
+                }
+                if (!is_v && j == 0) {
+                    // Q_A and Q_B of the item, after its first K tile
+                    if (lane == 0) {
+#pragma unroll
+                        for (int xq = 0; xq < 2 && ok; ++xq) {
+                            const Tile &tq = xq == 0 ? I.A : I.Bt;
+                            if (!tq.on)
+                                continue;
+                            ok = wait_bar(&q_empty[xq], free_par(q_n[xq]), abort_flag, p.status);
+                            if (!ok)
+                                break;
+                            uint8_t *qs = smem + L::kQ + xq * L::kTile;
+                            mbar_arrive_expect_tx(&q_full[xq], KB * p.rows_per_tile * 128);
+                            for (int kb = 0; kb < KB; ++kb)
+                                tc::tma_load_3d(qs + kb * kRows * 128, &tmap_q, kb * 64, I.g * p.G,
+                                                I.q0 + tq.t_begin, &q_full[xq]);
+                            ++q_n[xq];
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    q_n[0] = __shfl_sync(0xffffffffu, q_n[0], 0);
+                    q_n[1] = __shfl_sync(0xffffffffu, q_n[1], 0);
+                    if (!ok)
+                        break;
+                }
+            }
+            if (!ok)
+                break;
+        }
+        if (lane == 0 && *abort_flag) {
+            // let the copies already issued land before shared memory is released
+            for (int st = 0; st < kStages; ++st) {
+                const int uses = n_tiles / kStages + (st < n_tiles % kStages ? 1 : 0);
+                if (uses > 0)
+                    mbar_wait(&full[st], full_par(uses - 1), kWaitTimeoutNs / 10);
+            }
+            if (z_n > 0)
+                mbar_wait(v_land, full_par(z_n - 1), kWaitTimeoutNs / 10);
+            for (int xq = 0; xq < 2; ++xq)
+                if (q_n[xq] > 0)
+                    mbar_wait(&q_full[xq], full_par(q_n[xq] - 1), kWaitTimeoutNs / 10);
+        }
     }
     } else {
         tc::regs_grow<kRegsSoftmax>();
@@ -530,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t s_tmem = tmem + lane_addr + 128u * x;
         const uint32_t o_tmem = tmem + lane_addr + 256u + 128u * x;
         const float sl2 = p.scale_log2;
-        int n_item = 0, s_n = 0, pv_n = 0, o_n = 0, kv_base = 0;
+        int n_item = 0, s_n = 0, o_n = 0;
         bool ok = true;
         for (;;) {
             const int slot = n_item % kItemSlots;
@@ -546,22 +562,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_item;
             if (it < 0)
                 break;
-            const int kv_first = kv_base;  // index of this item's first K/V tile in the producer's order
-            kv_base += I.n_kv;
             const Tile &t = x == 0 ? I.A : I.Bt;
             if (!t.on)
                 continue;
             const int tl = r / p.G, gi = r % p.G;
             const bool row_valid = r < p.rows_per_tile && tl < t.n_tok;
             const int lim = row_valid ? I.ctx - I.qb + t.t_begin + tl : -1;
-            // the warpgroup whose P V first reads the item's last V tile clears the keys past the
-            // context end in it (P is 0 there, but 0 * NaN is NaN); everything it needs is fixed here
-            const int last_page = (I.ctx + 15) / 16 - 1;
-            const int zpg = last_page - 8 * (I.n_kv - 1);
-            const bool do_zero = ((x == 0) == (I.A.n_kv == I.n_kv)) && sub == 0 && (I.ctx & 15) &&
-                                 I.n_pages == last_page + 1 && zpg >= 0 && zpg < 8;
-            const int zr0 = I.ctx & 15;
-            const int zvn = kv_first + I.n_kv - 1;  // V load index of the item's last K/V step
             const int n_kv_t = t.n_kv;
             uint8_t *orow = static_cast<uint8_t *>(p.out) +
                             ((int64_t)(I.q0 + t.t_begin + tl) * p.H_q + I.g * p.G + gi) * (D * 2);
@@ -603,11 +609,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     grow = true;
                 }
                 if (__any_sync(0xffffffffu, grow)) {
-                    // O_X must hold every earlier P V product before it is rescaled
-                    ok = wait_bar(&pv_done[x], full_par(pv_n - 1), abort_flag, p.status);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok)
-                        break;
+                    // every earlier P V product of this tile is complete: S_X(j) was issued after them
+                    // by the same thread, and its completion (s_full) covers them
                     tc::fence_after_sync();
 #pragma unroll 1
                     for (int c = 0; c < D / 16; ++c) {
@@ -643,29 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::st32(s_tmem, raw);
                 tc::st32(s_tmem + 32, raw + 32);
                 tc::wait_st();
-                ++pv_n;  // the P V product of this tile
-                if (do_zero && j == n_kv_t - 1) {
-                    const int vstage = zvn % kStages;
-                    bool landed = wait_bar(&v_full[vstage], full_par(zvn / kStages), abort_flag, p.status);
-                    landed = __all_sync(0xffffffffu, landed);
-                    if (landed) {
-                        uint8_t *vsm = smem + L::kV + vstage * L::kTile;
-                        const int per_kb = (16 - zr0) * 8;  // 16-byte chunks to clear per column block
-                        for (int i = lane; i < per_kb * KB; i += 32) {
-                            const int kb = i / per_kb, rem = i % per_kb;
-                            const int row = zpg * 16 + zr0 + rem / 8;
-                            *reinterpret_cast<uint4 *>(vsm + kb * kRows * 128 + row * 128 + (rem & 7) * 16) =
-                                make_uint4(0, 0, 0, 0);
-                        }
-                        fence_proxy_async_smem();
-                    }
-                    __syncwarp();
-                    ok = landed;
-                }
                 tc::fence_before_sync();
                 mbar_arrive(&p_full[x]);
-                if (!ok)
-                    break;
             }
             if (!ok)
                 break;
@@ -704,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 1)
+    if (warp == 0)
         tc::tmem_dealloc(tmem, kTmemCols);
 }
 
