@@ -114,7 +114,7 @@ struct Smem {
     static constexpr int kK = 2 * kTile;             // K ring
     static constexpr int kV = kK + kStages * kTile;  // V ring
     static constexpr int kBars = kV + kStages * kTile;
-    static constexpr int kNumBars = 2 * 2 + 4 * kStages + 4 * 2 + 2 * kItemSlots + 2;
+    static constexpr int kNumBars = 2 * 2 + 4 * kStages + 4 * 2 + 2 * kItemSlots + 4;
     static constexpr int kItems = kBars + 8 * kNumBars;
     static constexpr int kTmemSlot = kItems + ((int(sizeof(ItemSlot)) * kItemSlots + 15) / 16) * 16;
     static constexpr int kAbort = kTmemSlot + 8;
@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *item_empty = item_full + kItemSlots;
     uint64_t *drain = item_empty + kItemSlots;  // [1] both MMA threads' products complete
     uint64_t *v_land = drain + 1;               // [1] V tile with a context end landed (before zeroing)
+    uint64_t *tok = v_land + 1;                 // [2] tok[X]: MMA thread X may issue its next batch
     ItemSlot *item_slot = reinterpret_cast<ItemSlot *>(smem + L::kItems);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kAbort);
@@ -239,6 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(drain, 2);
         mbar_init(v_land, 1);
+        mbar_init(&tok[0], 1);
+        mbar_init(&tok[1], 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&tmap_q);
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t q_addr = smem_u32(smem + L::kQ + x * L::kTile);
         const uint32_t s_tm = tmem + 128u * x;
         const uint32_t o_tm = tmem + 256u + 128u * x;
-        int n_item = 0, k_base = 0, q_n = 0, pv_n = 0, o_n = 0;
+        int n_item = 0, k_base = 0, q_n = 0, pv_n = 0, o_n = 0, n_batch = 0;
         bool ok = true;
         for (;;) {
             const int slot = n_item % kItemSlots;
@@ -326,19 +329,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ++o_n;
                     }
                 };
+                // Batch 0 of the item is S_X(0); batch j + 1 is P_X(j) V_j followed by S_X(j + 1).  The
+                // two threads issue their batches in turn (a token passed through tok[]), every
+                // thread n + 1 batches per item (empty ones where its tile has fewer K/V tiles), so the
+                // tensor core runs one tile's batch while the other tile's softmax runs.  All waits
+                // for data come before the token is taken.
+                auto take_turn = [&]() {
+                    const uint32_t par = x == 0 ? free_par(n_batch) : full_par(n_batch);
+                    return wait_bar(&tok[x], par, abort_flag, p.status);
+                };
+                auto pass_turn = [&]() {
+                    mbar_arrive(&tok[x ^ 1]);
+                    ++n_batch;
+                };
                 ok = wait_k(0);
                 if (ok && nt > 0) {
                     ok = wait_bar(&q_full[x], full_par(q_n), abort_flag, p.status);
-                    if (ok) {
-                        ++q_n;
+                    ++q_n;
+                }
+                if (ok)
+                    ok = take_turn();
+                if (ok) {
+                    if (nt > 0) {
                         tc::fence_after_sync();
                         issue_s(0);
                     }
-                }
-                if (ok)
+                    pass_turn();
                     tc::commit(&k_empty[k_base % kStages]);
+                }
                 for (int j = 0; j < n && ok; ++j) {
-                    // V_j and K_(j+1) are normally in place long before P_X(j): check them first
+                    // V_j and K_(j+1) are normally in place long before P_X(j)
                     ok = wait_v(j);
                     if (ok && j + 1 < n)
                         ok = wait_k(j + 1);
@@ -346,19 +366,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = wait_bar(&p_full[x], full_par(pv_n), abort_flag, p.status);
                         if (ok && j == 0)
                             ok = wait_bar(&o_free[x], free_par(o_n), abort_flag, p.status);
-                        if (ok) {
-                            tc::fence_after_sync();
-                            issue_pv(j);
-                        }
                     }
+                    if (ok)
+                        ok = take_turn();
                     if (!ok)
                         break;
-                    tc::commit(&v_empty[(k_base + j) % kStages]);
-                    if (j + 1 < n) {
+                    if (j < nt) {
+                        tc::fence_after_sync();
+                        issue_pv(j);
                         if (j + 1 < nt)
                             issue_s(j + 1);
-                        tc::commit(&k_empty[(k_base + j + 1) % kStages]);
                     }
+                    pass_turn();
+                    tc::commit(&v_empty[(k_base + j) % kStages]);
+                    if (j + 1 < n)
+                        tc::commit(&k_empty[(k_base + j + 1) % kStages]);
                 }
                 k_base += n;
             }
@@ -367,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             q_n = __shfl_sync(0xffffffffu, q_n, 0);
             pv_n = __shfl_sync(0xffffffffu, pv_n, 0);
             o_n = __shfl_sync(0xffffffffu, o_n, 0);
+            n_batch = __shfl_sync(0xffffffffu, n_batch, 0);
             if (!ok)
                 break;
         }
