@@ -340,33 +340,38 @@ def run_ours(args):
 
 
 def run_e2e(st, w, args, stream, device, step_bytes):
-    """The step with host buffers: H2D of the step inputs (pinned), the calls, D2H of the output."""
+    """The step with host buffers: H2D of the step inputs (pinned), the calls, D2H of the output.
+
+    The inputs of a step (Q, the new K/V rows, slot mapping, block table, context lengths,
+    cu_seqlens) are staged in one pinned host buffer and sent with one copy into one device
+    buffer, whose views the library calls take; the output comes back with one copy.
+    """
     import torch
+    from paged_kv_attention_34_b200 import kv_cache_write, paged_attn_decode
 
     call = st.calls[0]
-    host = {
-        "q": w.q.pin_memory(),
-        "k_new": w.k_new.pin_memory(),
-        "v_new": w.v_new.pin_memory(),
-        "slot": w.slot_mapping.pin_memory(),
-        "bt": call.bt.cpu().pin_memory(),
-        "ctx": call.ctx.cpu().pin_memory(),
-        "cu": call.cu.cpu().pin_memory(),
-    }
+    parts = [("q", w.q), ("k_new", w.k_new), ("v_new", w.v_new), ("slot", w.slot_mapping),
+             ("bt", call.bt.cpu()), ("ctx", call.ctx.cpu()), ("cu", call.cu.cpu())]
+    offs, off = {}, 0
+    for name, t in parts:
+        offs[name] = off
+        off += (t.numel() * t.element_size() + 255) // 256 * 256
+    host_buf = torch.zeros(off, dtype=torch.uint8).pin_memory()
+    dev_buf = torch.empty(off, dtype=torch.uint8, device=device)
+    views = {}
+    for name, t in parts:
+        n = t.numel() * t.element_size()
+        host_buf[offs[name]:offs[name] + n].copy_(t.contiguous().view(-1).view(torch.uint8))
+        views[name] = dev_buf[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
     out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = off
     d2h = out_host.numel() * out_host.element_size()
 
     def one():
-        st.q.copy_(host["q"], non_blocking=True)
-        st.k_new.copy_(host["k_new"], non_blocking=True)
-        st.v_new.copy_(host["v_new"], non_blocking=True)
-        st.slot_mapping.copy_(host["slot"], non_blocking=True)
-        call.bt.copy_(host["bt"], non_blocking=True)
-        call.ctx.copy_(host["ctx"], non_blocking=True)
-        call.cu.copy_(host["cu"], non_blocking=True)
-        st.write()
-        st.attend(call)
+        dev_buf.copy_(host_buf, non_blocking=True)
+        kv_cache_write(views["k_new"], views["v_new"], views["slot"], st.key_cache, st.value_cache, status=st.status)
+        paged_attn_decode(views["q"], st.key_cache, st.value_cache, views["bt"], views["cu"], views["ctx"],
+                          call.max_ctx, w.scale, out=st.out, workspace=call.ws)
         out_host.copy_(st.out, non_blocking=True)
 
     with torch.cuda.stream(stream):

@@ -102,7 +102,9 @@ int pa_kv_block_copy(void *key_cache, void *value_cache, int64_t num_blocks, int
 
 /*
  * pa_decode_workspace_bytes -- device workspace that pa_paged_attn_decode needs
- * for these sizes (status word + split-KV partial outputs and log-sum-exps).
+ * for these sizes: the status word area, the order in which the sequences are
+ * scheduled (B int32, most pages first, written by the call itself), and with
+ * more than one KV split the split-KV partial outputs and log-sum-exps.
  * Pure host function.  Returns 0 for invalid sizes.
  */
 size_t pa_decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx);
@@ -115,7 +117,10 @@ size_t pa_decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int
  * split keeps its own running max / sum and the splits are merged by
  * log-sum-exp in a second kernel on the same stream ("FlashDecoding" answer
  * of the interview Q&A page: split the long KV sequence over blocks, local
- * softmax per block, then a cross-block reduction).
+ * softmax per block, then a cross-block reduction).  A one-CTA kernel first orders the
+ * sequences by page count, longest first, so that the CTAs of the longest
+ * sequences start first and short ones fill the last wave; the order changes
+ * no result.
  *   out          [T][H_q][d] written (same dtype as q)
  *   q            [T][H_q][d], T = cu_seqlens_q[B]
  *   cu_seqlens_q [B+1], each q_b in 1..8      context_lens [B], q_b <= ctx_b <= max_ctx
@@ -162,8 +167,10 @@ int pa_paged_attn_decode_noalloc(void *out, const void *q, const void *key_cache
                                  void *stream);
 
 /*
- * pa_prefill_workspace_bytes -- device workspace of pa_paged_attn_prefill
- * (status word and the tile scheduler's state).  Pure host function.
+ * pa_prefill_workspace_bytes -- device workspace of pa_paged_attn_prefill:
+ * the status word area (with the work counter of the tile scheduler) and the
+ * order in which the (query-tile pair, sequence) work is handed out, written
+ * by the call itself (most K/V tiles first).  Pure host function.
  */
 size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len);
 

@@ -43,6 +43,7 @@ struct RowsParams {
     const int32_t *context_lens;
     float *ws_o;    // [max_splits][T][H_q][D] normalised partial outputs
     float *ws_lse;  // [max_splits][T][H_q] log2-sum-exp of the scaled scores
+    const int32_t *order;  // [B] sequences by decreasing page count: grid z -> sequence
     int32_t *status;
     int64_t num_blocks;
     int64_t T;
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // ---- which (sequence, KV head, row group, split) --------------------------------
-    const int b = blockIdx.z;
+    const int b = __ldg(p.order + blockIdx.z);
     const int split = blockIdx.x;
     const int g = blockIdx.y / p.n_rg, rg = blockIdx.y % p.n_rg;
     const int q0 = __ldg(p.cu_seqlens + b), q1 = __ldg(p.cu_seqlens + b + 1);
@@ -507,6 +508,28 @@ static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtens
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// Longest sequences first: decode CTAs are dispatched in grid order, so putting the sequences with
+// the most pages at the front leaves short CTAs for the last wave (longest-processing-time-first
+// list scheduling; the order among equal page counts is arbitrary and changes no result).
+__global__ void __launch_bounds__(kOrderThreads) pa_seq_order_kernel(const int32_t *context_lens, int B, int32_t *order)
+{
+    order_by_key_desc(
+        B,
+        [&](int b) {
+            const int ctx = __ldg(context_lens + b);
+            const int pages = ctx > 0 ? (ctx + 15) / 16 : 0;
+            return min(pages, kOrderKeys - 1);
+        },
+        order);
+}
+
+int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, cudaStream_t stream)
+{
+    pa_seq_order_kernel<<<1, kOrderThreads, 0, stream>>>(context_lens, B, order);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 template <int D, bool BF16>
 static int launch_merge(const RowsParams &rp, cudaStream_t stream)
 {
@@ -551,10 +574,14 @@ DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
     return pl;
 }
 
+// Workspace: status word area, the sequence order, then (with more than one split) the partial
+// outputs and their log-sum-exps.
+size_t seq_order_bytes(int B) { return (static_cast<size_t>(B) * sizeof(int32_t) + 255) / 256 * 256; }
+
 size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx)
 {
     const DecodePlan pl = decode_plan(B, H_q, H_kv, d, max_ctx);
-    size_t bytes = PA_STATUS_BYTES;
+    size_t bytes = PA_STATUS_BYTES + seq_order_bytes(B);
     if (pl.max_splits > 1) {
         const size_t rows = static_cast<size_t>(pl.max_splits) * static_cast<size_t>(T) * H_q;
         bytes += rows * d * sizeof(float);
@@ -594,16 +621,20 @@ static int run(const AttnArgs &a)
         const DecodePlan pl = decode_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx);
         rp.n_rg = pl.row_groups;
         rp.split_pages = pl.split_pages;
+        int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES);
+        rp.order = order;
         if (pl.max_splits > 1) {
             const size_t rows = static_cast<size_t>(pl.max_splits) * static_cast<size_t>(a.T) * a.H_q;
-            uint8_t *ws = static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES;
+            uint8_t *ws = static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES + seq_order_bytes(a.B);
             rp.ws_o = reinterpret_cast<float *>(ws);
             rp.ws_lse = reinterpret_cast<float *>(ws + rows * D * sizeof(float));
         }
         if (a.B > 65535 || (int64_t)a.H_kv * pl.row_groups > 65535)
             return PA_ERR_UNSUPPORTED;
         dim3 grid(pl.max_splits, a.H_kv * pl.row_groups, a.B);
-        rc = launch_rows<D, BF16>(rp, tk, tv, grid, a.stream);
+        rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
+        if (rc == PA_OK)
+            rc = launch_rows<D, BF16>(rp, tk, tv, grid, a.stream);
         if (rc == PA_OK && pl.max_splits > 1)
             rc = launch_merge<D, BF16>(rp, a.stream);
         return rc;

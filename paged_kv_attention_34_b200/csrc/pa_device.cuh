@@ -245,4 +245,65 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
     return v;
 }
 
+// ---- longest-first ordering -------------------------------------------------------------------
+
+constexpr int kOrderKeys = 4096;
+constexpr int kOrderThreads = 1024;
+
+// One CTA of kOrderThreads threads, all of which call this: order[r] = the element of rank r when
+// the n elements are sorted by decreasing key_of(e) in [0, kOrderKeys) (a counting sort; elements
+// with equal keys in arbitrary order).
+template <class KeyOf>
+__device__ void order_by_key_desc(int n, KeyOf key_of, int32_t *order)
+{
+    __shared__ int cnt[kOrderKeys];
+    __shared__ int warp_tot[kOrderThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < kOrderKeys; i += kOrderThreads)
+        cnt[i] = 0;
+    __syncthreads();
+    for (int e = tid; e < n; e += kOrderThreads)
+        atomicAdd(&cnt[key_of(e)], 1);
+    __syncthreads();
+    // exclusive prefix sum in descending key order: thread t owns keys kOrderKeys-1-PER*t downwards
+    constexpr int PER = kOrderKeys / kOrderThreads;
+    int v[PER], run = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        v[i] = cnt[kOrderKeys - 1 - (tid * PER + i)];
+        run += v[i];
+    }
+    int incl = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    if (lane == 31)
+        warp_tot[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int t = warp_tot[lane];
+        int ti = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o)
+                ti += y;
+        }
+        warp_tot[lane] = ti - t;  // exclusive over warps
+    }
+    __syncthreads();
+    int base = warp_tot[warp] + incl - run;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        cnt[kOrderKeys - 1 - (tid * PER + i)] = base;
+        base += v[i];
+    }
+    __syncthreads();
+    for (int e = tid; e < n; e += kOrderThreads)
+        order[atomicAdd(&cnt[key_of(e)], 1)] = e;
+}
+
 }  // namespace pa

@@ -65,7 +65,12 @@ struct DecodePlan {
 DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx);
 size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx);
 
+// Sequence order by decreasing page count (one CTA, on `stream`): order[r] = the sequence of rank r.
+// The workspace holds it right after the status area, seq_order_bytes(B) bytes.
+size_t seq_order_bytes(int B);
+int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, cudaStream_t stream);
 int launch_decode(const AttnArgs &a);
+size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int max_q_len);
 int launch_prefill(const AttnArgs &a);
 
 }  // namespace pa

@@ -30,8 +30,9 @@
 //     reads the TMEM columns it overwrites (tcgen05.mma operations of one thread execute in issue
 //     order), and the two threads feed the tensor core independently, so one tile's products run
 //     while the other tile's softmax runs;
-//   * warp 2 hands out work items from a global counter, heaviest first (later query tiles see
-//     more keys), loads the Q tiles and feeds the K ring; warp 3 feeds the V ring and clears the
+//   * warp 2 hands out work items from a global counter, heaviest first (sequences with the most
+//     pages first, and within one the later query tiles, which see more keys), loads the Q tiles
+//     and feeds the K ring; warp 3 feeds the V ring and clears the
 //     V rows past the context end in the tile that holds it (P is 0 there, but 0 * NaN is NaN);
 //     lanes 0-7 each fetch one page of a tile (one thread issuing all boxes of a tile is limited
 //     by the per-instruction issue cost of TMA).  The first warpgroup shrinks its register budget
@@ -67,6 +68,7 @@ struct Params {
     const int32_t *block_tables;
     const int32_t *cu_seqlens;
     const int32_t *context_lens;
+    const int32_t *order;  // [n_pairs_max * B] (pair, sequence) entries by decreasing K/V tiles
     void *out;
     int32_t *status;
     int *counter;
@@ -130,14 +132,42 @@ __device__ __forceinline__ void make_tile(const Params &p, const Item &I, int qt
     t.n_kv = t.on ? (I.ctx - I.qb + t.t_begin + t.n_tok - 1) / kKeys + 1 : 0;
 }
 
-// Decode work item `it`; false when it has no query token (or its sequence is invalid).
+// K/V tiles read by query-tile pair `pair` of a sequence (0 when it has no query token or the
+// sequence's lengths are invalid): the work of its items.
+__device__ __forceinline__ int pair_kv_tiles(int pair, int qb, int ctx, int tok_per_tile)
+{
+    const int64_t t0 = 2ll * pair * tok_per_tile;
+    if (qb < 1 || ctx < qb || t0 >= qb)
+        return 0;
+    const int64_t end = t0 + 2 * tok_per_tile;
+    const int last = static_cast<int>(end < qb ? end : qb) - 1;
+    return (ctx - qb + last) / kKeys + 1;
+}
+
+// Longest-processing-time-first order of the work: the (pair, sequence) entries by decreasing
+// K/V tiles, so the heaviest items are drawn first and short ones fill the end.
+__global__ void __launch_bounds__(kOrderThreads) pa_prefill_order_kernel(const int32_t *cu_seqlens,
+                                                                           const int32_t *context_lens, int B,
+                                                                           int n_pairs, int tok_per_tile, int32_t *order)
+{
+    order_by_key_desc(
+        n_pairs * B,
+        [&](int e) {
+            const int b = e % B;
+            const int qb = __ldg(cu_seqlens + b + 1) - __ldg(cu_seqlens + b);
+            return min(pair_kv_tiles(e / B, qb, __ldg(context_lens + b), tok_per_tile), kOrderKeys - 1);
+        },
+        order);
+}
+
+// Decode work item `it` (the KV heads of one entry of the order are consecutive items); false when
+// it has no query token (or its sequence is invalid).
 __device__ __forceinline__ bool get_item(const Params &p, int it, Item &I, bool report)
 {
-    const int per = p.B * p.H_kv;
-    const int pair = p.n_pairs_max - 1 - it / per;  // heaviest first
-    const int rem = it % per;
-    I.b = rem / p.H_kv;
-    I.g = rem % p.H_kv;
+    const int e = __ldg(p.order + it / p.H_kv);
+    const int pair = e / p.B;
+    I.b = e % p.B;
+    I.g = it % p.H_kv;
     I.q0 = __ldg(p.cu_seqlens + I.b);
     const int q1 = __ldg(p.cu_seqlens + I.b + 1);
     I.qb = q1 - I.q0;
@@ -729,6 +759,8 @@ static int run(const AttnArgs &a)
     p.out = a.out;
     p.status = static_cast<int32_t *>(a.workspace);
     p.counter = reinterpret_cast<int *>(static_cast<uint8_t *>(a.workspace) + kCounterOffset);
+    int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES);
+    p.order = order;
     p.num_blocks = a.num_blocks;
     p.T = a.T;
     p.max_blocks = a.max_blocks;
@@ -760,6 +792,11 @@ static int run(const AttnArgs &a)
         return rc;
     if (cudaMemsetAsync(p.counter, 0, sizeof(int), a.stream) != cudaSuccess)
         return PA_ERR_CUDA;
+    pa_prefill_order_kernel<<<1, kOrderThreads, 0, a.stream>>>(a.cu_seqlens_q, a.context_lens, a.B, p.n_pairs_max,
+                                                                 p.tok_per_tile, order);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess)
+        return PA_ERR_CUDA;
 
     auto kern = pa_prefill_tc_kernel<D, BF16>;
     static uint64_t configured = 0;
@@ -786,6 +823,15 @@ static int run(const AttnArgs &a)
 }
 
 }  // namespace tcp
+
+// Workspace: the status area (status word, work counter), then the (pair, sequence) order.
+size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int max_q_len)
+{
+    const int G = H_q / H_kv;
+    const int tok = G >= 1 && G <= tcp::kRows ? tcp::kRows / G : 1;
+    const int64_t n_pairs = ((int64_t)(max_q_len + tok - 1) / tok + 1) / 2;
+    return PA_STATUS_BYTES + (static_cast<size_t>(n_pairs) * B * sizeof(int32_t) + 255) / 256 * 256;
+}
 
 int launch_prefill(const AttnArgs &a)
 {

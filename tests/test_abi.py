@@ -117,9 +117,11 @@ def test_prefill_rejects_bad_args(L):
 
 
 def test_workspace_queries(L):
-    # one split needs only the status word; long contexts need partials
+    # one split needs the status word and the sequence order (B int32 in 256-byte units);
+    # long contexts need partials
     small = pa.decode_workspace_bytes(3, 3, 4, 4, 64, 50)
-    assert small == pa.PA_STATUS_BYTES
+    assert small == pa.PA_STATUS_BYTES + 256
+    assert pa.decode_workspace_bytes(3, 65, 4, 4, 64, 50) == pa.PA_STATUS_BYTES + 512
     big = pa.decode_workspace_bytes(16, 16, 64, 8, 128, 32768)
     assert big > pa.PA_STATUS_BYTES
     # monotone in T and max_ctx
