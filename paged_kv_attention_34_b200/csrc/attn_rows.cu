@@ -552,20 +552,30 @@ static int split_pages_override()
 
 DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
 {
-    (void)d;
     DecodePlan pl;
     const int G = H_q / H_kv;
     pl.row_groups = (8 * G + kRowsPerCta - 1) / kRowsPerCta;
     const int64_t pages = (int64_t)(max_ctx + 15) / 16;
-    // Aim for about 8 waves of CTAs over the SMs (2 resident per SM), never
-    // fewer than 16 pages (256 keys) per split; a multiple of the stage size.
+    // Pages per split: the multiple of the stage size in [16, kMaxTablePages] that minimises the
+    // time of a batch whose every sequence has max_ctx keys, modelled as (full waves of CTAs over
+    // 2 per SM) x (split length + a per-CTA cost of ~80 KB of streaming, in pages).  Longer
+    // splits mean fewer CTAs and less fixed cost; the wave count rounds up, so a split that fills
+    // the last wave beats a slightly shorter one that leaves it nearly empty.
     const int64_t units = (int64_t)B * H_kv * pl.row_groups;
-    const int64_t slots = (int64_t)sm_count() * 2 * 8;
-    int64_t sp = units > 0 ? (units * pages + slots - 1) / slots : pages;
-    sp = sp < 16 ? 16 : sp;
-    sp = (sp + kPagesPerStage - 1) / kPagesPerStage * kPagesPerStage;
-    if (sp > kMaxTablePages)
-        sp = kMaxTablePages;
+    const int64_t slots = (int64_t)sm_count() * 2;
+    const int64_t page_bytes = 2 * 16 * (int64_t)d * 2;
+    const int64_t cta_cost = (80 * 1024 + page_bytes - 1) / page_bytes;
+    int64_t sp = kMaxTablePages, best = -1;
+    for (int64_t c = kMaxTablePages; c >= 16 && units > 0 && pages > 0; c -= kPagesPerStage) {
+        const int64_t ctas = units * ((pages + c - 1) / c);
+        const int64_t waves = (ctas + slots - 1) / slots;
+        const int64_t len = c < pages ? c : pages;
+        const int64_t cost = waves * (len + cta_cost);
+        if (best < 0 || cost < best) {
+            best = cost;
+            sp = c;
+        }
+    }
     const int ov = split_pages_override();
     if (ov > 0)
         sp = ov < kMaxTablePages ? ov : kMaxTablePages;
