@@ -226,3 +226,50 @@ def test_repeat_runs_identical():
     b = st.run().clone()
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def _ws_order(ws: torch.Tensor, n: int) -> np.ndarray:
+    """The scheduling order the call wrote after the status area of its workspace."""
+    return ws[pa.PA_STATUS_BYTES:pa.PA_STATUS_BYTES + 4 * n].cpu().view(torch.int32).numpy()
+
+
+def test_decode_schedules_longest_sequences_first():
+    # decode writes the sequences in non-increasing page count: a permutation of 0..B-1
+    w = W.config2(B=48)
+    st = DeviceStep(w)
+    st.run()
+    torch.cuda.synchronize()
+    call = st.calls[0]
+    B = call.ctx.shape[0]
+    order = _ws_order(call.ws, B)
+    assert sorted(order.tolist()) == list(range(B))
+    pages = np.minimum((call.ctx.cpu().numpy() + 15) // 16, 4095)
+    assert np.all(np.diff(pages[order]) <= 0)
+
+
+def test_prefill_schedules_heaviest_work_first():
+    # prefill writes the (query-tile pair, sequence) entries by non-increasing K/V tiles
+    w = W.config5()
+    st = DeviceStep(w)
+    st.run()
+    torch.cuda.synchronize()
+    call = next(c for c in st.calls if c.kind == "prefill")
+    q = (call.cu[1:] - call.cu[:-1]).cpu().numpy()
+    ctx = call.ctx.cpu().numpy()
+    B = q.shape[0]
+    tok = 128 // (w.H_q // w.H_kv)
+    n_pairs = ((call.max_q_len + tok - 1) // tok + 1) // 2
+    order = _ws_order(call.ws, n_pairs * B)
+    assert sorted(order.tolist()) == list(range(n_pairs * B))
+
+    def tiles(e):
+        pair, b = e // B, e % B
+        t0 = 2 * pair * tok
+        if t0 >= q[b]:
+            return 0
+        last = min(q[b], t0 + 2 * tok) - 1
+        return (ctx[b] - q[b] + last) // 128 + 1
+
+    keys = np.array([min(tiles(int(e)), 4095) for e in order])
+    assert np.all(np.diff(keys) <= 0)
+    assert keys[0] == max(tiles(e) for e in range(n_pairs * B))
