@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return pg;
     };
-    auto issue = [&](int st, bool from_global) {  // one thread
+    auto issue = [&](int st) {  // one thread; the page ids from the shared-memory copy
         const int slot = st % STAGES;
         uint8_t *kb = s_stage + slot * L::kStageBytes;
         uint8_t *vb = kb + kPagesPerStage * L::kPageBytes;
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         s_issued[slot] += 1;
         for (int k = 0; k < np; ++k) {
             const int i = st * kPagesPerStage + k;
-            const int pg = from_global ? checked(__ldg(table + page_lo + i)) : s_pages[i];
+            const int pg = s_pages[i];
             const int y = (pg * p.H_kv + g) * 16;
 #pragma unroll
             for (int bx = 0; bx < BOXES; ++bx) {
@@ -180,19 +180,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     };
-    if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&s_bar[s], 1);
-            s_count[s] = 0;
-            s_issued[s] = 0;
+    if (warp == 0) {
+        // the first stages go out before anything else: lane i < (STAGES - 1) * 4 reads the id of
+        // page i straight from the table in global memory and issues that page's boxes, so the
+        // id loads overlap instead of following one another
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&s_bar[s], 1);
+                s_count[s] = 0;
+                s_issued[s] = 0;
+            }
+            *s_abort = 0;
+            fence_barrier_init();
+            prefetch_tmap(&tmap_k);
+            prefetch_tmap(&tmap_v);
         }
-        *s_abort = 0;
-        fence_barrier_init();
-        prefetch_tmap(&tmap_k);
-        prefetch_tmap(&tmap_v);
-        // the first stages go out before anything else (their page ids straight from global)
-        for (int st = 0; st < min(STAGES - 1, n_stages); ++st)
-            issue(st, true);
+        const int first = min(STAGES - 1, n_stages);
+        const int i = lane;
+        const bool mine = i < first * kPagesPerStage && i < n_pages;
+        const int pg = mine ? checked(__ldg(table + page_lo + i)) : 0;
+        __syncwarp();
+        if (lane == 0) {
+            for (int st = 0; st < first; ++st) {
+                const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
+                mbar_arrive_expect_tx(&s_bar[st], np * 2 * L::kPageBytes);
+                s_issued[st] += 1;
+            }
+        }
+        __syncwarp();
+        if (mine) {
+            const int st = i / kPagesPerStage, k = i % kPagesPerStage;
+            uint8_t *kb = s_stage + st * L::kStageBytes;
+            uint8_t *vb = kb + kPagesPerStage * L::kPageBytes;
+            const int y = (pg * p.H_kv + g) * 16;
+#pragma unroll
+            for (int bx = 0; bx < BOXES; ++bx) {
+                tma_load_2d(kb + k * L::kPageBytes + bx * 2048, &tmap_k, bx * 64, y, &s_bar[st]);
+                tma_load_2d(vb + k * L::kPageBytes + bx * 2048, &tmap_v, bx * 64, y, &s_bar[st]);
+            }
+        }
     }
     for (int i = tid; i < n_pages; i += kThreads)
         s_pages[i] = checked(__ldg(table + page_lo + i));
@@ -228,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();  // Q is in registers: the last stage buffer can be loaded
     if (tid == 0 && STAGES - 1 < n_stages)
-        issue(STAGES - 1, false);
+        issue(STAGES - 1);
     float o[NT][4];
 #pragma unroll
     for (int i = 0; i < NT; ++i)
@@ -353,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && atomicAdd(&s_count[slot], 1) == 3) {
             s_count[slot] = 0;
             if (it + STAGES < n_stages && !*s_abort)
-                issue(it + STAGES, false);
+                issue(it + STAGES);
         }
         if (*s_abort)
             break;
