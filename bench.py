@@ -20,8 +20,10 @@ The same JSON line carries:
   prefill       causal varlen prefill (8 prompts U[256,2048], 40/40 heads, bf16):
                 TFLOP/s of exact causal pairs vs the measured bf16 peak
   legs          the GQA shared-prefix decode step and the mixed continuous-batching step
-  e2e           the same metric with host buffers: pinned H2D of the step inputs and
-                D2H of the output inside the timed region
+  e2e           the same metric with host buffers: every step's inputs go H2D from one pinned
+                buffer and its output comes back D2H, all inside the timed region; the copies
+                run on a second stream, overlapping the neighbouring steps' kernels (double-
+                buffered device inputs and outputs), as a serving loop would
   cpu_baseline  the fp64 CPU oracle, timed on a bounded sample of the same workload
   clocks        SM clock / throttle reasons sampled through NVML during the timed region
 
@@ -193,6 +195,21 @@ def time_calls(fn_list, steps, stream):
     return start.elapsed_time(end), per
 
 
+def time_steps(fn_list, steps, stream):
+    """Run `steps` iterations of the step between two CUDA events on `stream`; elapsed ms."""
+    import torch
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            for fn in fn_list:
+                fn()
+        end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
 def bench_leg(w, steps, warmup, stream, device):
     """Time one workload's step (copy, write, attention calls) with per-call events."""
     import torch
@@ -261,10 +278,16 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    n_launch0 = pa.launch_count()
     with ClockSampler(local_rank) as clk:
-        total_ms, per = time_calls(fns, args.steps, stream)
-    n_launch = pa.launch_count() - n_launch0
+        # per-call durations (CUDA events around every call), then the timed steps themselves with
+        # events only at the two ends, so the step time carries no per-call event overhead
+        _, per = time_calls(fns, args.steps, stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        n_launch0 = pa.launch_count()
+        total_ms = time_steps(fns, args.steps, stream)
+        n_launch = pa.launch_count() - n_launch0
     torch.cuda.synchronize()
     barrier()
     total_ms_max = reduce_max(total_ms, device)
@@ -343,8 +366,12 @@ def run_e2e(st, w, args, stream, device, step_bytes):
     """The step with host buffers: H2D of the step inputs (pinned), the calls, D2H of the output.
 
     The inputs of a step (Q, the new K/V rows, slot mapping, block table, context lengths,
-    cu_seqlens) are staged in one pinned host buffer and sent with one copy into one device
-    buffer, whose views the library calls take; the output comes back with one copy.
+    cu_seqlens) are staged in one pinned host buffer and sent with one copy into one of two device
+    buffers, whose views the library calls take; the output goes to one of two device buffers and
+    comes back with one copy.  The copies run on a copy stream ordered by events: step k's inputs
+    land before its kernels start, step k+1's inputs are copied while step k computes, and step
+    k's output is read back while step k+1 computes.  The timed region opens before the first
+    input copy and closes after the last output copy.
     """
     import torch
     from paged_kv_attention_34_b200 import kv_cache_write, paged_attn_decode
@@ -357,33 +384,90 @@ def run_e2e(st, w, args, stream, device, step_bytes):
         offs[name] = off
         off += (t.numel() * t.element_size() + 255) // 256 * 256
     host_buf = torch.zeros(off, dtype=torch.uint8).pin_memory()
-    dev_buf = torch.empty(off, dtype=torch.uint8, device=device)
-    views = {}
     for name, t in parts:
         n = t.numel() * t.element_size()
         host_buf[offs[name]:offs[name] + n].copy_(t.contiguous().view(-1).view(torch.uint8))
-        views[name] = dev_buf[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
+    dev_bufs = [torch.empty(off, dtype=torch.uint8, device=device) for _ in range(2)]
+    views = []
+    for db in dev_bufs:
+        v = {}
+        for name, t in parts:
+            n = t.numel() * t.element_size()
+            v[name] = db[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
+        views.append(v)
+    outs = [torch.empty_like(st.out) for _ in range(2)]
     out_host = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
     h2d = off
     d2h = out_host.numel() * out_host.element_size()
+    copy = torch.cuda.Stream(device)
 
-    def one():
-        dev_buf.copy_(host_buf, non_blocking=True)
-        kv_cache_write(views["k_new"], views["v_new"], views["slot"], st.key_cache, st.value_cache, status=st.status)
-        paged_attn_decode(views["q"], st.key_cache, st.value_cache, views["bt"], views["cu"], views["ctx"],
-                          call.max_ctx, w.scale, out=st.out, workspace=call.ws)
-        out_host.copy_(st.out, non_blocking=True)
+    def run(n_steps):
+        """n_steps pipelined steps; returns (start, end) events on the compute stream."""
+        ev = torch.cuda.Event
+        landed = [ev() for _ in range(n_steps)]     # inputs of step k are on the device
+        computed = [ev() for _ in range(n_steps)]   # kernels of step k are done
+        read = [ev() for _ in range(n_steps)]       # output of step k is on the host
+        start, end = ev(enable_timing=True), ev(enable_timing=True)
+        start.record(stream)
+        copy.wait_event(start)
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            one()
+        def h2d_step(k):
+            with torch.cuda.stream(copy):
+                if k >= 2:
+                    copy.wait_event(computed[k - 2])  # buffer k % 2 is free again
+                dev_bufs[k % 2].copy_(host_buf, non_blocking=True)
+                landed[k].record(copy)
+
+        h2d_step(0)
+        for k in range(n_steps):
+            if k + 1 < n_steps:
+                h2d_step(k + 1)
+            with torch.cuda.stream(stream):
+                stream.wait_event(landed[k])
+                if k >= 2:
+                    stream.wait_event(read[k - 2])  # output buffer k % 2 has been read back
+                v = views[k % 2]
+                kv_cache_write(v["k_new"], v["v_new"], v["slot"], st.key_cache, st.value_cache, status=st.status)
+                paged_attn_decode(v["q"], st.key_cache, st.value_cache, v["bt"], v["cu"], v["ctx"], call.max_ctx,
+                                  w.scale, out=outs[k % 2], workspace=call.ws)
+                computed[k].record(stream)
+            with torch.cuda.stream(copy):
+                copy.wait_event(computed[k])
+                out_host.copy_(outs[k % 2], non_blocking=True)
+                read[k].record(copy)
+        stream.wait_event(read[n_steps - 1])
+        end.record(stream)
+        return start, end
+
+    def serial_step():
+        # the same copies and calls one after the other on one stream, no overlap
+        dev_bufs[0].copy_(host_buf, non_blocking=True)
+        v = views[0]
+        kv_cache_write(v["k_new"], v["v_new"], v["slot"], st.key_cache, st.value_cache, status=st.status)
+        paged_attn_decode(v["q"], st.key_cache, st.value_cache, v["bt"], v["cu"], v["ctx"], call.max_ctx, w.scale,
+                          out=outs[0], workspace=call.ws)
+        out_host.copy_(outs[0], non_blocking=True)
+
+    run(args.warmup)
     torch.cuda.synchronize()
     barrier()
-    total_ms, _ = time_calls([one], args.steps, stream)
-    total_ms = reduce_max(total_ms, device)
+    start, end = run(args.steps)
+    end.synchronize()
+    torch.cuda.synchronize()
+    total_ms = reduce_max(start.elapsed_time(end), device)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            serial_step()
+    torch.cuda.synchronize()
+    barrier()
+    serial_ms = reduce_max(time_steps([serial_step], args.steps, stream), device)
     bytes_all = reduce_sum(float(step_bytes * args.steps), device)
     return {"value": round(bytes_all / (total_ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(total_ms / args.steps, 6)}
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(total_ms / args.steps, 6),
+            "overlap": "step k+1's H2D and step k-1's D2H run on a copy stream during step k's kernels",
+            "serial": {"value": round(bytes_all / (serial_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                       "ms_per_step": round(serial_ms / args.steps, 6),
+                       "note": "the same copies and calls in series on one stream"}}
 
 
 def leg_prefill(args, stream, device, bf16_peak, peak_src, rank):
