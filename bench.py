@@ -19,7 +19,9 @@ The same JSON line carries:
   roofline      decode call (split kernel + merge) vs the measured HBM copy peak
   prefill       causal varlen prefill (8 prompts U[256,2048], 40/40 heads, bf16):
                 TFLOP/s of exact causal pairs vs the measured bf16 peak
-  legs          the GQA shared-prefix decode step and the mixed continuous-batching step
+  legs          the GQA shared-prefix decode step, the mixed continuous-batching step, and
+                the preemption swap of KV blocks to a pinned host pool and back (GB/s against
+                a plain pinned cudaMemcpyAsync of the same bytes)
   e2e           the same metric with host buffers: every step's inputs go H2D from one pinned
                 buffer and its output comes back D2H, all inside the timed region; the copies
                 run on a second stream, overlapping the neighbouring steps' kernels (double-
@@ -351,6 +353,7 @@ def run_ours(args):
         result["legs"] = {
             "gqa_shared_prefix": leg_gqa(args, stream, device, hbm_peak, rank),
             "mixed_step": leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank),
+            "block_swap": leg_swap(args, stream, device, rank),
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
@@ -513,6 +516,46 @@ def leg_gqa(args, stream, device, hbm_peak, rank):
             "note": "shared prefix counted once; its blocks may stay in L2 across sequences"}
 
 
+def leg_swap(args, stream, device, rank, n_blocks=512):
+    """Preemption swap: n_blocks blocks of the 13B-shaped cache (40 heads, d 128, fp16; 320 KB of
+    K+V per block) out to a pinned host pool and back in, each direction timed on its own, against
+    one cudaMemcpyAsync of the same number of bytes between pinned host and device memory in the
+    same run (the host link's measured copy rate)."""
+    import torch
+
+    from paged_kv_attention_34_b200 import kv_block_swap
+
+    g = torch.Generator().manual_seed(shard_seed(34_102, rank))
+    NB, H, d = 2 * n_blocks, 40, 128
+    kc = torch.randn((NB, H, 16, d), generator=g).half().to(device)
+    vc = torch.randn((NB, H, 16, d), generator=g).half().to(device)
+    hk = torch.empty((n_blocks, H, 16, d), dtype=torch.float16).pin_memory()
+    hv = torch.empty((n_blocks, H, 16, d), dtype=torch.float16).pin_memory()
+    perm = torch.randperm(NB, generator=g)[:n_blocks].to(torch.int32)
+    pairs = torch.stack([perm, torch.randperm(n_blocks, generator=g).to(torch.int32)], 1).contiguous().to(device)
+    nbytes = 2 * n_blocks * H * 16 * d * 2
+    dev_flat = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    host_flat = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    steps = max(args.steps, 5)
+    res = {}
+    for name, fn in (("out", lambda: kv_block_swap(kc, vc, hk, hv, pairs, to_host=True, stream=stream)),
+                     ("in", lambda: kv_block_swap(kc, vc, hk, hv, pairs, to_host=False, stream=stream)),
+                     ("memcpy_d2h", lambda: host_flat.copy_(dev_flat, non_blocking=True)),
+                     ("memcpy_h2d", lambda: dev_flat.copy_(host_flat, non_blocking=True))):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fn()
+        torch.cuda.synchronize()
+        ms = time_steps([fn], steps, stream) / steps
+        res[name] = round(nbytes / (ms * 1e-3) / 1e9, 2)
+    return {"workload": f"swap of {n_blocks} blocks (40 heads, d 128, fp16: {nbytes / 1e6:.0f} MB of K+V) "
+                        "to a pinned host pool and back",
+            "unit": "GB/s", "out_GB/s": res["out"], "in_GB/s": res["in"],
+            "frac_out": round(res["out"] / res["memcpy_d2h"], 4), "frac_in": round(res["in"] / res["memcpy_h2d"], 4),
+            "peak_source": "cudaMemcpyAsync of the same bytes, pinned host <-> device, same run",
+            "memcpy_GB/s": {"d2h": res["memcpy_d2h"], "h2d": res["memcpy_h2d"]}}
+
+
 def leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank):
     from paged_kv_attention_34_b200 import workloads as W
     from paged_kv_attention_34_b200.step import attn_bytes, attn_flops, write_bytes
@@ -639,6 +682,8 @@ def run_one_leg(args):
         res = leg_prefill(args, stream, device, bf16, peak_src, 0)
     elif args.only == "gqa":
         res = leg_gqa(args, stream, device, hbm, 0)
+    elif args.only == "swap":
+        res = leg_swap(args, stream, device, 0)
     else:
         res = leg_mixed(args, stream, device, hbm, bf16, 0)
     print(json.dumps({"leg": args.only, **res}), flush=True)
@@ -653,7 +698,7 @@ def main(argv=None):
     ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
-    ap.add_argument("--only", choices=["prefill", "gqa", "mixed"], default=None,
+    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap"], default=None,
                     help="run one leg alone and print its JSON object (profiling runs)")
     ap.add_argument("--batch", type=int, default=64,
                     help="sequences of the headline decode workload (64 = the 13B-shaped layer; smaller for profiling)")

@@ -100,6 +100,33 @@ int pa_kv_cache_write(const void *k_new, const void *v_new, const int32_t *slot_
 int pa_kv_block_copy(void *key_cache, void *value_cache, int64_t num_blocks, int H_kv, int d, pa_dtype dtype,
                      const int32_t *pairs, int64_t n, int32_t *status, void *stream);
 
+/* Directions of pa_kv_block_swap. */
+#define PA_SWAP_OUT 0 /* device cache -> host pool */
+#define PA_SWAP_IN 1  /* host pool -> device cache */
+
+/*
+ * pa_kv_block_swap -- move whole blocks between the device caches and a pool
+ * of blocks in page-locked host memory: the swap-out of a preempted request's
+ * KV blocks to CPU memory, and their swap-in when it resumes (the interview
+ * Q&A page, its answer on combining continuous batching with PagedAttention:
+ * preemption under memory pressure).  For each pair (dev, host) =
+ * (pairs[2i], pairs[2i+1]) copy K and V of every head and all 16 rows of
+ * device block `dev` to host block `host` (PA_SWAP_OUT) or back (PA_SWAP_IN).
+ * Pairs with an id outside [0, num_blocks) / [0, host_blocks) are skipped and
+ * reported through `status`.  No destination may appear twice in one call.
+ * Bit-exact.  One kernel reads and writes the host pool over the host link
+ * through its device-mapped address; nothing is staged.
+ *   host_key, host_value  [host_blocks][H_kv][16][d], page-locked host memory
+ *                         that the device can address (cudaHostAlloc or a
+ *                         pinned torch tensor); anything else -> PA_ERR_ARG,
+ *                         before any launch.  Owned by the caller.
+ *   pairs                 int32 [n][2], device memory
+ *   direction             PA_SWAP_OUT or PA_SWAP_IN
+ */
+int pa_kv_block_swap(void *key_cache, void *value_cache, int64_t num_blocks, void *host_key, void *host_value,
+                     int64_t host_blocks, int H_kv, int d, pa_dtype dtype, const int32_t *pairs, int64_t n,
+                     int direction, int32_t *status, void *stream);
+
 /*
  * pa_decode_workspace_bytes -- device workspace that pa_paged_attn_decode needs
  * for these sizes: the status word area, the order in which the sequences are

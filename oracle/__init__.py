@@ -43,6 +43,8 @@ def _declare(L):
     L.oracle_kv_cache_write.argtypes = [P, P, P, c.c_int64, P, P, c.c_int64, c.c_int, c.c_int]
     L.oracle_kv_block_copy.restype = c.c_int64
     L.oracle_kv_block_copy.argtypes = [P, P, c.c_int64, c.c_int, c.c_int, P, c.c_int64]
+    L.oracle_kv_block_swap.restype = c.c_int64
+    L.oracle_kv_block_swap.argtypes = [P, P, c.c_int64, P, P, c.c_int64, c.c_int, c.c_int, P, c.c_int64, c.c_int]
     L.oracle_paged_attention.restype = c.c_int
     L.oracle_paged_attention.argtypes = [
         P, P, P, P, P, c.c_int, P, c.c_int, P, P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_double, P, c.c_int64, c.c_int,
@@ -130,6 +132,15 @@ def kv_block_copy(key_cache: np.ndarray, value_cache: np.ndarray, pairs, L=None)
     pr = _i32(pairs).reshape(-1, 2)
     NB, H_kv, _, d = key_cache.shape
     return (L or lib()).oracle_kv_block_copy(_p(key_cache), _p(value_cache), NB, H_kv, d, _p(pr), pr.shape[0])
+
+
+def kv_block_swap(key_cache: np.ndarray, value_cache: np.ndarray, host_key: np.ndarray, host_value: np.ndarray,
+                  pairs, to_host: bool, L=None) -> int:
+    """Blocks pairs[i, 0] (device caches) <-> pairs[i, 1] (host pool), in place; returns the pairs skipped."""
+    pr = _i32(pairs).reshape(-1, 2)
+    NB, H_kv, _, d = key_cache.shape
+    return (L or lib()).oracle_kv_block_swap(_p(key_cache), _p(value_cache), NB, _p(host_key), _p(host_value),
+                                             host_key.shape[0], H_kv, d, _p(pr), pr.shape[0], 1 if to_host else 0)
 
 
 def paged_attention(

@@ -142,6 +142,37 @@ int64_t oracle_kv_block_copy(uint16_t *key_cache, uint16_t *value_cache, int64_t
     return bad;
 }
 
+/* Swap of whole blocks between the device caches and a host pool (the interview
+ * Q&A page, its answer on combining continuous batching with PagedAttention:
+ * a preempted request's KV blocks go out to CPU memory and come back when it
+ * resumes).  Pair i = (device block, host block); to_host != 0 copies device
+ * -> host, else host -> device.  Pairs with an id out of range are skipped and
+ * counted. */
+int64_t oracle_kv_block_swap(uint16_t *key_cache, uint16_t *value_cache, int64_t num_blocks, uint16_t *host_key,
+                             uint16_t *host_value, int64_t host_blocks, int H_kv, int d, const int32_t *pairs,
+                             int64_t n, int to_host)
+{
+    int64_t bad = 0;
+    int64_t per_block = (int64_t)H_kv * ORACLE_BLOCK * d;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t dev = pairs[2 * i], hst = pairs[2 * i + 1];
+        if (dev < 0 || hst < 0 || dev >= num_blocks || hst >= host_blocks) {
+            ++bad;
+            continue;
+        }
+        for (int64_t e = 0; e < per_block; ++e) {
+            if (to_host) {
+                host_key[hst * per_block + e] = key_cache[dev * per_block + e];
+                host_value[hst * per_block + e] = value_cache[dev * per_block + e];
+            } else {
+                key_cache[dev * per_block + e] = host_key[hst * per_block + e];
+                value_cache[dev * per_block + e] = host_value[hst * per_block + e];
+            }
+        }
+    }
+    return bad;
+}
+
 /* ---- attention over the paged cache ---------------------------------------- */
 
 /* One output row: query token t (of sequence b, index i within its q_b new

@@ -56,6 +56,8 @@ def _declare(L):
     L.pa_kv_cache_write.argtypes = [P, P, P, I64, P, P, I64, I, I, I, P, P]
     L.pa_kv_block_copy.restype = I
     L.pa_kv_block_copy.argtypes = [P, P, I64, I, I, I, P, I64, P, P]
+    L.pa_kv_block_swap.restype = I
+    L.pa_kv_block_swap.argtypes = [P, P, I64, P, P, I64, I, I, I, P, I64, I, P, P]
     L.pa_decode_workspace_bytes.restype = SZ
     L.pa_decode_workspace_bytes.argtypes = [I64, I, I, I, I, I]
     L.pa_paged_attn_decode.restype = I
@@ -169,6 +171,33 @@ def kv_block_copy(key_cache, value_cache, pairs, status=None, stream=None):
         _ptr(status), ctypes.c_void_p(_stream(stream)),
     )
     _check(rc, "pa_kv_block_copy")
+
+
+PA_SWAP_OUT, PA_SWAP_IN = 0, 1
+
+
+def kv_block_swap(key_cache, value_cache, host_key, host_value, pairs, to_host: bool, status=None, stream=None):
+    """Swap blocks between the device caches and a pinned host pool (pairs: int32 [n, 2] of
+    (device block, host block)): device -> host when `to_host`, else host -> device."""
+    _cuda(key_cache, "key_cache", ndim=4)
+    _cuda(value_cache, "value_cache", key_cache.dtype, 4)
+    _cuda(pairs, "pairs", torch.int32, 2)
+    NB, H_kv, _, d = key_cache.shape
+    for name, t in (("host_key", host_key), ("host_value", host_value)):
+        if t.device.type != "cpu" or not t.is_pinned() or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous pinned CPU tensor")
+        if t.dtype != key_cache.dtype or t.dim() != 4 or tuple(t.shape[1:]) != (H_kv, 16, d):
+            raise ValueError(f"{name} must be [host_blocks, {H_kv}, 16, {d}] {key_cache.dtype}")
+    if host_value.shape[0] != host_key.shape[0]:
+        raise ValueError("host_key and host_value must hold the same number of blocks")
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    rc = lib().pa_kv_block_swap(
+        _ptr(key_cache), _ptr(value_cache), NB, ctypes.c_void_p(host_key.data_ptr()),
+        ctypes.c_void_p(host_value.data_ptr()), host_key.shape[0], H_kv, d, _dtype_code(key_cache), _ptr(pairs),
+        pairs.shape[0], PA_SWAP_OUT if to_host else PA_SWAP_IN, _ptr(status), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_kv_block_swap")
 
 
 def decode_workspace_bytes(T: int, B: int, H_q: int, H_kv: int, d: int, max_ctx: int) -> int:

@@ -161,6 +161,35 @@ def pin_block_copy(L):
     assert oracle.kv_block_copy(k16, v16, torch.tensor([[0, NB]], dtype=torch.int32), L=L) == 1
 
 
+def pin_block_swap(L):
+    """Swap-out then swap-in into other device blocks restores their contents bit for bit; blocks
+    outside the pairs are untouched; out-of-range pairs are skipped and counted."""
+    g = torch.Generator().manual_seed(16)
+    NB, HB, H, d = 8, 5, 2, 16
+    kc = torch.randn((NB, H, 16, d), generator=g).half()
+    vc = torch.randn((NB, H, 16, d), generator=g).half()
+    k16, v16 = oracle._u16(kc).copy(), oracle._u16(vc).copy()
+    hk, hv = np.zeros((HB, H, 16, d), np.uint16), np.zeros((HB, H, 16, d), np.uint16)
+    out_pairs = torch.tensor([[6, 0], [2, 3], [5, 1]], dtype=torch.int32)
+    assert oracle.kv_block_swap(k16, v16, hk, hv, out_pairs, to_host=True, L=L) == 0
+    assert np.array_equal(k16, oracle._u16(kc)) and np.array_equal(v16, oracle._u16(vc))  # source untouched
+    assert not hk[2].any() and not hk[4].any()                                              # unused host blocks
+    # the device blocks are reused for something else, then the request resumes in other blocks
+    k16[[6, 2, 5]] = 0
+    v16[[6, 2, 5]] = 0
+    in_pairs = torch.tensor([[7, 0], [0, 3], [4, 1]], dtype=torch.int32)
+    assert oracle.kv_block_swap(k16, v16, hk, hv, in_pairs, to_host=False, L=L) == 0
+    for (src, _), (dst, _) in zip(out_pairs.tolist(), in_pairs.tolist()):
+        assert np.array_equal(k16[dst], oracle._u16(kc)[src]) and np.array_equal(v16[dst], oracle._u16(vc)[src])
+    for b in (1, 3):  # neither swapped out nor in
+        assert np.array_equal(k16[b], oracle._u16(kc)[b]) and np.array_equal(v16[b], oracle._u16(vc)[b])
+    before = (k16.copy(), hk.copy())
+    bad = torch.tensor([[NB, 0], [0, HB], [-1, 2]], dtype=torch.int32)
+    assert oracle.kv_block_swap(k16, v16, hk, hv, bad, to_host=True, L=L) == 3
+    assert oracle.kv_block_swap(k16, v16, hk, hv, bad, to_host=False, L=L) == 3
+    assert np.array_equal(before[0], k16) and np.array_equal(before[1], hk)
+
+
 def pin_sdpa_library(L):
     """Paged fp64 oracle == torch fp64 SDPA on the gathered contiguous K/V (ragged, GQA, causal)."""
     for w in _small_cases():
@@ -423,6 +452,7 @@ ALL_PINS = [
     pin_bf16_decoding,
     pin_cache_write,
     pin_block_copy,
+    pin_block_swap,
     pin_sdpa_library,
     pin_dense_three_pass,
     pin_block_permutation,

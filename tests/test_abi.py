@@ -2,11 +2,15 @@
 point, and rejects bad arguments on the host before touching the device.
 
 Only host-side paths run here (no GPU): every call below returns from its
-argument checks before any CUDA runtime call.
+argument checks before any launch; the only CUDA runtime call made is the
+block swap's pointer-attribute query of its host pools, which refuses them
+cleanly when there is no device.
 """
 import ctypes
 import os
 import re
+
+import numpy as np
 import subprocess
 
 import pytest
@@ -82,6 +86,29 @@ def test_block_copy_rejects_bad_args(L):
     assert f(_fake(), _fake(), 8, 2, 64, 0, _fake(), -1, None, None) == -1
     assert f(_fake(0x10004), _fake(), 8, 2, 64, 0, _fake(), 3, None, None) == -3
     assert f(_fake(), _fake(), 8, 2, 64, 0, _fake(), 0, None, None) == 0
+
+
+def test_block_swap_rejects_bad_args(L):
+    f = L.pa_kv_block_swap
+
+    def call(NB=8, HB=4, H=2, d=64, dt=0, n=3, direction=0, hk=None, hv=None):
+        hk = hk if hk is not None else _fake()
+        hv = hv if hv is not None else _fake()
+        return f(_fake(), _fake(), NB, hk, hv, HB, H, d, dt, _fake(), n, direction, None, None)
+
+    assert call(d=80) == -2
+    assert call(n=-1) == -1
+    assert call(HB=0) == -1
+    assert call(NB=0) == -1
+    assert call(direction=2) == -1
+    assert call(dt=5) == -1
+    assert call(n=0) == 0  # nothing to do, nothing launched
+    # host pools that are not page-locked host memory are refused before any launch
+    n0 = pa.launch_count()
+    host = np.zeros(1 << 16, np.uint8)
+    ptr = ctypes.c_void_p(host.ctypes.data)
+    assert call(hk=ptr, hv=ptr) == -1
+    assert pa.launch_count() == n0
 
 
 def _decode(L, *, B=2, T=2, H_q=8, H_kv=2, d=128, max_ctx=100, NB=16, ws=_fake(), wsb=1 << 20, q=_fake(),

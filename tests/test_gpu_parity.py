@@ -219,6 +219,66 @@ def test_block_copy_bitexact_random():
     assert np.array_equal(_u16(kd), k16) and np.array_equal(_u16(vd), v16)
 
 
+def _pool(n, H, d, dtype):
+    return torch.zeros((n, H, 16, d), dtype=dtype).pin_memory()
+
+
+def test_block_swap_bitexact_round_trip():
+    # swap a request's blocks out to a pinned host pool, reuse the device blocks, swap it back in
+    # elsewhere: both directions byte for byte as the oracle (caches hold NaN outside contexts too)
+    g = torch.Generator().manual_seed(5)
+    NB, HB, H, d = 48, 20, 8, 128
+    kc = torch.randn((NB, H, 16, d), generator=g).bfloat16()
+    vc = torch.randn((NB, H, 16, d), generator=g).bfloat16()
+    kc[5, :, 9:] = float("nan")
+    hk, hv = _pool(HB, H, d, torch.bfloat16), _pool(HB, H, d, torch.bfloat16)
+    k16, v16 = _u16(kc).copy(), _u16(vc).copy()
+    hk16, hv16 = np.zeros((HB, H, 16, d), np.uint16), np.zeros((HB, H, 16, d), np.uint16)
+    out_pairs = torch.tensor([[3, 0], [17, 5], [40, 19], [5, 7]], dtype=torch.int32)
+    in_pairs = torch.tensor([[10, 0], [11, 5], [12, 19], [47, 7]], dtype=torch.int32)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kd, vd = kc.cuda(), vc.cuda()
+    assert oracle.kv_block_swap(k16, v16, hk16, hv16, out_pairs, to_host=True) == 0
+    pa.kv_block_swap(kd, vd, hk, hv, out_pairs.cuda(), to_host=True, status=status)
+    torch.cuda.synchronize()
+    assert np.array_equal(_u16(hk), hk16) and np.array_equal(_u16(hv), hv16)
+    assert oracle.kv_block_swap(k16, v16, hk16, hv16, in_pairs, to_host=False) == 0
+    pa.kv_block_swap(kd, vd, hk, hv, in_pairs.cuda(), to_host=False, status=status)
+    torch.cuda.synchronize()
+    assert np.array_equal(_u16(kd), k16) and np.array_equal(_u16(vd), v16)
+    assert pa.read_status(status) == 0
+
+
+def test_block_swap_bad_ids_are_reported_and_skipped():
+    NB, HB, H, d = 6, 3, 2, 64
+    kd = torch.randn((NB, H, 16, d), device="cuda").half()
+    vd = torch.randn((NB, H, 16, d), device="cuda").half()
+    hk, hv = _pool(HB, H, d, torch.float16), _pool(HB, H, d, torch.float16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pairs = torch.tensor([[NB, 0], [1, HB], [2, 1]], dtype=torch.int32, device="cuda")
+    pa.kv_block_swap(kd, vd, hk, hv, pairs, to_host=True, status=status)
+    torch.cuda.synchronize()
+    assert pa.read_status(status) == -7  # PA_ERR_BOUNDS
+    assert torch.equal(hk[1], kd[2].cpu()) and torch.equal(hv[1], vd[2].cpu())
+    assert not hk[0].any() and not hk[2].any()
+
+
+def test_block_swap_refuses_pageable_host_memory():
+    import ctypes
+
+    NB, HB, H, d = 4, 2, 2, 64
+    kd = torch.zeros((NB, H, 16, d), device="cuda").half()
+    host = torch.zeros((HB, H, 16, d)).half()  # pageable
+    pairs = torch.tensor([[0, 0]], dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):
+        pa.kv_block_swap(kd, kd.clone(), host, host.clone(), pairs, to_host=True)
+    n0 = pa.launch_count()
+    rc = pa.lib().pa_kv_block_swap(ctypes.c_void_p(kd.data_ptr()), ctypes.c_void_p(kd.data_ptr()), NB,
+                                   ctypes.c_void_p(host.data_ptr()), ctypes.c_void_p(host.data_ptr()), HB, H, d, 0,
+                                   ctypes.c_void_p(pairs.data_ptr()), 1, 0, None, None)
+    assert rc == -1 and pa.launch_count() == n0
+
+
 def test_repeat_runs_identical():
     w = W.random_workload(8, B=4, q_max=3, ctx_max=600, H_kv=2, G=4, d=128, dtype=W.BF16, kind="decode")
     st = DeviceStep(w)

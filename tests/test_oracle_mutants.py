@@ -45,6 +45,14 @@ MUTANTS = {
         "key_cache[dst * per_block + e] = key_cache[src * per_block + e];",
         "key_cache[src * per_block + e] = key_cache[dst * per_block + e];",
     ),
+    "swap_in_reads_keys_for_values": (
+        "value_cache[dev * per_block + e] = host_value[hst * per_block + e];",
+        "value_cache[dev * per_block + e] = host_key[hst * per_block + e];",
+    ),
+    "swap_out_wrong_host_block": (
+        "host_key[hst * per_block + e] = key_cache[dev * per_block + e];",
+        "host_key[dev * per_block + e] = key_cache[dev * per_block + e];",
+    ),
     "online_no_rescale": ("o[c] = alpha * o[c] + acc;", "o[c] = o[c] + acc;"),
     "merge_sign": ("double w = exp(lses[s] - m) / z;", "double w = exp(m - lses[s]) / z;"),
 }
