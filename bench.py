@@ -19,7 +19,8 @@ The same JSON line carries:
   roofline      decode call (split kernel + merge) vs the measured HBM copy peak
   prefill       causal varlen prefill (8 prompts U[256,2048], 40/40 heads, bf16):
                 TFLOP/s of exact causal pairs vs the measured bf16 peak
-  legs          the GQA shared-prefix decode step, the mixed continuous-batching step, and
+  legs          the GQA shared-prefix decode step, the mixed continuous-batching step, the
+                tree-attention verify of speculative drafts (HBM roofline), and
                 the preemption swap of KV blocks to a pinned host pool and back (GB/s against
                 a plain pinned cudaMemcpyAsync of the same bytes)
   e2e           the same metric with host buffers: every step's inputs go H2D from one pinned
@@ -353,6 +354,7 @@ def run_ours(args):
         result["legs"] = {
             "gqa_shared_prefix": leg_gqa(args, stream, device, hbm_peak, rank),
             "mixed_step": leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank),
+            "tree_verify": leg_tree(args, stream, device, hbm_peak, rank),
             "block_swap": leg_swap(args, stream, device, rank),
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -514,6 +516,43 @@ def leg_gqa(args, stream, device, hbm_peak, rank):
             "unique_bytes": b, "decode_ms": round(ms, 5), "step_ms": round(step_ms, 5),
             "per_call_ms": {k: round(v, 5) for k, v in per.items()},
             "note": "shared prefix counted once; its blocks may stay in L2 across sequences"}
+
+
+def leg_tree(args, stream, device, hbm_peak, rank):
+    """Tree-attention verification: 64 sequences x 8 drafted tokens in a random draft tree,
+    contexts U[512, 4096], 32/8 heads, bf16; step = cache write + tree-verify decode."""
+    import torch
+
+    from paged_kv_attention_34_b200 import paged_attn_decode_tree
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import DeviceStep, attn_bytes
+
+    w = W.tree_verify(seed=shard_seed(34_105, rank))
+    tm = W.random_tree_masks(shard_seed(34_105, rank), w.q_lens).to(device)
+    with torch.cuda.stream(stream):
+        st = DeviceStep(w, device=device)
+    call = st.calls[0]
+
+    def attend():
+        paged_attn_decode_tree(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, tm, call.max_ctx,
+                               w.scale, out=call.out, workspace=call.ws)
+
+    fns = [st.write, attend]
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            for fn in fns:
+                fn()
+    torch.cuda.synchronize()
+    total, per = time_calls(fns, max(args.steps, 5), stream)
+    if any(st.statuses()):
+        raise RuntimeError(f"device status {st.statuses()}")
+    b = attn_bytes(w)
+    gbs = b / (per[1] * 1e-3) / 1e9
+    return {"workload": "tree-attention verify: 64 sequences x 8 drafts (random draft tree), ctx U[512,4096], "
+                        "32/8 heads, d 128, bf16",
+            "decode_GB/s": round(gbs, 1), "frac": round(gbs / hbm_peak, 4), "bytes": b,
+            "decode_ms": round(per[1], 5), "per_call_ms": {"kv_cache_write": round(per[0], 5),
+                                                           "paged_attn_decode_tree": round(per[1], 5)}}
 
 
 def leg_swap(args, stream, device, rank, n_blocks=512):
@@ -684,6 +723,8 @@ def run_one_leg(args):
         res = leg_gqa(args, stream, device, hbm, 0)
     elif args.only == "swap":
         res = leg_swap(args, stream, device, 0)
+    elif args.only == "tree":
+        res = leg_tree(args, stream, device, hbm, 0)
     else:
         res = leg_mixed(args, stream, device, hbm, bf16, 0)
     print(json.dumps({"leg": args.only, **res}), flush=True)
@@ -698,7 +739,7 @@ def main(argv=None):
     ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
-    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap"], default=None,
+    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap", "tree"], default=None,
                     help="run one leg alone and print its JSON object (profiling runs)")
     ap.add_argument("--batch", type=int, default=64,
                     help="sequences of the headline decode workload (64 = the 13B-shaped layer; smaller for profiling)")

@@ -164,6 +164,24 @@ int pa_paged_attn_decode(void *out, const void *q, const void *key_cache, const 
                          size_t workspace_bytes, void *stream);
 
 /*
+ * pa_paged_attn_decode_tree -- pa_paged_attn_decode for tree-attention
+ * verification of speculative drafts (the interview Q&A page, speculative
+ * decoding with a tree of drafts): the q_b new tokens of a sequence are the
+ * nodes of a draft tree, and token t sees every cached key before the new
+ * tokens plus new token j exactly when bit j of tree_mask[t] is set (its own
+ * bit and its ancestors' in the usual case).  The chain mask, bits 0..i for
+ * the i-th new token, is the causal verify of pa_paged_attn_decode.  Same
+ * sizes, layouts, workspace and errors as pa_paged_attn_decode, plus:
+ *   tree_mask  int32 [T], device memory; only bits 0 .. q_b - 1 are read.
+ *              NULL -> PA_ERR_ARG.  A token that sees no key at all gets O = 0.
+ */
+int pa_paged_attn_decode_tree(void *out, const void *q, const void *key_cache, const void *value_cache,
+                              int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
+                              const int32_t *cu_seqlens_q, const int32_t *context_lens, const int32_t *tree_mask,
+                              int B, int max_ctx, int64_t T, int H_q, int H_kv, int d, float scale, pa_dtype dtype,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * pa_paged_attn_decode_noalloc -- pa_paged_attn_decode without a caller workspace.
  * The pages have no counterpart: this is an interface for callers that may not
  * allocate device memory when they call, such as plugins inside an engine that

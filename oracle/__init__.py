@@ -49,6 +49,11 @@ def _declare(L):
     L.oracle_paged_attention.argtypes = [
         P, P, P, P, P, c.c_int, P, c.c_int, P, P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_double, P, c.c_int64, c.c_int,
     ]
+    L.oracle_paged_attention_tree.restype = c.c_int
+    L.oracle_paged_attention_tree.argtypes = [
+        P, P, P, P, P, c.c_int, P, c.c_int, P, P, P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_double, P, c.c_int64,
+        c.c_int,
+    ]
     L.oracle_dense_attention.restype = None
     L.oracle_dense_attention.argtypes = [P, P, P, P, c.c_int, c.c_int, c.c_int, c.c_double, c.c_int64]
     L.oracle_online_softmax.restype = None
@@ -157,12 +162,14 @@ def paged_attention(
     n_threads: int = 0,
     with_lse: bool = False,
     L=None,
+    tree_mask=None,
 ):
     """fp64 attention over the paged cache.
 
     q: [T, H_q, d] (16-bit); caches [NB, H_kv, 16, d] (16-bit).  ``rows`` selects
     flattened ``t * H_q + h`` rows; the result is then ``[len(rows), d]``, else
-    ``[T, H_q, d]``.
+    ``[T, H_q, d]``.  ``tree_mask`` (int32 [T]): tree-attention verification, token t sees the
+    cached keys before its sequence's new tokens and new token j when bit j is set; None = causal.
     """
     qq = _u16(q)
     T, H_q, d = qq.shape
@@ -180,10 +187,19 @@ def paged_attention(
         n_rows = r.shape[0]
         out = np.empty((n_rows, d), dtype=np.float64)
     lse = np.empty(n_rows, dtype=np.float64) if with_lse else None
-    rc = (L or lib()).oracle_paged_attention(
-        _p(out), _p(lse), _p(qq), _p(kc), _p(vc), dtype, _p(bt), bt.shape[1], _p(cu), _p(cl), B, H_q, H_kv, d,
-        float(scale), _p(r), n_rows, n_threads,
-    )
+    if tree_mask is None:
+        rc = (L or lib()).oracle_paged_attention(
+            _p(out), _p(lse), _p(qq), _p(kc), _p(vc), dtype, _p(bt), bt.shape[1], _p(cu), _p(cl), B, H_q, H_kv, d,
+            float(scale), _p(r), n_rows, n_threads,
+        )
+    else:
+        tm = _i32(tree_mask)
+        if tm.shape != (T,):
+            raise ValueError("tree_mask must be int32 [T]")
+        rc = (L or lib()).oracle_paged_attention_tree(
+            _p(out), _p(lse), _p(qq), _p(kc), _p(vc), dtype, _p(bt), bt.shape[1], _p(cu), _p(cl), _p(tm), B, H_q,
+            H_kv, d, float(scale), _p(r), n_rows, n_threads,
+        )
     if rc != 0:
         raise ValueError(f"oracle_paged_attention rejected its arguments (code {rc})")
     return (out, lse) if with_lse else out

@@ -179,20 +179,34 @@ int64_t oracle_kv_block_swap(uint16_t *key_cache, uint16_t *value_cache, int64_t
  * tokens), query head h.  Keys are gathered one by one through the block
  * table.  out_row receives d doubles.  Also returns the natural-log
  * log-sum-exp of the scaled scores when lse != NULL. */
+/* Key j of a row is visible: every key up to `last` under the causal rule (tree == NULL); with a
+ * tree mask, every cached key before the new tokens and new token j - base when its bit is set. */
+static int key_visible(int j, int base, const int32_t *tree)
+{
+    return !tree || j < base || ((*tree >> (j - base)) & 1);
+}
+
 static int attention_row(double *out_row, double *lse, const uint16_t *q, const uint16_t *key_cache,
                          const uint16_t *value_cache, int dtype, const int32_t *block_tables, int max_blocks,
                          int b, int i, int q_b, int ctx_b, int64_t t, int h, int H_q, int H_kv, int d,
-                         double scale, double *s /* scratch, >= ctx_b doubles */)
+                         double scale, double *s /* scratch, >= ctx_b doubles */, const int32_t *tree)
 {
     int G = H_q / H_kv;
     int g = h / G; /* consecutive query heads share one KV head */
     int last = ctx_b - q_b + i; /* causal: keys 0 .. last */
+    int base = ctx_b - q_b;     /* first new token */
+    if (tree)
+        last = ctx_b - 1; /* tree verify: the mask decides among the new tokens */
     if (last < 0)
         return -1;
     const uint16_t *qrow = q + (t * H_q + h) * (int64_t)d;
 
-    /* scores s_j = scale * <q, K_j> */
+    /* scores s_j = scale * <q, K_j> (masked keys: -inf) */
     for (int j = 0; j <= last; ++j) {
+        if (!key_visible(j, base, tree)) {
+            s[j] = -INFINITY;
+            continue;
+        }
         int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
         int64_t off = j % ORACLE_BLOCK;
         const uint16_t *krow = key_cache + ((block * H_kv + g) * ORACLE_BLOCK + off) * d;
@@ -206,6 +220,8 @@ static int attention_row(double *out_row, double *lse, const uint16_t *q, const 
     for (int j = 0; j <= last; ++j)
         if (s[j] > m)
             m = s[j];
+    if (m == -INFINITY)
+        return -1; /* no visible key */
     double z = 0.0;
     for (int j = 0; j <= last; ++j) {
         s[j] = exp(s[j] - m);
@@ -218,6 +234,8 @@ static int attention_row(double *out_row, double *lse, const uint16_t *q, const 
         int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
         int64_t off = j % ORACLE_BLOCK;
         const uint16_t *vrow = value_cache + ((block * H_kv + g) * ORACLE_BLOCK + off) * d;
+        if (!key_visible(j, base, tree))
+            continue; /* masked key of a tree row (its V may be anything) */
         double w = s[j] / z;
         for (int k = 0; k < d; ++k)
             out_row[k] += w * widen(vrow[k], dtype);
@@ -232,10 +250,11 @@ static int attention_row(double *out_row, double *lse, const uint16_t *q, const 
  * [n_rows] natural-log log-sum-exp per row.
  * Returns 0, or -1 if some sequence has ctx_b < q_b or q_b < 0,
  * -2 if H_q is not a multiple of H_kv. */
-int oracle_paged_attention(double *out, double *lse_out, const uint16_t *q, const uint16_t *key_cache,
+static int paged_attention_impl(double *out, double *lse_out, const uint16_t *q, const uint16_t *key_cache,
                            const uint16_t *value_cache, int dtype, const int32_t *block_tables, int max_blocks,
                            const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int H_q, int H_kv,
-                           int d, double scale, const int64_t *rows, int64_t n_rows, int n_threads)
+                           int d, double scale, const int64_t *rows, int64_t n_rows, int n_threads,
+                                const int32_t *tree_mask)
 {
     if (H_kv <= 0 || H_q % H_kv != 0)
         return -2;
@@ -271,7 +290,7 @@ int oracle_paged_attention(double *out, double *lse_out, const uint16_t *q, cons
             int q_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
             int rc = attention_row(out + r * d, lse_out ? lse_out + r : NULL, q, key_cache, value_cache, dtype,
                                    block_tables, max_blocks, b, i, q_b, context_lens[b], t, h, H_q, H_kv, d,
-                                   scale, s);
+                                   scale, s, tree_mask ? tree_mask + t : NULL);
             if (rc) {
 #pragma omp atomic write
                 status = rc;
@@ -280,6 +299,31 @@ int oracle_paged_attention(double *out, double *lse_out, const uint16_t *q, cons
         free(s);
     }
     return status;
+}
+
+
+int oracle_paged_attention(double *out, double *lse_out, const uint16_t *q, const uint16_t *key_cache,
+                           const uint16_t *value_cache, int dtype, const int32_t *block_tables, int max_blocks,
+                           const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int H_q, int H_kv,
+                           int d, double scale, const int64_t *rows, int64_t n_rows, int n_threads)
+{
+    return paged_attention_impl(out, lse_out, q, key_cache, value_cache, dtype, block_tables, max_blocks,
+                                cu_seqlens_q, context_lens, B, H_q, H_kv, d, scale, rows, n_rows, n_threads, NULL);
+}
+
+/* Tree-attention verification (the interview Q&A page, speculative decoding with a draft tree):
+ * query token t of sequence b sees every cached key before the sequence's q_b new tokens, and new
+ * token j exactly when bit j of tree_mask[t] is set (the drafts on its path from the root).  The
+ * causal verify is the chain mask, bits 0 .. i for the i-th new token. */
+int oracle_paged_attention_tree(double *out, double *lse_out, const uint16_t *q, const uint16_t *key_cache,
+                                const uint16_t *value_cache, int dtype, const int32_t *block_tables, int max_blocks,
+                                const int32_t *cu_seqlens_q, const int32_t *context_lens, const int32_t *tree_mask,
+                                int B, int H_q, int H_kv, int d, double scale, const int64_t *rows, int64_t n_rows,
+                                int n_threads)
+{
+    return paged_attention_impl(out, lse_out, q, key_cache, value_cache, dtype, block_tables, max_blocks,
+                                cu_seqlens_q, context_lens, B, H_q, H_kv, d, scale, rows, n_rows, n_threads,
+                                tree_mask);
 }
 
 /* ---- dense forms on contiguous fp64 data (tiny inputs) ---------------------- */

@@ -62,6 +62,9 @@ def _declare(L):
     L.pa_decode_workspace_bytes.argtypes = [I64, I, I, I, I, I]
     L.pa_paged_attn_decode.restype = I
     L.pa_paged_attn_decode.argtypes = [P, P, P, P, I64, P, I, P, P, I, I, I64, I, I, I, c.c_float, I, P, SZ, P]
+    L.pa_paged_attn_decode_tree.restype = I
+    L.pa_paged_attn_decode_tree.argtypes = [P, P, P, P, I64, P, I, P, P, P, I, I, I64, I, I, I, c.c_float, I, P, SZ,
+                                            P]
     L.pa_prefill_workspace_bytes.restype = SZ
     L.pa_prefill_workspace_bytes.argtypes = [I, I, I, I, I]
     L.pa_paged_attn_prefill.restype = I
@@ -261,6 +264,27 @@ def paged_attn_decode(q, key_cache, value_cache, block_tables, cu_seqlens_q, con
     )
     _check(rc, "pa_paged_attn_decode")
     paged_attn_decode.last_workspace = ws
+    return out
+
+
+def paged_attn_decode_tree(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, tree_mask,
+                           max_ctx: int, scale: float, out=None, workspace=None, stream=None):
+    """Tree-attention verification: decode where token t sees the cached keys before its sequence's
+    new tokens and new token j when bit j of tree_mask[t] (int32 [T]) is set; returns out."""
+    out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
+                                               context_lens, out)
+    _cuda(tree_mask, "tree_mask", torch.int32, 1)
+    if tree_mask.shape[0] != T:
+        raise ValueError(f"tree_mask must be int32 [{T}]")
+    nbytes = decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx)
+    ws = _workspace(workspace, nbytes, q.device)
+    rc = lib().pa_paged_attn_decode_tree(
+        _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
+        _ptr(cu_seqlens_q), _ptr(context_lens), _ptr(tree_mask), B, int(max_ctx), T, H_q, H_kv, d, float(scale),
+        _dtype_code(q), _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_paged_attn_decode_tree")
+    paged_attn_decode_tree.last_workspace = ws
     return out
 
 

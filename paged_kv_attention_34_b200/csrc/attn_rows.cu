@@ -44,6 +44,7 @@ struct RowsParams {
     float *ws_o;    // [max_splits][T][H_q][D] normalised partial outputs
     float *ws_lse;  // [max_splits][T][H_q] log2-sum-exp of the scaled scores
     const int32_t *order;  // [B] sequences by decreasing page count: grid z -> sequence
+    const int32_t *tree;   // [T] tree verification: bit j = the token sees new token j; nullptr = causal
     int32_t *status;
     int64_t num_blocks;
     int64_t T;
@@ -135,7 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (row0 >= R)
         return;
     const int rows_here = min(kRowsPerCta, R - row0);
-    const int lim_cta = ctx - qb + (row0 + rows_here - 1) / G;  // last key any row here sees
+    const bool tree = p.tree != nullptr;
+    const int base = ctx - qb;  // first new token of the sequence
+    // last key any row here sees (a tree row may see every new token)
+    const int lim_cta = tree ? ctx - 1 : ctx - qb + (row0 + rows_here - 1) / G;
     const int pages_need = lim_cta / 16 + 1;
     const int pages_ctx = (ctx + 15) / 16;
     const int n_splits = (pages_ctx + p.split_pages - 1) / p.split_pages;
@@ -237,10 +241,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- per-thread row state --------------------------------------------------------------
     // This thread holds rows ra = lane/4 and rb = ra + 8 of its warp's m-tile.
+    // Key k is visible to a row when k <= lim and, among the new tokens (k >= base), its bit is set:
+    // causal rows see keys up to their own position with every bit set; tree rows see up to the
+    // last key with their own mask.
     const int ra = mt * 16 + (lane >> 2), rb = ra + 8;
-    const int lim_a = ra < rows_here ? ctx - qb + (row0 + ra) / G : -1;
-    const int lim_b = rb < rows_here ? ctx - qb + (row0 + rb) / G : -1;
-    const int lim_warp = has_rows ? ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G : -1;
+    const int lim_a = ra < rows_here ? (tree ? ctx - 1 : ctx - qb + (row0 + ra) / G) : -1;
+    const int lim_b = rb < rows_here ? (tree ? ctx - 1 : ctx - qb + (row0 + rb) / G) : -1;
+    const uint32_t bits_a = tree && ra < rows_here ? static_cast<uint32_t>(__ldg(p.tree + q0 + (row0 + ra) / G)) : ~0u;
+    const uint32_t bits_b = tree && rb < rows_here ? static_cast<uint32_t>(__ldg(p.tree + q0 + (row0 + rb) / G)) : ~0u;
+    const int lim_warp =
+        has_rows ? (tree ? ctx - 1 : ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G) : -1;
+    auto visible = [&](int key, int lim, uint32_t bits) {
+        return key <= lim && (key < base || ((bits >> (key - base)) & 1u));
+    };
 
     uint32_t qa[KSTEPS][4];
     if (has_rows) {
@@ -307,8 +320,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         const int key = j0 + nt * 8 + 2 * kq + c;
-                        s[nt][c] = key <= lim_a ? s[nt][c] * sl2 : -INFINITY;
-                        s[nt][2 + c] = key <= lim_b ? s[nt][2 + c] * sl2 : -INFINITY;
+                        s[nt][c] = visible(key, lim_a, bits_a) ? s[nt][c] * sl2 : -INFINITY;
+                        s[nt][2 + c] = visible(key, lim_b, bits_b) ? s[nt][2 + c] * sl2 : -INFINITY;
                         mx_a = fmaxf(mx_a, s[nt][c]);
                         mx_b = fmaxf(mx_b, s[nt][2 + c]);
                     }
@@ -653,6 +666,7 @@ static int run(const AttnArgs &a)
     rp.max_ctx = a.max_ctx;
     rp.max_q_len = a.max_q_len;
     rp.scale_log2 = a.scale * 1.4426950408889634f;
+    rp.tree = a.tree_mask;
     {
         const DecodePlan pl = decode_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx);
         rp.n_rg = pl.row_groups;

@@ -148,6 +148,33 @@ extern "C" int pa_paged_attn_decode(void *out, const void *q, const void *key_ca
     return launch_decode(a);
 }
 
+extern "C" int pa_paged_attn_decode_tree(void *out, const void *q, const void *key_cache, const void *value_cache,
+                                         int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
+                                         const int32_t *cu_seqlens_q, const int32_t *context_lens,
+                                         const int32_t *tree_mask, int B, int max_ctx, int64_t T, int H_q, int H_kv,
+                                         int d, float scale, pa_dtype dtype, void *workspace, size_t workspace_bytes,
+                                         void *stream)
+{
+    AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
+               context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
+               static_cast<cudaStream_t>(stream), tree_mask};
+    int rc = check_attn(a, true);
+    if (rc != PA_OK)
+        return rc;
+    if (B > 0 && T > 0) {
+        if (!tree_mask)
+            return PA_ERR_ARG;
+        if (!aligned4(tree_mask))
+            return PA_ERR_ALIGN;
+    }
+    if (workspace_bytes < decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx))
+        return PA_ERR_WORKSPACE;
+    rc = reset_status(workspace, a.stream);
+    if (rc != PA_OK || B == 0 || T == 0)
+        return rc;
+    return launch_decode(a);
+}
+
 extern "C" size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len)
 {
     if (B < 0 || H_q < 1 || H_kv < 1 || (d != 64 && d != 128) || max_q_len < 0 || H_q % H_kv)

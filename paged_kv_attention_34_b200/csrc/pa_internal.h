@@ -54,6 +54,7 @@ struct AttnArgs {
     void *workspace;
     size_t workspace_bytes;
     cudaStream_t stream;
+    const int32_t *tree_mask = nullptr;  // decode only: per-token visibility bits of the new tokens
 };
 
 // Split-KV decode plan: pages per split and the number of splits.

@@ -462,6 +462,49 @@ def config5(
     )
 
 
+def random_tree_masks(seed: int, q_lens) -> torch.Tensor:
+    """Draft-tree visibility masks for tree-attention verification, int32 [sum(q_lens)].
+
+    The q_b new tokens of a sequence are the nodes of a random forest drafted in order: node i has
+    a parent drawn uniformly from the earlier nodes or none (a new root).  Bit j of node i's mask
+    is set when node j is node i itself or one of its ancestors.
+    """
+    g = _gen(seed)
+    masks = []
+    for qb in q_lens:
+        m = []
+        for i in range(int(qb)):
+            parent = int(torch.randint(-1, i, (1,), generator=g)) if i > 0 else -1
+            m.append((m[parent] if parent >= 0 else 0) | (1 << i))
+        masks.extend(m)
+    return torch.tensor(masks, dtype=torch.int32)
+
+
+def chain_masks(q_lens) -> torch.Tensor:
+    """The causal verify as a tree: node i sees nodes 0 .. i."""
+    return torch.tensor([(1 << (i + 1)) - 1 for qb in q_lens for i in range(int(qb))], dtype=torch.int32)
+
+
+def tree_verify(seed: int = 34_105, fill: str = "nan", B: int = 64, q: int = 8) -> Workload:
+    """Tree-attention verification of speculative drafts: B sequences with q drafted tokens each
+    (a random draft forest, ``random_tree_masks``) on contexts U[512, 4096] (the verify rows of the
+    mixed step, with a tree instead of a chain); 32/8 heads, d 128, bf16."""
+    g = _gen(seed + 1_000_000)
+    ctx = _uniform_int(g, 512, 4096, B)
+    return build_workload(
+        "tree_verify",
+        q_lens=[q] * B,
+        ctx_lens=ctx,
+        H_q=32,
+        H_kv=8,
+        d=128,
+        dtype=BF16,
+        seed=seed,
+        calls=[AttnCall("decode", 0, B)],
+        fill=fill,
+    )
+
+
 def make_config(idx: int, **kw) -> Workload:
     return {1: config1, 2: config2, 3: config3, 4: config4, 5: config5}[idx](**kw)
 

@@ -40,8 +40,9 @@ def gather_contiguous(cache: torch.Tensor, table_row: torch.Tensor, n: int) -> t
     return x[:, :n]
 
 
-def sdpa_reference(w: W.Workload) -> np.ndarray:
-    """torch fp64 scaled_dot_product_attention per sequence on gathered K/V -> [T, H_q, d]."""
+def sdpa_reference(w: W.Workload, tree_mask=None) -> np.ndarray:
+    """torch fp64 scaled_dot_product_attention per sequence on gathered K/V -> [T, H_q, d]; with
+    ``tree_mask`` each new token sees the cached keys and the new tokens whose bits are set."""
     G = w.H_q // w.H_kv
     kc, vc = w.key_cache.clone(), w.value_cache.clone()
     # the step's new tokens are part of the context
@@ -60,14 +61,20 @@ def sdpa_reference(w: W.Workload) -> np.ndarray:
         Q = w.q[int(cu[b]) : int(cu[b + 1])].double().permute(1, 0, 2)  # [H_q, qb, d]
         i = torch.arange(qb).unsqueeze(1)
         j = torch.arange(ctx).unsqueeze(0)
-        mask = j <= (ctx - qb + i)
+        if tree_mask is None:
+            mask = j <= (ctx - qb + i)
+        else:
+            bits = tree_mask[int(cu[b]) : int(cu[b + 1])].long().unsqueeze(1)  # [qb, 1]
+            new = j - (ctx - qb)                                               # index among the new tokens
+            mask = (new < 0) | ((bits >> new.clamp(min=0)) & 1).bool()
         o = F.scaled_dot_product_attention(Q, K, V, attn_mask=mask, scale=w.scale)
         out[int(cu[b]) : int(cu[b + 1])] = o.permute(1, 0, 2)
     return out.numpy()
 
 
-def oracle_step(w: W.Workload, L, rows=None, n_threads: int = 0):
-    """Run the step on the oracle: block copies, cache write, then attention over all sequences."""
+def oracle_step(w: W.Workload, L, rows=None, n_threads: int = 0, tree_mask=None):
+    """Run the step on the oracle: block copies, cache write, then attention over all sequences
+    (tree-attention verification when ``tree_mask`` is given)."""
     kc = oracle._u16(w.key_cache).copy()
     vc = oracle._u16(w.value_cache).copy()
     if w.copy_pairs is not None:
@@ -75,7 +82,7 @@ def oracle_step(w: W.Workload, L, rows=None, n_threads: int = 0):
     assert oracle.kv_cache_write(w.k_new, w.v_new, w.slot_mapping, kc, vc, L=L) == 0
     out = oracle.paged_attention(
         w.q, kc, vc, oracle.dtype_code(w.dtype), w.block_tables, w.cu_seqlens_q, w.context_lens, w.H_kv,
-        w.scale, rows=rows, n_threads=n_threads, L=L,
+        w.scale, rows=rows, n_threads=n_threads, L=L, tree_mask=tree_mask,
     )
     return out, kc, vc
 
@@ -197,6 +204,27 @@ def pin_sdpa_library(L):
         ref = sdpa_reference(w)
         err = np.abs(got - ref).max()
         assert err < 1e-12, f"{w.name}: oracle vs SDPA max err {err}"
+
+
+def pin_tree_verify(L):
+    """Tree-attention verification == torch fp64 SDPA with the tree's boolean mask; the chain mask
+    reproduces the causal verify exactly."""
+    for k, w in enumerate(_small_cases()):
+        if max(w.q_lens) > 8:
+            continue
+        tm = W.random_tree_masks(300 + k, w.q_lens)
+        got, _, _ = oracle_step(w, L, tree_mask=tm)
+        ref = sdpa_reference(w, tree_mask=tm)
+        err = np.abs(got - ref).max()
+        assert err < 1e-12, f"{w.name}: tree oracle vs SDPA max err {err}"
+        causal, _, _ = oracle_step(w, L)
+        chain, _, _ = oracle_step(w, L, tree_mask=W.chain_masks(w.q_lens))
+        assert np.array_equal(causal, chain)
+    # a forest where some tokens see no other draft: only their own bit
+    w = _small_cases()[2]
+    solo = torch.tensor([1 << i for qb in w.q_lens for i in range(int(qb))], dtype=torch.int32)
+    got, _, _ = oracle_step(w, L, tree_mask=solo)
+    assert np.abs(got - sdpa_reference(w, tree_mask=solo)).max() < 1e-12
 
 
 def pin_dense_three_pass(L):
@@ -454,6 +482,7 @@ ALL_PINS = [
     pin_block_copy,
     pin_block_swap,
     pin_sdpa_library,
+    pin_tree_verify,
     pin_dense_three_pass,
     pin_block_permutation,
     pin_paged_equals_contiguous,

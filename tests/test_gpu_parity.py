@@ -130,6 +130,83 @@ def test_prefill_fresh_prompts_exact_lengths():
     run_and_compare(w)
 
 
+# ---- tree-attention verification ---------------------------------------------------------
+
+def _tree_run(w, tm):
+    """Cache write, then the tree-verify decode on the device; returns (output, step)."""
+    st = DeviceStep(w)
+    st.copy_blocks()
+    st.write()
+    call = st.calls[0]
+    out = pa.paged_attn_decode_tree(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, tm.cuda(),
+                                    call.max_ctx, w.scale, out=call.out, workspace=call.ws)
+    torch.cuda.synchronize()
+    assert st.statuses() == [0] * (1 + len(st.calls)), st.statuses()
+    return out, st
+
+
+TREE_CASES = [
+    (4, 8, 500, 2, 4, 128, W.BF16),
+    (3, 8, 300, 2, 8, 64, W.F16),
+    (5, 6, 2000, 2, 4, 128, W.BF16),  # several splits
+    (2, 8, 40, 1, 16, 128, W.BF16),   # two row groups, short contexts
+    (4, 5, 9, 2, 1, 64, W.F16),       # contexts barely longer than the drafts
+]
+
+
+@pytest.mark.parametrize("idx", range(len(TREE_CASES)), ids=lambda i: _case_id(TREE_CASES[i]))
+def test_tree_verify_small(idx):
+    B, q_max, ctx_max, H_kv, G, d, dt = TREE_CASES[idx]
+    w = W.random_workload(500 + 13 * idx, B=B, q_max=q_max, ctx_max=ctx_max, H_kv=H_kv, G=G, d=d, dtype=dt,
+                          kind="decode")
+    tm = W.random_tree_masks(600 + idx, w.q_lens)
+    out, _ = _tree_run(w, tm)
+    ref, _, _ = oracle_step(w, oracle.lib(), tree_mask=tm)
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref).max()
+    assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
+
+
+def test_tree_chain_mask_is_the_causal_verify():
+    # the chain mask takes exactly the decisions of the causal rule: the same bits out
+    w = W.random_workload(71, B=5, q_max=8, ctx_max=900, H_kv=2, G=4, d=128, dtype=W.BF16, kind="decode")
+    st = DeviceStep(w)
+    causal = st.run().clone()
+    torch.cuda.synchronize()
+    tree, _ = _tree_run(w, W.chain_masks(w.q_lens))
+    assert torch.equal(causal.view(torch.int16), tree.view(torch.int16))
+
+
+def test_tree_verify_full_size_sampled():
+    # the benchmark's tree-verify workload (64 x 8 drafts, contexts U[512, 4096], 32/8 heads)
+    w = W.tree_verify()
+    tm = W.random_tree_masks(34_105, w.q_lens)
+    out, _ = _tree_run(w, tm)
+    rows = sample_rows(w, 300, seed=5)
+    ref, _, _ = oracle_step(w, oracle.lib(), rows=rows, tree_mask=tm)
+    got = out.double().cpu().numpy().reshape(w.T * w.H_q, w.d)[rows]
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref).max()
+    assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
+
+
+def test_tree_verify_rejects_a_missing_mask():
+    import ctypes
+
+    w = W.random_workload(3, B=2, q_max=4, ctx_max=50, H_kv=1, G=2, d=64, dtype=W.F16, kind="decode")
+    st = DeviceStep(w)
+    call = st.calls[0]
+    n0 = pa.launch_count()
+    rc = pa.lib().pa_paged_attn_decode_tree(
+        ctypes.c_void_p(call.out.data_ptr()), ctypes.c_void_p(call.q.data_ptr()),
+        ctypes.c_void_p(st.key_cache.data_ptr()), ctypes.c_void_p(st.value_cache.data_ptr()), st.key_cache.shape[0],
+        ctypes.c_void_p(call.bt.data_ptr()), call.bt.shape[1], ctypes.c_void_p(call.cu.data_ptr()),
+        ctypes.c_void_p(call.ctx.data_ptr()), None, call.ctx.shape[0], call.max_ctx, call.q.shape[0], w.H_q, w.H_kv,
+        w.d, w.scale, 0, ctypes.c_void_p(call.ws.data_ptr()), call.ws.numel(), None)
+    assert rc == -1 and pa.launch_count() == n0
+
+
 # ---- the five configurations ----------------------------------------------------------------
 
 def test_config1_tiny_decode_all_rows():

@@ -53,6 +53,14 @@ MUTANTS = {
         "host_key[hst * per_block + e] = key_cache[dev * per_block + e];",
         "host_key[dev * per_block + e] = key_cache[dev * per_block + e];",
     ),
+    "tree_bit_off_by_one": (
+        "return !tree || j < base || ((*tree >> (j - base)) & 1);",
+        "return !tree || j < base || ((*tree >> (j - base + 1)) & 1);",
+    ),
+    "tree_hides_context": (
+        "return !tree || j < base || ((*tree >> (j - base)) & 1);",
+        "return !tree || ((*tree >> (j - base)) & 1);",
+    ),
     "online_no_rescale": ("o[c] = alpha * o[c] + acc;", "o[c] = o[c] + acc;"),
     "merge_sign": ("double w = exp(lses[s] - m) / z;", "double w = exp(m - lses[s]) / z;"),
 }
