@@ -43,6 +43,17 @@ def _declare(L):
     L.oracle_kv_cache_write.argtypes = [P, P, P, c.c_int64, P, P, c.c_int64, c.c_int, c.c_int]
     L.oracle_kv_block_copy.restype = c.c_int64
     L.oracle_kv_block_copy.argtypes = [P, P, c.c_int64, c.c_int, c.c_int, P, c.c_int64]
+    L.oracle_e4m3_to_f64.restype = c.c_double
+    L.oracle_e4m3_to_f64.argtypes = [c.c_uint8]
+    L.oracle_f64_to_e4m3.restype = c.c_uint8
+    L.oracle_f64_to_e4m3.argtypes = [c.c_double]
+    L.oracle_kv_cache_write_fp8.restype = c.c_int64
+    L.oracle_kv_cache_write_fp8.argtypes = [P, P, c.c_int, P, c.c_int64, P, P, P, P, c.c_int64, c.c_int, c.c_int]
+    L.oracle_paged_attention_fp8.restype = c.c_int
+    L.oracle_paged_attention_fp8.argtypes = [
+        P, P, c.c_int, P, P, P, P, P, c.c_int, P, P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_double, P, c.c_int64,
+        c.c_int,
+    ]
     L.oracle_kv_block_swap.restype = c.c_int64
     L.oracle_kv_block_swap.argtypes = [P, P, c.c_int64, P, P, c.c_int64, c.c_int, c.c_int, P, c.c_int64, c.c_int]
     L.oracle_paged_attention.restype = c.c_int
@@ -137,6 +148,50 @@ def kv_block_copy(key_cache: np.ndarray, value_cache: np.ndarray, pairs, L=None)
     pr = _i32(pairs).reshape(-1, 2)
     NB, H_kv, _, d = key_cache.shape
     return (L or lib()).oracle_kv_block_copy(_p(key_cache), _p(value_cache), NB, H_kv, d, _p(pr), pr.shape[0])
+
+
+def e4m3_to_f64(code: int, L=None) -> float:
+    return (L or lib()).oracle_e4m3_to_f64(code)
+
+
+def f64_to_e4m3(x: float, L=None) -> int:
+    return (L or lib()).oracle_f64_to_e4m3(float(x))
+
+
+def kv_cache_write_fp8(k_new, v_new, dtype: int, slot_mapping, key_cache: np.ndarray, value_cache: np.ndarray,
+                       key_scale: np.ndarray, value_scale: np.ndarray, L=None) -> int:
+    """FP8 cache write: codes uint8 [NB, H_kv, 16, d], scales float32 [NB, H_kv, 16]; in place."""
+    kn, vn = _u16(k_new), _u16(v_new)
+    sm = _i32(slot_mapping)
+    NB, H_kv, _, d = key_cache.shape
+    for a, dt in ((key_cache, np.uint8), (value_cache, np.uint8), (key_scale, np.float32), (value_scale, np.float32)):
+        assert a.dtype == dt and a.flags.c_contiguous
+    return (L or lib()).oracle_kv_cache_write_fp8(_p(kn), _p(vn), dtype, _p(sm), sm.shape[0], _p(key_cache),
+                                                  _p(value_cache), _p(key_scale), _p(value_scale), NB, H_kv, d)
+
+
+def paged_attention_fp8(q, dtype: int, key_cache: np.ndarray, value_cache: np.ndarray, key_scale: np.ndarray,
+                        value_scale: np.ndarray, block_tables, cu_seqlens_q, context_lens, H_kv: int, scale: float,
+                        rows: Optional[np.ndarray] = None, n_threads: int = 0, L=None):
+    """fp64 attention over the FP8 cache (K and V dequantised exactly: code value x row scale)."""
+    qq = _u16(q)
+    T, H_q, d = qq.shape
+    bt, cu, cl = _i32(block_tables), _i32(cu_seqlens_q), _i32(context_lens)
+    B = cl.shape[0]
+    if rows is None:
+        out = np.empty((T, H_q, d), dtype=np.float64)
+        n_rows, r = T * H_q, None
+    else:
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        n_rows = r.shape[0]
+        out = np.empty((n_rows, d), dtype=np.float64)
+    rc = (L or lib()).oracle_paged_attention_fp8(
+        _p(out), _p(qq), dtype, _p(key_cache), _p(value_cache), _p(key_scale), _p(value_scale), _p(bt), bt.shape[1],
+        _p(cu), _p(cl), B, H_q, H_kv, d, float(scale), _p(r), n_rows, n_threads,
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_paged_attention_fp8 rejected its arguments (code {rc})")
+    return out
 
 
 def kv_block_swap(key_cache: np.ndarray, value_cache: np.ndarray, host_key: np.ndarray, host_value: np.ndarray,

@@ -197,6 +197,103 @@ def pin_block_swap(L):
     assert np.array_equal(before[0], k16) and np.array_equal(before[1], hk)
 
 
+def _e4m3_values(codes) -> torch.Tensor:
+    """E4M3 codes -> float64 through torch's float8_e4m3fn (a decoder independent of the oracle)."""
+    return torch.as_tensor(codes, dtype=torch.uint8).view(torch.float8_e4m3fn).double()
+
+
+def pin_e4m3_codec(L):
+    """The oracle's E4M3 decode and nearest-even encode against the format's definition (worked
+    codes), torch's float8_e4m3fn decoder and encoder (finite range), and saturation at +-448."""
+    worked = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x3F: 1.875, 0x40: 2.0,
+              0x70: 128.0, 0x77: 240.0, 0x7E: 448.0, 0xFE: -448.0, 0xB8: -1.0}
+    for c, v in worked.items():
+        assert oracle.e4m3_to_f64(c, L=L) == v, hex(c)
+    assert math.isnan(oracle.e4m3_to_f64(0x7F, L=L)) and math.isnan(oracle.e4m3_to_f64(0xFF, L=L))
+    finite = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    ref = _e4m3_values(finite).tolist()
+    for c, v in zip(finite, ref):
+        assert oracle.e4m3_to_f64(c, L=L) == v, hex(c)
+        assert oracle.f64_to_e4m3(v, L=L) == c, hex(c)  # every code round-trips (including -0)
+    g = torch.Generator().manual_seed(8)
+    xs = torch.cat([torch.randn(3000, generator=g) * 40, torch.randn(1000, generator=g) * 0.01,
+                    (torch.rand(1000, generator=g) * 2 - 1) * 447.9])
+    want = xs.to(torch.float8_e4m3fn).view(torch.uint8).tolist()
+    for x, c in zip(xs.tolist(), want):
+        assert oracle.f64_to_e4m3(x, L=L) == c, (x, c)
+    # ties go to the even code; beyond 448 the codes saturate
+    assert oracle.f64_to_e4m3(1.0625, L=L) == 0x38 and oracle.f64_to_e4m3(1.1875, L=L) == 0x3A
+    assert oracle.f64_to_e4m3(1.5 * 2.0 ** -9, L=L) == 0x02 and oracle.f64_to_e4m3(0.5 * 2.0 ** -9, L=L) == 0x00
+    for x in (448.5, 464.0, 500.0, 1e30):
+        assert oracle.f64_to_e4m3(x, L=L) == 0x7E and oracle.f64_to_e4m3(-x, L=L) == 0xFE
+
+
+def _fp8_case(seed, B=3, q_max=1, ctx_max=60, H_kv=2, G=2, d=32, dt=W.BF16):
+    """A small decode workload with its cache written to FP8 by the oracle (every context row)."""
+    w = W.random_workload(seed, B=B, q_max=q_max, ctx_max=ctx_max, H_kv=H_kv, G=G, d=d, dtype=dt, kind="decode")
+    NB = w.key_cache.shape[0]
+    kc8 = np.zeros((NB, H_kv, 16, d), np.uint8)
+    vc8 = np.zeros((NB, H_kv, 16, d), np.uint8)
+    ks = np.ones((NB, H_kv, 16), np.float32)
+    vs = np.ones((NB, H_kv, 16), np.float32)
+    # every stored row (the cached context and the step's new tokens) goes through the FP8 write
+    rows_k = w.key_cache.reshape(NB, H_kv, 16, d).permute(0, 2, 1, 3).reshape(NB * 16, H_kv, d)
+    rows_v = w.value_cache.reshape(NB, H_kv, 16, d).permute(0, 2, 1, 3).reshape(NB * 16, H_kv, d)
+    slots = torch.arange(NB * 16, dtype=torch.int32)
+    dtc = oracle.dtype_code(w.dtype)
+    assert oracle.kv_cache_write_fp8(rows_k.contiguous(), rows_v.contiguous(), dtc, slots, kc8, vc8, ks, vs) == 0
+    assert oracle.kv_cache_write_fp8(w.k_new, w.v_new, dtc, w.slot_mapping, kc8, vc8, ks, vs) == 0
+    return w, kc8, vc8, ks, vs
+
+
+def pin_fp8_write(L):
+    """FP8 write: the row maximum lands on 448 exactly, the scale is amax / 448 in float, every
+    value is within half an E4M3 step of the original, a zero row gets scale 1; bad slots count."""
+    g = torch.Generator().manual_seed(12)
+    T, H, d = 6, 3, 64
+    kn = torch.randn((T, H, d), generator=g).bfloat16()
+    vn = (torch.randn((T, H, d), generator=g) * 30).bfloat16()
+    vn[2, 1] = 0
+    NB = 2
+    kc8, vc8 = np.zeros((NB, H, 16, d), np.uint8), np.zeros((NB, H, 16, d), np.uint8)
+    ks, vs = np.zeros((NB, H, 16), np.float32), np.zeros((NB, H, 16), np.float32)
+    slots = torch.tensor([0, 5, 17, 31, -1, 16], dtype=torch.int32)
+    assert oracle.kv_cache_write_fp8(kn, vn, oracle.dtype_code(W.BF16), slots, kc8, vc8, ks, vs, L=L) == 0
+    for t, sl in enumerate(slots.tolist()):
+        if sl < 0:
+            continue
+        for h in range(H):
+            for new, c8, sc in ((kn, kc8, ks), (vn, vc8, vs)):
+                x = new[t, h].double()
+                amax = float(x.abs().max())
+                s_ref = np.float32(amax) / np.float32(448.0) if amax > 0 else np.float32(1.0)
+                assert sc[sl // 16, h, sl % 16] == s_ref
+                deq = _e4m3_values(c8[sl // 16, h, sl % 16]) * float(s_ref)
+                if amax > 0:
+                    assert float(deq.abs().max()) == 448.0 * float(s_ref)
+                # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 for normals, absolute 2^-10 * scale below
+                bound = torch.maximum(x.abs() * 2.0 ** -4, torch.full_like(x, 2.0 ** -10 * float(s_ref)))
+                assert bool(((deq - x).abs() <= bound + 1e-12).all())
+    assert not vc8[1, 1, 1].any() and vs[1, 1, 1] == 1.0  # the zero row (token 2 -> slot 17)
+    assert oracle.kv_cache_write_fp8(kn[:1], vn[:1], oracle.dtype_code(W.BF16), torch.tensor([NB * 16], dtype=torch.int32), kc8, vc8,
+                                     ks, vs, L=L) == 1
+
+
+def pin_fp8_attention(L):
+    """Attention over the FP8 cache == torch fp64 SDPA on the cache dequantised through torch's
+    float8 decoder (ragged, GQA, causal verify rows)."""
+    for seed, kw in ((21, {}), (22, dict(q_max=6, G=4, d=64, dt=W.F16)), (23, dict(B=2, q_max=3, ctx_max=90))):
+        w, kc8, vc8, ks, vs = _fp8_case(seed, **kw)
+        got = oracle.paged_attention_fp8(w.q, oracle.dtype_code(w.dtype), kc8, vc8, ks, vs, w.block_tables,
+                                         w.cu_seqlens_q, w.context_lens, w.H_kv, w.scale, L=L)
+        deq = lambda c8, sc: (_e4m3_values(c8.reshape(-1)).reshape(c8.shape) * torch.from_numpy(sc).double()[..., None])
+        w2 = W.Workload(**{**vars(w), "key_cache": deq(kc8, ks), "value_cache": deq(vc8, vs),
+                           "slot_mapping": torch.full_like(w.slot_mapping, -1)})
+        ref = sdpa_reference(w2)
+        err = np.abs(got - ref).max()
+        assert err < 1e-12, f"fp8 oracle vs SDPA max err {err}"
+
+
 def pin_sdpa_library(L):
     """Paged fp64 oracle == torch fp64 SDPA on the gathered contiguous K/V (ragged, GQA, causal)."""
     for w in _small_cases():
@@ -481,6 +578,9 @@ ALL_PINS = [
     pin_cache_write,
     pin_block_copy,
     pin_block_swap,
+    pin_e4m3_codec,
+    pin_fp8_write,
+    pin_fp8_attention,
     pin_sdpa_library,
     pin_tree_verify,
     pin_dense_three_pass,

@@ -61,6 +61,11 @@ MUTANTS = {
         "return !tree || j < base || ((*tree >> (j - base)) & 1);",
         "return !tree || ((*tree >> (j - base)) & 1);",
     ),
+    "e4m3_bias": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "fp8_scale_constant": ("float sc = amax > 0.0f ? amax / 448.0f : 1.0f;",
+                           "float sc = amax > 0.0f ? amax / 240.0f : 1.0f;"),
+    "fp8_value_scale_from_keys": ("double w = s[j] / z, vs = value_scale[row];",
+                                  "double w = s[j] / z, vs = key_scale[row];"),
     "online_no_rescale": ("o[c] = alpha * o[c] + acc;", "o[c] = o[c] + acc;"),
     "merge_sign": ("double w = exp(lses[s] - m) / z;", "double w = exp(m - lses[s]) / z;"),
 }
