@@ -173,183 +173,6 @@ int64_t oracle_kv_block_swap(uint16_t *key_cache, uint16_t *value_cache, int64_t
     return bad;
 }
 
-/* ---- FP8 (E4M3) KV cache ------------------------------------------------------
- * An 8-bit cache with one float scale per stored row (token, KV head): the FP8 KV cache of the
- * serving pages (vLLM's fp8 KV-cache option; FP8 with scaling on the interview Q&A page).  The
- * scale of a row is set when the row is written, amax / 448, so nothing already stored ever has
- * to be requantised.  E4M3 (OCP 8-bit floating point): sign, 4 exponent bits with bias 7, 3
- * mantissa bits, subnormals, no infinities, S.1111.111 = NaN, largest finite 448. */
-
-double oracle_e4m3_to_f64(uint8_t c)
-{
-    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
-    double v;
-    if (e == 15 && m == 7)
-        return NAN;
-    if (e == 0)
-        v = ldexp((double)m / 8.0, -6); /* subnormal: 0.m x 2^-6 */
-    else
-        v = ldexp(1.0 + (double)m / 8.0, e - 7);
-    return s ? -v : v;
-}
-
-/* The E4M3 code nearest to x (ties to the code with an even last bit), saturated to +-448:
- * every finite non-negative code is tried. */
-uint8_t oracle_f64_to_e4m3(double x)
-{
-    if (isnan(x))
-        return 0x7f;
-    uint8_t sign = signbit(x) ? 0x80 : 0x00;
-    double a = fabs(x);
-    if (a >= 448.0)
-        return sign | 0x7e;
-    int best = 0;
-    double best_err = INFINITY;
-    for (int c = 0; c <= 0x7e; ++c) {
-        double err = fabs(a - oracle_e4m3_to_f64((uint8_t)c));
-        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
-            best = c;
-            best_err = err;
-        }
-    }
-    return sign | (uint8_t)best;
-}
-
-/* One row of d 16-bit values -> d codes and the row's scale: scale = amax / 448 (1 when amax is
- * 0), code_k = e4m3(x_k / scale), both divisions in float rounded to nearest, as the device does. */
-static float quant_row(const uint16_t *src, int dtype, int d, uint8_t *dst)
-{
-    float amax = 0.0f;
-    for (int k = 0; k < d; ++k) {
-        float v = fabsf((float)widen(src[k], dtype));
-        if (v > amax)
-            amax = v;
-    }
-    float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
-    for (int k = 0; k < d; ++k) {
-        float q = (float)widen(src[k], dtype) / sc;
-        dst[k] = oracle_f64_to_e4m3((double)q);
-    }
-    return sc;
-}
-
-/* kv_cache_write into the FP8 cache: codes [NB][H_kv][16][d], scales [NB][H_kv][16]. */
-int64_t oracle_kv_cache_write_fp8(const uint16_t *k_new, const uint16_t *v_new, int dtype,
-                                  const int32_t *slot_mapping, int64_t T, uint8_t *key_cache, uint8_t *value_cache,
-                                  float *key_scale, float *value_scale, int64_t num_blocks, int H_kv, int d)
-{
-    int64_t bad = 0;
-    for (int64_t t = 0; t < T; ++t) {
-        int64_t slot = slot_mapping[t];
-        if (slot < 0)
-            continue; /* padding token */
-        if (slot >= num_blocks * ORACLE_BLOCK) {
-            ++bad;
-            continue;
-        }
-        int64_t block = slot / ORACLE_BLOCK;
-        int64_t offset = slot % ORACLE_BLOCK;
-        for (int h = 0; h < H_kv; ++h) {
-            int64_t row = (block * H_kv + h) * ORACLE_BLOCK + offset;
-            int64_t src = (t * H_kv + h) * (int64_t)d;
-            key_scale[row] = quant_row(k_new + src, dtype, d, key_cache + row * d);
-            value_scale[row] = quant_row(v_new + src, dtype, d, value_cache + row * d);
-        }
-    }
-    return bad;
-}
-
-/* Attention of one row over the FP8 cache: K_j = e4m3(code) * scale of its row, likewise V. */
-static int attention_row_fp8(double *out_row, const uint16_t *q, int dtype, const uint8_t *key_cache,
-                             const uint8_t *value_cache, const float *key_scale, const float *value_scale,
-                             const int32_t *block_tables, int max_blocks, int b, int i, int q_b, int ctx_b,
-                             int64_t t, int h, int H_q, int H_kv, int d, double scale, double *s)
-{
-    int G = H_q / H_kv;
-    int g = h / G;
-    int last = ctx_b - q_b + i; /* causal: keys 0 .. last */
-    if (last < 0)
-        return -1;
-    const uint16_t *qrow = q + (t * H_q + h) * (int64_t)d;
-    for (int j = 0; j <= last; ++j) {
-        int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
-        int64_t row = (block * H_kv + g) * ORACLE_BLOCK + j % ORACLE_BLOCK;
-        double ks = key_scale[row], acc = 0.0;
-        for (int k = 0; k < d; ++k)
-            acc += widen(qrow[k], dtype) * (oracle_e4m3_to_f64(key_cache[row * d + k]) * ks);
-        s[j] = scale * acc;
-    }
-    double m = -INFINITY;
-    for (int j = 0; j <= last; ++j)
-        if (s[j] > m)
-            m = s[j];
-    double z = 0.0;
-    for (int j = 0; j <= last; ++j) {
-        s[j] = exp(s[j] - m);
-        z += s[j];
-    }
-    for (int k = 0; k < d; ++k)
-        out_row[k] = 0.0;
-    for (int j = 0; j <= last; ++j) {
-        int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
-        int64_t row = (block * H_kv + g) * ORACLE_BLOCK + j % ORACLE_BLOCK;
-        double w = s[j] / z, vs = value_scale[row];
-        for (int k = 0; k < d; ++k)
-            out_row[k] += w * (oracle_e4m3_to_f64(value_cache[row * d + k]) * vs);
-    }
-    return 0;
-}
-
-int oracle_paged_attention_fp8(double *out, const uint16_t *q, int dtype, const uint8_t *key_cache,
-                               const uint8_t *value_cache, const float *key_scale, const float *value_scale,
-                               const int32_t *block_tables, int max_blocks, const int32_t *cu_seqlens_q,
-                               const int32_t *context_lens, int B, int H_q, int H_kv, int d, double scale,
-                               const int64_t *rows, int64_t n_rows, int n_threads)
-{
-    if (H_kv <= 0 || H_q % H_kv != 0)
-        return -2;
-    int max_ctx = 0;
-    for (int b = 0; b < B; ++b) {
-        int q_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
-        if (q_b < 0 || context_lens[b] < q_b)
-            return -1;
-        if (context_lens[b] > max_ctx)
-            max_ctx = context_lens[b];
-    }
-    int64_t T = cu_seqlens_q[B];
-    int64_t total = rows ? n_rows : T * H_q;
-    int status = 0;
-#ifdef _OPENMP
-    if (n_threads > 0)
-        omp_set_num_threads(n_threads);
-#else
-    (void)n_threads;
-#endif
-#pragma omp parallel
-    {
-        double *s = (double *)malloc(sizeof(double) * (size_t)(max_ctx > 0 ? max_ctx : 1));
-#pragma omp for schedule(dynamic, 1)
-        for (int64_t r = 0; r < total; ++r) {
-            int64_t row = rows ? rows[r] : r;
-            int64_t t = row / H_q;
-            int h = (int)(row % H_q);
-            int b = 0;
-            while (b < B && cu_seqlens_q[b + 1] <= t)
-                ++b;
-            int i = (int)(t - cu_seqlens_q[b]);
-            int q_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
-            if (attention_row_fp8(out + r * d, q, dtype, key_cache, value_cache, key_scale, value_scale,
-                                  block_tables, max_blocks, b, i, q_b, context_lens[b], t, h, H_q, H_kv, d, scale,
-                                  s)) {
-#pragma omp atomic write
-                status = -1;
-            }
-        }
-        free(s);
-    }
-    return status;
-}
-
 /* ---- attention over the paged cache ---------------------------------------- */
 
 /* One output row: query token t (of sequence b, index i within its q_b new
@@ -644,4 +467,181 @@ void oracle_lse_merge(double *out, double *lse_out, const double *parts, const d
             out[c] += w * parts[(int64_t)s * d + c];
     }
     *lse_out = m + log(z);
+}
+
+/* ---- FP8 (E4M3) KV cache ------------------------------------------------------
+ * An 8-bit cache with one float scale per stored row (token, KV head): the FP8 KV cache of the
+ * serving pages (vLLM's fp8 KV-cache option; FP8 with scaling on the interview Q&A page).  The
+ * scale of a row is set when the row is written, amax / 448, so nothing already stored ever has
+ * to be requantised.  E4M3 (OCP 8-bit floating point): sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, subnormals, no infinities, S.1111.111 = NaN, largest finite 448. */
+
+double oracle_e4m3_to_f64(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6); /* subnormal: 0.m x 2^-6 */
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* The E4M3 code nearest to x (ties to the code with an even last bit), saturated to +-448:
+ * every finite non-negative code is tried. */
+uint8_t oracle_f64_to_e4m3(double x)
+{
+    if (isnan(x))
+        return 0x7f;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0)
+        return sign | 0x7e;
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7e; ++c) {
+        double err = fabs(a - oracle_e4m3_to_f64((uint8_t)c));
+        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* One row of d 16-bit values -> d codes and the row's scale: scale = amax / 448 (1 when amax is
+ * 0), code_k = e4m3(x_k / scale), both divisions in float rounded to nearest, as the device does. */
+static float quant_row(const uint16_t *src, int dtype, int d, uint8_t *dst)
+{
+    float amax = 0.0f;
+    for (int k = 0; k < d; ++k) {
+        float v = fabsf((float)widen(src[k], dtype));
+        if (v > amax)
+            amax = v;
+    }
+    float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
+    for (int k = 0; k < d; ++k) {
+        float q = (float)widen(src[k], dtype) / sc;
+        dst[k] = oracle_f64_to_e4m3((double)q);
+    }
+    return sc;
+}
+
+/* kv_cache_write into the FP8 cache: codes [NB][H_kv][16][d], scales [NB][H_kv][16]. */
+int64_t oracle_kv_cache_write_fp8(const uint16_t *k_new, const uint16_t *v_new, int dtype,
+                                  const int32_t *slot_mapping, int64_t T, uint8_t *key_cache, uint8_t *value_cache,
+                                  float *key_scale, float *value_scale, int64_t num_blocks, int H_kv, int d)
+{
+    int64_t bad = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue; /* padding token */
+        if (slot >= num_blocks * ORACLE_BLOCK) {
+            ++bad;
+            continue;
+        }
+        int64_t block = slot / ORACLE_BLOCK;
+        int64_t offset = slot % ORACLE_BLOCK;
+        for (int h = 0; h < H_kv; ++h) {
+            int64_t row = (block * H_kv + h) * ORACLE_BLOCK + offset;
+            int64_t src = (t * H_kv + h) * (int64_t)d;
+            key_scale[row] = quant_row(k_new + src, dtype, d, key_cache + row * d);
+            value_scale[row] = quant_row(v_new + src, dtype, d, value_cache + row * d);
+        }
+    }
+    return bad;
+}
+
+/* Attention of one row over the FP8 cache: K_j = e4m3(code) * scale of its row, likewise V. */
+static int attention_row_fp8(double *out_row, const uint16_t *q, int dtype, const uint8_t *key_cache,
+                             const uint8_t *value_cache, const float *key_scale, const float *value_scale,
+                             const int32_t *block_tables, int max_blocks, int b, int i, int q_b, int ctx_b,
+                             int64_t t, int h, int H_q, int H_kv, int d, double scale, double *s)
+{
+    int G = H_q / H_kv;
+    int g = h / G;
+    int last = ctx_b - q_b + i; /* causal: keys 0 .. last */
+    if (last < 0)
+        return -1;
+    const uint16_t *qrow = q + (t * H_q + h) * (int64_t)d;
+    for (int j = 0; j <= last; ++j) {
+        int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
+        int64_t row = (block * H_kv + g) * ORACLE_BLOCK + j % ORACLE_BLOCK;
+        double ks = key_scale[row], acc = 0.0;
+        for (int k = 0; k < d; ++k)
+            acc += widen(qrow[k], dtype) * (oracle_e4m3_to_f64(key_cache[row * d + k]) * ks);
+        s[j] = scale * acc;
+    }
+    double m = -INFINITY;
+    for (int j = 0; j <= last; ++j)
+        if (s[j] > m)
+            m = s[j];
+    double z = 0.0;
+    for (int j = 0; j <= last; ++j) {
+        s[j] = exp(s[j] - m);
+        z += s[j];
+    }
+    for (int k = 0; k < d; ++k)
+        out_row[k] = 0.0;
+    for (int j = 0; j <= last; ++j) {
+        int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
+        int64_t row = (block * H_kv + g) * ORACLE_BLOCK + j % ORACLE_BLOCK;
+        double w = s[j] / z, vs = value_scale[row];
+        for (int k = 0; k < d; ++k)
+            out_row[k] += w * (oracle_e4m3_to_f64(value_cache[row * d + k]) * vs);
+    }
+    return 0;
+}
+
+int oracle_paged_attention_fp8(double *out, const uint16_t *q, int dtype, const uint8_t *key_cache,
+                               const uint8_t *value_cache, const float *key_scale, const float *value_scale,
+                               const int32_t *block_tables, int max_blocks, const int32_t *cu_seqlens_q,
+                               const int32_t *context_lens, int B, int H_q, int H_kv, int d, double scale,
+                               const int64_t *rows, int64_t n_rows, int n_threads)
+{
+    if (H_kv <= 0 || H_q % H_kv != 0)
+        return -2;
+    int max_ctx = 0;
+    for (int b = 0; b < B; ++b) {
+        int q_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+        if (q_b < 0 || context_lens[b] < q_b)
+            return -1;
+        if (context_lens[b] > max_ctx)
+            max_ctx = context_lens[b];
+    }
+    int64_t T = cu_seqlens_q[B];
+    int64_t total = rows ? n_rows : T * H_q;
+    int status = 0;
+#ifdef _OPENMP
+    if (n_threads > 0)
+        omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(max_ctx > 0 ? max_ctx : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < total; ++r) {
+            int64_t row = rows ? rows[r] : r;
+            int64_t t = row / H_q;
+            int h = (int)(row % H_q);
+            int b = 0;
+            while (b < B && cu_seqlens_q[b + 1] <= t)
+                ++b;
+            int i = (int)(t - cu_seqlens_q[b]);
+            int q_b = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+            if (attention_row_fp8(out + r * d, q, dtype, key_cache, value_cache, key_scale, value_scale,
+                                  block_tables, max_blocks, b, i, q_b, context_lens[b], t, h, H_q, H_kv, d, scale,
+                                  s)) {
+#pragma omp atomic write
+                status = -1;
+            }
+        }
+        free(s);
+    }
+    return status;
 }
