@@ -20,7 +20,8 @@ The same JSON line carries:
   prefill       causal varlen prefill (8 prompts U[256,2048], 40/40 heads, bf16):
                 TFLOP/s of exact causal pairs vs the measured bf16 peak
   legs          the GQA shared-prefix decode step, the mixed continuous-batching step, the
-                tree-attention verify of speculative drafts (HBM roofline), and
+                tree-attention verify of speculative drafts (HBM roofline), the FP8 (E4M3) KV
+                cache on the 13B decode layer (HBM roofline, speed-up over 16 bits), and
                 the preemption swap of KV blocks to a pinned host pool and back (GB/s against
                 a plain pinned cudaMemcpyAsync of the same bytes)
   e2e           the same metric with host buffers: every step's inputs go H2D from one pinned
@@ -355,6 +356,7 @@ def run_ours(args):
             "gqa_shared_prefix": leg_gqa(args, stream, device, hbm_peak, rank),
             "mixed_step": leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank),
             "tree_verify": leg_tree(args, stream, device, hbm_peak, rank),
+            "fp8_cache": leg_fp8(args, stream, device, hbm_peak, rank),
             "block_swap": leg_swap(args, stream, device, rank),
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -516,6 +518,61 @@ def leg_gqa(args, stream, device, hbm_peak, rank):
             "unique_bytes": b, "decode_ms": round(ms, 5), "step_ms": round(step_ms, 5),
             "per_call_ms": {k: round(v, 5) for k, v in per.items()},
             "note": "shared prefix counted once; its blocks may stay in L2 across sequences"}
+
+
+def leg_fp8(args, stream, device, hbm_peak, rank):
+    """FP8 (E4M3) KV cache on the 13B-shaped decode layer (64 sequences, 40/40 heads, d 128, contexts
+    U[128, 4096], fp16 Q): cache written through the FP8 write, then the FP8 decode timed alone and
+    beside the 16-bit decode of the same data.  Algorithmic bytes: every context key's K and V codes
+    (1 byte per value) and their two row scales, Q, O and the table entries."""
+    import torch
+
+    import paged_kv_attention_34_b200 as pa
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import DeviceStep, attn_bytes
+
+    w = W.config2(seed=shard_seed(34_002, rank), fill="zero")
+    with torch.cuda.stream(stream):
+        st = DeviceStep(w, device=device)
+    call = st.calls[0]
+    NB, H, _, d = st.key_cache.shape
+    kc8 = torch.zeros((NB, H, 16, d), dtype=torch.uint8, device=device)
+    vc8 = torch.zeros_like(kc8)
+    ks = torch.ones((NB, H, 16), dtype=torch.float32, device=device)
+    vs = torch.ones_like(ks)
+    rows_k = st.key_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous()
+    rows_v = st.value_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous()
+    slots = torch.arange(NB * 16, dtype=torch.int32, device=device)
+    with torch.cuda.stream(stream):
+        pa.kv_cache_write_fp8(rows_k, rows_v, slots, kc8, vc8, ks, vs)
+    del rows_k, rows_v
+    torch.cuda.synchronize()
+
+    def fp8():
+        pa.paged_attn_decode_fp8(call.q, kc8, vc8, ks, vs, call.bt, call.cu, call.ctx, call.max_ctx, w.scale,
+                                 out=call.out, workspace=call.ws)
+
+    def bf():
+        st.attend(call)
+
+    steps = max(args.steps, 5)
+    ms = {}
+    for name, fn in (("fp8", fp8), ("16bit", bf)):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                fn()
+        torch.cuda.synchronize()
+        ms[name] = time_steps([fn], steps, stream) / steps
+    b16 = attn_bytes(w)
+    ctx_tokens = sum(int(c) for c in w.ctx_lens)
+    b8 = b16 - ctx_tokens * 2 * H * d * 2 + ctx_tokens * 2 * H * (d + 4)
+    gbs = b8 / (ms["fp8"] * 1e-3) / 1e9
+    return {"workload": "FP8 (E4M3) KV cache, 13B-shaped decode layer: B 64, 40/40 heads, d 128, fp16 Q, "
+                        "ctx U[128,4096]",
+            "decode_GB/s": round(gbs, 1), "frac": round(gbs / hbm_peak, 4), "bytes": b8,
+            "decode_ms": round(ms["fp8"], 5), "decode_16bit_ms": round(ms["16bit"], 5),
+            "speedup_vs_16bit": round(ms["16bit"] / ms["fp8"], 3),
+            "tokens_per_s": round(w.T / (ms["fp8"] * 1e-3), 1)}
 
 
 def leg_tree(args, stream, device, hbm_peak, rank):
@@ -725,6 +782,8 @@ def run_one_leg(args):
         res = leg_swap(args, stream, device, 0)
     elif args.only == "tree":
         res = leg_tree(args, stream, device, hbm, 0)
+    elif args.only == "fp8":
+        res = leg_fp8(args, stream, device, hbm, 0)
     else:
         res = leg_mixed(args, stream, device, hbm, bf16, 0)
     print(json.dumps({"leg": args.only, **res}), flush=True)
@@ -739,7 +798,7 @@ def main(argv=None):
     ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
-    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap", "tree"], default=None,
+    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap", "tree", "fp8"], default=None,
                     help="run one leg alone and print its JSON object (profiling runs)")
     ap.add_argument("--batch", type=int, default=64,
                     help="sequences of the headline decode workload (64 = the 13B-shaped layer; smaller for profiling)")

@@ -182,6 +182,39 @@ int pa_paged_attn_decode_tree(void *out, const void *q, const void *key_cache, c
                               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * FP8 (E4M3) KV cache -- an 8-bit cache with one float scale per stored row
+ * (the FP8 KV-cache option of the serving page; FP8 with scaling on the
+ * interview Q&A page): half the HBM bytes of a 16-bit cache per key.
+ *   key_cache, value_cache  uint8 [num_blocks][H_kv][16][d]: E4M3 codes
+ *                           (OCP FP8: bias 7, 3 mantissa bits, no infinities,
+ *                           largest finite 448)
+ *   key_scale, value_scale  float [num_blocks][H_kv][16]: the row's scale;
+ *                           the stored value is code x scale
+ * A row's scale is fixed when the row is written (amax / 448), so nothing
+ * stored is ever requantised.
+ *
+ * pa_kv_cache_write_fp8 -- pa_kv_cache_write into the FP8 cache: each new row
+ * (16-bit, `dtype`) gets scale = amax / 448 (1 for an all-zero row) and codes
+ * = the E4M3 value nearest to x / scale (ties to even, saturated at +-448),
+ * both divisions IEEE round-to-nearest: bit-exact given the inputs.
+ */
+int pa_kv_cache_write_fp8(const void *k_new, const void *v_new, const int32_t *slot_mapping, int64_t T,
+                          uint8_t *key_cache, uint8_t *value_cache, float *key_scale, float *value_scale,
+                          int64_t num_blocks, int H_kv, int d, pa_dtype dtype, int32_t *status, void *stream);
+
+/*
+ * pa_paged_attn_decode_fp8 -- pa_paged_attn_decode over the FP8 cache: the
+ * same sizes, workspace, scheduling and errors; K and V are dequantised
+ * (code x scale, rounded to `dtype`, the type of q and out) in shared memory
+ * and the attention runs as in the 16-bit call.  NULL scales -> PA_ERR_ARG.
+ */
+int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t *key_cache, const uint8_t *value_cache,
+                             const float *key_scale, const float *value_scale, int64_t num_blocks,
+                             const int32_t *block_tables, int max_blocks_per_seq, const int32_t *cu_seqlens_q,
+                             const int32_t *context_lens, int B, int max_ctx, int64_t T, int H_q, int H_kv, int d,
+                             float scale, pa_dtype dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * pa_paged_attn_decode_noalloc -- pa_paged_attn_decode without a caller workspace.
  * The pages have no counterpart: this is an interface for callers that may not
  * allocate device memory when they call, such as plugins inside an engine that

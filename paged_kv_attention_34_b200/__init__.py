@@ -62,6 +62,11 @@ def _declare(L):
     L.pa_decode_workspace_bytes.argtypes = [I64, I, I, I, I, I]
     L.pa_paged_attn_decode.restype = I
     L.pa_paged_attn_decode.argtypes = [P, P, P, P, I64, P, I, P, P, I, I, I64, I, I, I, c.c_float, I, P, SZ, P]
+    L.pa_kv_cache_write_fp8.restype = I
+    L.pa_kv_cache_write_fp8.argtypes = [P, P, P, I64, P, P, P, P, I64, I, I, I, P, P]
+    L.pa_paged_attn_decode_fp8.restype = I
+    L.pa_paged_attn_decode_fp8.argtypes = [P, P, P, P, P, P, I64, P, I, P, P, I, I, I64, I, I, I, c.c_float, I, P,
+                                           SZ, P]
     L.pa_paged_attn_decode_tree.restype = I
     L.pa_paged_attn_decode_tree.argtypes = [P, P, P, P, I64, P, I, P, P, P, I, I, I64, I, I, I, c.c_float, I, P, SZ,
                                             P]
@@ -264,6 +269,63 @@ def paged_attn_decode(q, key_cache, value_cache, block_tables, cu_seqlens_q, con
     )
     _check(rc, "pa_paged_attn_decode")
     paged_attn_decode.last_workspace = ws
+    return out
+
+
+def _fp8_cache(key_cache, value_cache, key_scale, value_scale):
+    _cuda(key_cache, "key_cache", torch.uint8, 4)
+    _cuda(value_cache, "value_cache", torch.uint8, 4)
+    NB, H_kv, bs, d = key_cache.shape
+    if bs != 16 or tuple(value_cache.shape) != tuple(key_cache.shape):
+        raise ValueError("FP8 caches must be uint8 [NB, H_kv, 16, d], both the same shape")
+    for name, t in (("key_scale", key_scale), ("value_scale", value_scale)):
+        _cuda(t, name, torch.float32, 3)
+        if tuple(t.shape) != (NB, H_kv, 16):
+            raise ValueError(f"{name} must be float32 [{NB}, {H_kv}, 16]")
+    return NB, H_kv, d
+
+
+def kv_cache_write_fp8(k_new, v_new, slot_mapping, key_cache, value_cache, key_scale, value_scale, status=None,
+                       stream=None):
+    """Quantise k_new/v_new [T, H_kv, d] (16-bit) into the FP8 cache (uint8 codes [NB, H_kv, 16, d] and
+    float32 row scales [NB, H_kv, 16]) at slot_mapping [T]."""
+    NB, H_kv, d = _fp8_cache(key_cache, value_cache, key_scale, value_scale)
+    _cuda(k_new, "k_new", None, 3)
+    _cuda(v_new, "v_new", k_new.dtype, 3)
+    _cuda(slot_mapping, "slot_mapping", torch.int32, 1)
+    if status is not None:
+        _cuda(status, "status", torch.int32)
+    rc = lib().pa_kv_cache_write_fp8(
+        _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), slot_mapping.shape[0], _ptr(key_cache), _ptr(value_cache),
+        _ptr(key_scale), _ptr(value_scale), NB, H_kv, d, _dtype_code(k_new), _ptr(status),
+        ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_kv_cache_write_fp8")
+
+
+def paged_attn_decode_fp8(q, key_cache, value_cache, key_scale, value_scale, block_tables, cu_seqlens_q,
+                          context_lens, max_ctx: int, scale: float, out=None, workspace=None, stream=None):
+    """Split-KV decode over the FP8 cache; returns out [T, H_q, d] in q's dtype."""
+    NB, H_kv, d = _fp8_cache(key_cache, value_cache, key_scale, value_scale)
+    _cuda(q, "q", None, 3)
+    T, H_q, dq = q.shape
+    if dq != d:
+        raise ValueError("q and the caches disagree on d")
+    _cuda(block_tables, "block_tables", torch.int32, 2)
+    _cuda(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _cuda(context_lens, "context_lens", torch.int32, 1)
+    B = context_lens.shape[0]
+    if out is None:
+        out = torch.empty_like(q)
+    nbytes = decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx)
+    ws = _workspace(workspace, nbytes, q.device)
+    rc = lib().pa_paged_attn_decode_fp8(
+        _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(key_scale), _ptr(value_scale), NB,
+        _ptr(block_tables), block_tables.shape[1], _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_ctx), T, H_q,
+        H_kv, d, float(scale), _dtype_code(q), _ptr(ws), ws.numel(), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_paged_attn_decode_fp8")
+    paged_attn_decode_fp8.last_workspace = ws
     return out
 
 

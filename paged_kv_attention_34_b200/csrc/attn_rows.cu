@@ -25,6 +25,8 @@
 // m16n8k16 with fp32 accumulators; P is rounded to the input type for P V.
 #include <cmath>
 
+#include <cuda_fp8.h>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -45,6 +47,8 @@ struct RowsParams {
     float *ws_lse;  // [max_splits][T][H_q] log2-sum-exp of the scaled scores
     const int32_t *order;  // [B] sequences by decreasing page count: grid z -> sequence
     const int32_t *tree;   // [T] tree verification: bit j = the token sees new token j; nullptr = causal
+    const float *k_scale;  // FP8 cache: [num_blocks][H_kv][16] scale of every stored K row
+    const float *v_scale;  // ... and V row
     int32_t *status;
     int64_t num_blocks;
     int64_t T;
@@ -57,14 +61,19 @@ struct RowsParams {
     float scale_log2;  // scale * log2(e)
 };
 
+// Epilogue buffer of a rows CTA: partial O, max and sum of every warp's 16 rows.
+template <int D>
+struct RowsEpi {
+    static constexpr int kStride = D + 8;  // floats per row of the epilogue buffer
+    static constexpr int kBytes = (4 * 16 * kStride + 2 * 64) * 4;
+};
+
 template <int D, int STAGES>
 struct RowsSmem {
     static constexpr int kPageBytes = 16 * D * 2;
     static constexpr int kStageBytes = 2 * kPagesPerStage * kPageBytes;  // K pages then V pages
     static constexpr int kQBytes = kRowsPerCta * D * 2;
-    static constexpr int kEpiStride = D + 8;  // floats per row of the epilogue buffer
-    static constexpr int kEpiBytes = (4 * 16 * kEpiStride + 2 * 64) * 4;
-    static_assert(kEpiBytes <= STAGES * kStageBytes, "epilogue must fit in the stage ring");
+    static_assert(RowsEpi<D>::kBytes <= STAGES * kStageBytes, "epilogue must fit in the stage ring");
     static_assert(kQBytes <= kStageBytes, "Q is staged through one stage buffer");
     static constexpr int kStageOff = 0;
     static constexpr int kQOff = (STAGES - 1) * kStageBytes;  // aliases the last stage during set-up
@@ -96,7 +105,206 @@ __device__ __forceinline__ bool seq_ok(int qb, int ctx, const RowsParams &p, int
     return qb >= 1 && ctx >= qb && qb <= p.max_q_len && ctx <= p.max_ctx && ctx <= p.max_blocks * 16 && q1 <= p.T;
 }
 
-template <int D, bool BF16, int STAGES>
+// One 16-key page for one warp: S = Q K^T for its m-tile (mma.sync m16n8k16 from ldmatrix of the
+// swizzled K page), mask, online softmax of its two rows, O += P V.  `kbase` and `vbase` are shared
+// addresses of the page's K and V in the 128-byte-swizzled 16-bit layout; keys j0 .. j0 + 15.
+// Key k is visible to a row when k <= lim and, among the new tokens (k >= base), its bit is set.
+// SCALED (the FP8 cache): K and V hold the codes' values unscaled and ksc / vsc the 16 row scales
+// of the page in shared memory; a key's K scale multiplies its score, its V scale its P (the row
+// sum l takes the unscaled P), which is K x scale and V x scale exactly up to rounding.
+template <int D, bool BF16, bool SCALED = false, bool TREE = false>
+__device__ __forceinline__ void rows_page(uint32_t kbase, uint32_t vbase, int j0, int lane,
+                                          const uint32_t (&qa)[D / 16][4], float (&o)[D / 8][4], float &m_a,
+                                          float &m_b, float &l_a, float &l_b, int lim_a, int lim_b, uint32_t bits_a,
+                                          uint32_t bits_b, int base, int ctx, float sl2, const float *ksc = nullptr,
+                                          const float *vsc = nullptr)
+{
+    constexpr int KSTEPS = D / 16;  // k-steps of S = Q K^T
+    constexpr int NT = D / 8;       // n-tiles of O
+    const int kq = lane & 3;
+    auto visible = [&](int key, int lim, uint32_t bits) {
+        if constexpr (TREE)
+            return key <= lim && (key < base || ((bits >> (key - base)) & 1u));
+        else
+            return key <= lim;
+    };
+
+    // S (16 rows x 16 keys) = Q K^T
+    float s[2][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = (mi >> 1) * 8 + rr;
+        const int c = 2 * ks + (mi & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kbase + (c >> 3) * 2048 + key * 128 + (((c & 7) ^ (key & 7)) << 4), b0, b1, b2, b3);
+        mma16816<BF16>(s[0], qa[ks], b0, b1);
+        mma16816<BF16>(s[1], qa[ks], b2, b3);
+    }
+    // mask (causal / context end), scale to log2 units, online softmax
+    float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const int key = j0 + nt * 8 + 2 * kq + c;
+            float f = sl2;
+            if constexpr (SCALED)
+                f *= ksc[nt * 8 + 2 * kq + c];
+            s[nt][c] = visible(key, lim_a, bits_a) ? s[nt][c] * f : -INFINITY;
+            s[nt][2 + c] = visible(key, lim_b, bits_b) ? s[nt][2 + c] * f : -INFINITY;
+            mx_a = fmaxf(mx_a, s[nt][c]);
+            mx_b = fmaxf(mx_b, s[nt][2 + c]);
+        }
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+    const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
+    const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
+    const float al_a = fast_exp2(m_a - base_a), al_b = fast_exp2(m_b - base_b);
+    m_a = mn_a;
+    m_b = mn_b;
+    float ps_a = 0.f, ps_b = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        s[nt][0] = fast_exp2(s[nt][0] - base_a);
+        s[nt][1] = fast_exp2(s[nt][1] - base_a);
+        s[nt][2] = fast_exp2(s[nt][2] - base_b);
+        s[nt][3] = fast_exp2(s[nt][3] - base_b);
+        ps_a += s[nt][0] + s[nt][1];
+        ps_b += s[nt][2] + s[nt][3];
+    }
+    l_a = l_a * al_a + ps_a;
+    l_b = l_b * al_b + ps_b;
+    if (__any_sync(0xffffffffu, al_a != 1.f || al_b != 1.f)) {
+#pragma unroll
+        for (int nd = 0; nd < NT; ++nd) {
+            o[nd][0] *= al_a;
+            o[nd][1] *= al_a;
+            o[nd][2] *= al_b;
+            o[nd][3] *= al_b;
+        }
+    }
+    if constexpr (SCALED) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const float vs = vsc[nt * 8 + 2 * kq + c];
+                s[nt][c] *= vs;
+                s[nt][2 + c] *= vs;
+            }
+    }
+    uint32_t pa_[4];
+    pa_[0] = pack2<BF16>(s[0][0], s[0][1]);
+    pa_[1] = pack2<BF16>(s[0][2], s[0][3]);
+    pa_[2] = pack2<BF16>(s[1][0], s[1][1]);
+    pa_[3] = pack2<BF16>(s[1][2], s[1][3]);
+
+    // keys past the context end may hold anything (NaN): zero their V
+    uint32_t vm_lo = 0xffffffffu, vm_hi = 0xffffffffu;
+    if (j0 + 16 > ctx) {
+        const int valid = ctx - j0;
+        const int k0 = 2 * kq;
+        vm_lo = (k0 < valid ? 0x0000ffffu : 0u) | (k0 + 1 < valid ? 0xffff0000u : 0u);
+        vm_hi = (k0 + 8 < valid ? 0x0000ffffu : 0u) | (k0 + 9 < valid ? 0xffff0000u : 0u);
+    }
+    // O (16 x D) += P (16 x 16 keys) V (16 keys x D)
+#pragma unroll
+    for (int ndp = 0; ndp < NT / 2; ++ndp) {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = (mi & 1) * 8 + rr;
+        const int c = 2 * ndp + (mi >> 1);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_t(vbase + (c >> 3) * 2048 + key * 128 + (((c & 7) ^ (key & 7)) << 4), r0, r1, r2, r3);
+        r0 &= vm_lo;
+        r1 &= vm_hi;
+        r2 &= vm_lo;
+        r3 &= vm_hi;
+        mma16816<BF16>(o[2 * ndp], pa_, r0, r1);
+        mma16816<BF16>(o[2 * ndp + 1], pa_, r2, r3);
+    }
+}
+
+// Epilogue of a rows CTA: merge the warps of each m-tile (several warps on different pages of the
+// same rows, like splits) through shared memory `e_o` (at least RowsEpi<D>::kBytes), normalise,
+// and store the rows: straight to `out` when the sequence has one split, else the normalised
+// partial and its log2-sum-exp to the workspace.
+template <int D, bool BF16>
+__device__ __forceinline__ void rows_epilogue(float *e_o, const RowsParams &p, const float (&o)[D / 8][4], float m_a,
+                                              float m_b, float l_a, float l_b, bool has_rows, int rows_here,
+                                              int row0, int q0, int g, int split, int n_splits, int KG)
+{
+    constexpr int NT = D / 8;
+    constexpr int kEpiStride = RowsEpi<D>::kStride;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, kq = lane & 3;
+    const int G = p.G;
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    float *e_m = e_o + 4 * 16 * kEpiStride;        // [4][16]
+    float *e_l = e_m + 64;                            // [4][16]
+    if (has_rows) {
+        const int la = lane >> 2, lb = la + 8;
+#pragma unroll
+        for (int nd = 0; nd < NT; ++nd) {
+            const int col = nd * 8 + 2 * kq;
+            *reinterpret_cast<float2 *>(e_o + (warp * 16 + la) * kEpiStride + col) = make_float2(o[nd][0], o[nd][1]);
+            *reinterpret_cast<float2 *>(e_o + (warp * 16 + lb) * kEpiStride + col) = make_float2(o[nd][2], o[nd][3]);
+        }
+        if (kq == 0) {
+            e_m[warp * 16 + la] = m_a;
+            e_m[warp * 16 + lb] = m_b;
+            e_l[warp * 16 + la] = l_a;
+            e_l[warp * 16 + lb] = l_b;
+        }
+    }
+    __syncthreads();
+    const bool final_out = n_splits == 1;
+    for (int i = tid; i < rows_here * (D / 4); i += kThreads) {
+        const int r = i / (D / 4), c4 = i % (D / 4);
+        const int mtr = r >> 4, lr = r & 15;
+        float M = -INFINITY;
+        for (int k = 0; k < KG; ++k)
+            M = fmaxf(M, e_m[(mtr * KG + k) * 16 + lr]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float Lsum = 0.f;
+        for (int k = 0; k < KG; ++k) {
+            const int w = mtr * KG + k;
+            const float mk = e_m[w * 16 + lr];
+            const float wt = mk == -INFINITY ? 0.f : fast_exp2(mk - M);
+            Lsum += wt * e_l[w * 16 + lr];
+            const float4 v = *reinterpret_cast<const float4 *>(e_o + (w * 16 + lr) * kEpiStride + c4 * 4);
+            acc.x += wt * v.x;
+            acc.y += wt * v.y;
+            acc.z += wt * v.z;
+            acc.w += wt * v.w;
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        const int ridx = row0 + r;
+        const int64_t t = q0 + ridx / G;
+        const int h = g * G + ridx % G;
+        const int64_t orow = t * p.H_q + h;
+        if (final_out) {
+            store4<BF16>(static_cast<uint8_t *>(p.out) + (orow * D + c4 * 4) * 2, acc.x * inv, acc.y * inv,
+                         acc.z * inv, acc.w * inv);
+        } else {
+            const int64_t prow = (int64_t)split * p.T * p.H_q + orow;
+            *reinterpret_cast<float4 *>(p.ws_o + prow * D + c4 * 4) =
+                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            if (c4 == 0)
+                p.ws_lse[prow] = Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
+        }
+    }
+}
+
+template <int D, bool BF16, int STAGES, bool TREE>
 __global__ void __launch_bounds__(kThreads, 1)
     pa_attn_rows_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const RowsParams p)
@@ -136,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (row0 >= R)
         return;
     const int rows_here = min(kRowsPerCta, R - row0);
-    const bool tree = p.tree != nullptr;
+    constexpr bool tree = TREE;  // p.tree is set exactly when TREE is
     const int base = ctx - qb;  // first new token of the sequence
     // last key any row here sees (a tree row may see every new token)
     const int lim_cta = tree ? ctx - 1 : ctx - qb + (row0 + rows_here - 1) / G;
@@ -251,9 +459,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bits_b = tree && rb < rows_here ? static_cast<uint32_t>(__ldg(p.tree + q0 + (row0 + rb) / G)) : ~0u;
     const int lim_warp =
         has_rows ? (tree ? ctx - 1 : ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G) : -1;
-    auto visible = [&](int key, int lim, uint32_t bits) {
-        return key <= lim && (key < base || ((bits >> (key - base)) & 1u));
-    };
 
     uint32_t qa[KSTEPS][4];
     if (has_rows) {
@@ -274,7 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     const float sl2 = p.scale_log2;
-    const int kq = lane & 3;
 
     // ---- main loop over stages ---------------------------------------------------------------
     int it = 0;
@@ -297,94 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;  // every row of this warp is causally masked on this page
                 const uint32_t kbase = smem_u32(kst + k * L::kPageBytes);
                 const uint32_t vbase = smem_u32(vst + k * L::kPageBytes);
-
-                // S (16 rows x 16 keys) = Q K^T
-                float s[2][4];
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-                    s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-                for (int ks = 0; ks < KSTEPS; ++ks) {
-                    const int mi = lane >> 3, rr = lane & 7;
-                    const int key = (mi >> 1) * 8 + rr;
-                    const int c = 2 * ks + (mi & 1);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kbase + (c >> 3) * 2048 + key * 128 + (((c & 7) ^ (key & 7)) << 4), b0, b1, b2, b3);
-                    mma16816<BF16>(s[0], qa[ks], b0, b1);
-                    mma16816<BF16>(s[1], qa[ks], b2, b3);
-                }
-                // mask (causal / context end), scale to log2 units, online softmax
-                float mx_a = -INFINITY, mx_b = -INFINITY;
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const int key = j0 + nt * 8 + 2 * kq + c;
-                        s[nt][c] = visible(key, lim_a, bits_a) ? s[nt][c] * sl2 : -INFINITY;
-                        s[nt][2 + c] = visible(key, lim_b, bits_b) ? s[nt][2 + c] * sl2 : -INFINITY;
-                        mx_a = fmaxf(mx_a, s[nt][c]);
-                        mx_b = fmaxf(mx_b, s[nt][2 + c]);
-                    }
-                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-                mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-                mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-                const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-                const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
-                const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
-                const float al_a = fast_exp2(m_a - base_a), al_b = fast_exp2(m_b - base_b);
-                m_a = mn_a;
-                m_b = mn_b;
-                float ps_a = 0.f, ps_b = 0.f;
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    s[nt][0] = fast_exp2(s[nt][0] - base_a);
-                    s[nt][1] = fast_exp2(s[nt][1] - base_a);
-                    s[nt][2] = fast_exp2(s[nt][2] - base_b);
-                    s[nt][3] = fast_exp2(s[nt][3] - base_b);
-                    ps_a += s[nt][0] + s[nt][1];
-                    ps_b += s[nt][2] + s[nt][3];
-                }
-                l_a = l_a * al_a + ps_a;
-                l_b = l_b * al_b + ps_b;
-                if (__any_sync(0xffffffffu, al_a != 1.f || al_b != 1.f)) {
-#pragma unroll
-                    for (int nd = 0; nd < NT; ++nd) {
-                        o[nd][0] *= al_a;
-                        o[nd][1] *= al_a;
-                        o[nd][2] *= al_b;
-                        o[nd][3] *= al_b;
-                    }
-                }
-                uint32_t pa_[4];
-                pa_[0] = pack2<BF16>(s[0][0], s[0][1]);
-                pa_[1] = pack2<BF16>(s[0][2], s[0][3]);
-                pa_[2] = pack2<BF16>(s[1][0], s[1][1]);
-                pa_[3] = pack2<BF16>(s[1][2], s[1][3]);
-
-                // keys past the context end may hold anything (NaN): zero their V
-                uint32_t vm_lo = 0xffffffffu, vm_hi = 0xffffffffu;
-                if (j0 + 16 > ctx) {
-                    const int valid = ctx - j0;
-                    const int k0 = 2 * kq;
-                    vm_lo = (k0 < valid ? 0x0000ffffu : 0u) | (k0 + 1 < valid ? 0xffff0000u : 0u);
-                    vm_hi = (k0 + 8 < valid ? 0x0000ffffu : 0u) | (k0 + 9 < valid ? 0xffff0000u : 0u);
-                }
-                // O (16 x D) += P (16 x 16 keys) V (16 keys x D)
-#pragma unroll
-                for (int ndp = 0; ndp < NT / 2; ++ndp) {
-                    const int mi = lane >> 3, rr = lane & 7;
-                    const int key = (mi & 1) * 8 + rr;
-                    const int c = 2 * ndp + (mi >> 1);
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4_t(vbase + (c >> 3) * 2048 + key * 128 + (((c & 7) ^ (key & 7)) << 4), r0, r1, r2, r3);
-                    r0 &= vm_lo;
-                    r1 &= vm_hi;
-                    r2 &= vm_lo;
-                    r3 &= vm_hi;
-                    mma16816<BF16>(o[2 * ndp], pa_, r0, r1);
-                    mma16816<BF16>(o[2 * ndp + 1], pa_, r2, r3);
-                }
+                rows_page<D, BF16, false, TREE>(kbase, vbase, j0, lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, bits_a, bits_b,
+                                   base, ctx, sl2);
             }
         }
         // the last warp done with this slot refills it
@@ -407,66 +525,285 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
 
-    // ---- epilogue: merge the warps of each m-tile, normalise, store --------------------------
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-    float *e_o = reinterpret_cast<float *>(s_stage);  // [4 warps][16 rows][kEpiStride]
-    float *e_m = e_o + 4 * 16 * L::kEpiStride;        // [4][16]
-    float *e_l = e_m + 64;                            // [4][16]
-    if (has_rows) {
-        const int la = lane >> 2, lb = la + 8;
-#pragma unroll
-        for (int nd = 0; nd < NT; ++nd) {
-            const int col = nd * 8 + 2 * kq;
-            *reinterpret_cast<float2 *>(e_o + (warp * 16 + la) * L::kEpiStride + col) = make_float2(o[nd][0], o[nd][1]);
-            *reinterpret_cast<float2 *>(e_o + (warp * 16 + lb) * L::kEpiStride + col) = make_float2(o[nd][2], o[nd][3]);
+    // ---- epilogue ---------------------------------------------------------------------------
+    rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_stage), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0, g,
+                           split, n_splits, KG);
+}
+
+// ---- FP8 (E4M3) cache -----------------------------------------------------------------------
+// The same split-KV decode over an 8-bit cache with one float scale per stored row.  TMA brings
+// each page's codes (16 rows x d bytes, one box for K and one for V) into a three-stage ring; per
+// stage the whole CTA converts the four pages' codes into their 16-bit values in one stage laid
+// out like the 16-bit cache's (128-byte swizzle) and stages the row scales, and the warps run
+// rows_page on it with the scales folded into the scores and into P.  Half the HBM bytes of the
+// 16-bit cache per key.
+constexpr int kFp8Stages = 3;
+
+template <int D>
+struct Fp8Smem {
+    static constexpr int kPage8 = 16 * D;                            // codes of one page
+    static constexpr int kStage8 = 2 * kPagesPerStage * kPage8;      // K pages then V pages
+    static constexpr int kPage16 = 16 * D * 2;
+    static constexpr int kStage16 = 2 * kPagesPerStage * kPage16;    // one dequantised stage
+    static constexpr int kQBytes = kRowsPerCta * D * 2;
+    static constexpr int kWork = ((kStage16 > RowsEpi<D>::kBytes ? kStage16 : RowsEpi<D>::kBytes) + 1023) / 1024 * 1024;
+    static_assert(kQBytes <= kWork, "Q is staged through the dequantised stage");
+    static constexpr int kWorkOff = 0;                               // dequantised stage / Q / epilogue
+    static constexpr int kRingOff = kWork;
+    static constexpr int kBarOff = kRingOff + kFp8Stages * kStage8;
+    static constexpr int kIssuedOff = kBarOff + 8 * kFp8Stages;
+    static constexpr int kCountOff = kIssuedOff + 4 * kFp8Stages;               // warps done with each stage
+    static constexpr int kFlagOff = kCountOff + 4 * kFp8Stages;                 // abort flag
+    static constexpr int kScaleOff = kFlagOff + 16;                             // [K, V][4 pages][16 rows]
+    static constexpr int kTableOff = kScaleOff + 4 * 2 * kPagesPerStage * 16;
+    static constexpr int kBytes = kTableOff + 4 * kMaxTablePages;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    pa_attn_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                            const RowsParams p)
+{
+    using L = Fp8Smem<D>;
+    constexpr int CH = D / 8;       // 16-byte chunks of a 16-bit row
+    constexpr int KSTEPS = D / 16;  // k-steps of S = Q K^T
+    constexpr int NT = D / 8;       // n-tiles of O
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *s_work = smem + L::kWorkOff;
+    uint8_t *s_ring = smem + L::kRingOff;
+    uint64_t *s_bar = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    int *s_issued = reinterpret_cast<int *>(smem + L::kIssuedOff);
+    int32_t *s_pages = reinterpret_cast<int32_t *>(smem + L::kTableOff);
+    float *s_scale = reinterpret_cast<float *>(smem + L::kScaleOff);
+    int *s_count = reinterpret_cast<int *>(smem + L::kCountOff);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- which (sequence, KV head, row group, split): as the 16-bit kernel ----------------
+    const int b = __ldg(p.order + blockIdx.z);
+    const int split = blockIdx.x;
+    const int g = blockIdx.y / p.n_rg, rg = blockIdx.y % p.n_rg;
+    const int q0 = __ldg(p.cu_seqlens + b), q1 = __ldg(p.cu_seqlens + b + 1);
+    const int qb = q1 - q0, ctx = __ldg(p.context_lens + b);
+    if (!seq_ok(qb, ctx, p, q1)) {
+        if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+            set_status(p.status, PA_ERR_SEQ);
+        return;
+    }
+    const int G = p.G;
+    const int R = G * qb;
+    const int row0 = rg * kRowsPerCta;
+    if (row0 >= R)
+        return;
+    const int rows_here = min(kRowsPerCta, R - row0);
+    const int base = ctx - qb;
+    const int lim_cta = ctx - qb + (row0 + rows_here - 1) / G;
+    const int pages_need = lim_cta / 16 + 1;
+    const int pages_ctx = (ctx + 15) / 16;
+    const int n_splits = (pages_ctx + p.split_pages - 1) / p.split_pages;
+    if (split >= n_splits)
+        return;
+    const int page_lo = split * p.split_pages;
+    const int page_hi = min(page_lo + p.split_pages, pages_need);
+    const int n_pages = max(0, page_hi - page_lo);
+    const int n_stages = (n_pages + kPagesPerStage - 1) / kPagesPerStage;
+    const int MT = rows_here <= 16 ? 1 : (rows_here <= 32 ? 2 : 4);
+    const int KG = 4 / MT;
+    const int mt = warp / KG, kg = warp % KG;
+    const bool has_rows = mt * 16 < rows_here;
+
+    // ---- set-up ----------------------------------------------------------------------------
+    const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
+    auto issue = [&](int st) {  // one thread
+        const int slot = st % kFp8Stages;
+        uint8_t *kb = s_ring + slot * L::kStage8;
+        uint8_t *vb = kb + kPagesPerStage * L::kPage8;
+        const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&s_bar[slot], np * 2 * L::kPage8);
+        s_issued[slot] += 1;
+        for (int k = 0; k < np; ++k) {
+            const int y = (s_pages[st * kPagesPerStage + k] * p.H_kv + g) * 16;
+            tma_load_2d(kb + k * L::kPage8, &tmap_k, 0, y, &s_bar[slot]);
+            tma_load_2d(vb + k * L::kPage8, &tmap_v, 0, y, &s_bar[slot]);
         }
-        if (kq == 0) {
-            e_m[warp * 16 + la] = m_a;
-            e_m[warp * 16 + lb] = m_b;
-            e_l[warp * 16 + la] = l_a;
-            e_l[warp * 16 + lb] = l_b;
+    };
+    if (tid == 0) {
+        for (int s = 0; s < kFp8Stages; ++s) {
+            mbar_init(&s_bar[s], 1);
+            s_issued[s] = 0;
+            s_count[s] = 0;
         }
+        *s_abort = 0;
+        fence_barrier_init();
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+    }
+    for (int i = tid; i < n_pages; i += kThreads) {
+        int pg = __ldg(table + page_lo + i);
+        if (pg < 0 || pg >= p.num_blocks) {
+            set_status(p.status, PA_ERR_BOUNDS);
+            pg = static_cast<int>(p.num_blocks);  // past the pool: TMA fills zeros, scale 0
+        }
+        s_pages[i] = pg;
+    }
+    for (int i = tid; i < kRowsPerCta * CH; i += kThreads) {
+        const int r = i / CH, c = i % CH;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < rows_here) {
+            const int ridx = row0 + r;
+            const int64_t t = q0 + ridx / G;
+            const int h = g * G + ridx % G;
+            v = __ldg(reinterpret_cast<const uint4 *>(p.q) + (t * p.H_q + h) * CH + c);
+        }
+        *reinterpret_cast<uint4 *>(s_work + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
     }
     __syncthreads();
-    const bool final_out = n_splits == 1;
-    for (int i = tid; i < rows_here * (D / 4); i += kThreads) {
-        const int r = i / (D / 4), c4 = i % (D / 4);
-        const int mtr = r >> 4, lr = r & 15;
-        float M = -INFINITY;
-        for (int k = 0; k < KG; ++k)
-            M = fmaxf(M, e_m[(mtr * KG + k) * 16 + lr]);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        float Lsum = 0.f;
-        for (int k = 0; k < KG; ++k) {
-            const int w = mtr * KG + k;
-            const float mk = e_m[w * 16 + lr];
-            const float wt = mk == -INFINITY ? 0.f : fast_exp2(mk - M);
-            Lsum += wt * e_l[w * 16 + lr];
-            const float4 v = *reinterpret_cast<const float4 *>(e_o + (w * 16 + lr) * L::kEpiStride + c4 * 4);
-            acc.x += wt * v.x;
-            acc.y += wt * v.y;
-            acc.z += wt * v.z;
-            acc.w += wt * v.w;
-        }
-        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-        const int ridx = row0 + r;
-        const int64_t t = q0 + ridx / G;
-        const int h = g * G + ridx % G;
-        const int64_t orow = t * p.H_q + h;
-        if (final_out) {
-            store4<BF16>(static_cast<uint8_t *>(p.out) + (orow * D + c4 * 4) * 2, acc.x * inv, acc.y * inv,
-                         acc.z * inv, acc.w * inv);
-        } else {
-            const int64_t prow = (int64_t)split * p.T * p.H_q + orow;
-            *reinterpret_cast<float4 *>(p.ws_o + prow * D + c4 * 4) =
-                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-            if (c4 == 0)
-                p.ws_lse[prow] = Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
+    if (tid == 0)
+        for (int st = 0; st < min(kFp8Stages, n_stages); ++st)
+            issue(st);
+    const int ra = mt * 16 + (lane >> 2), rb = ra + 8;
+    const int lim_a = ra < rows_here ? ctx - qb + (row0 + ra) / G : -1;
+    const int lim_b = rb < rows_here ? ctx - qb + (row0 + rb) / G : -1;
+    const int lim_warp = has_rows ? ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G : -1;
+    uint32_t qa[KSTEPS][4];
+    if (has_rows) {
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+            const int mi = lane >> 3, rr = lane & 7;
+            const int r = mt * 16 + (mi & 1) * 8 + rr;
+            const int c = 2 * ks + (mi >> 1);
+            ldsm_x4(smem_u32(s_work + r * (D * 2) + ((c ^ (r & 7)) << 4)), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
         }
     }
+    __syncthreads();  // Q is in registers: the work buffer takes the dequantised stages
+    float o[NT][4];
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+        o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    const float sl2 = p.scale_log2;
+
+    // Convert row `row` of page `k` of stage `it` (kv 0 = K, 1 = V): the codes become their values in
+    // the 16-bit type (exact: every E4M3 value is an f16 and a bf16 value), in 8-byte pieces from a
+    // per-thread offset (spreading the banks), into the work buffer laid out like the 16-bit cache's;
+    // the row's scale goes to shared memory (0 past the context end, whose rows may hold anything).
+    auto convert_row = [&](int it, int kv, int k, int row) {
+        const int pidx = it * kPagesPerStage + k;
+        const int pg = s_pages[pidx];
+        const float *scales = kv ? p.v_scale : p.k_scale;
+        const bool live = pg < p.num_blocks && (page_lo + pidx) * 16 + row < ctx;
+        s_scale[(kv * kPagesPerStage + k) * 16 + row] =
+            live ? __ldg(scales + ((int64_t)pg * p.H_kv + g) * 16 + row) : 0.f;
+        const uint8_t *src = s_ring + (it % kFp8Stages) * L::kStage8 + kv * kPagesPerStage * L::kPage8 +
+                             k * L::kPage8 + row * D;
+        uint8_t *dst = s_work + kv * kPagesPerStage * L::kPage16 + k * L::kPage16;
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int ch = (i + row) % CH;
+            const uint2 codes = *reinterpret_cast<const uint2 *>(src + ch * 8);
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t word = q < 2 ? codes.x : codes.y;
+                const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((word >> (16 * (q & 1))) & 0xffffu);
+                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+                if constexpr (BF16) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+                    w[q] = pack2<true>(f.x, f.y);
+                } else {
+                    w[q] = static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+                }
+            }
+            *reinterpret_cast<uint4 *>(dst + (ch >> 3) * 2048 + row * 128 + (((ch & 7) ^ (row & 7)) << 4)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    };
+
+    bool aborted = false;
+    if (MT == 1) {
+        // ---- one m-tile: warp w owns page w of every stage (converts it, then computes it), no CTA
+        // barrier; the last warp done with a stage refills it (as the 16-bit kernel) ------------
+        static_assert(kPagesPerStage == 4, "one page per warp");
+        for (int it = 0; it < n_stages; ++it) {
+            const int slot = it % kFp8Stages;
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_bar[slot], (it / kFp8Stages) & 1));
+            if (!ok) {
+                *s_abort = 1;
+                set_status(p.status, PA_ERR_TIMEOUT);
+            }
+            const int k = warp, pidx = it * kPagesPerStage + k;
+            if (ok && pidx < n_pages) {
+                convert_row(it, lane >> 4, k, lane & 15);
+                __syncwarp();
+                const int j0 = (page_lo + pidx) * 16;
+                if (has_rows && j0 <= lim_warp)
+                    rows_page<D, BF16, true>(smem_u32(s_work + k * L::kPage16),
+                                             smem_u32(s_work + kPagesPerStage * L::kPage16 + k * L::kPage16), j0,
+                                             lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, ~0u, ~0u, base, ctx, sl2,
+                                             s_scale + k * 16, s_scale + (kPagesPerStage + k) * 16);
+            }
+            __syncwarp();
+            if (lane == 0 && atomicAdd(&s_count[slot], 1) == 3) {
+                s_count[slot] = 0;
+                if (it + kFp8Stages < n_stages && !*s_abort)
+                    issue(it + kFp8Stages);
+            }
+            if (*s_abort)
+                break;
+        }
+        __syncthreads();
+        aborted = *s_abort != 0;
+    } else {
+    // ---- several m-tiles: the CTA converts each stage together, then computes it -----------
+    for (int it = 0; it < n_stages; ++it) {
+        const int slot = it % kFp8Stages;
+        // every thread waits; the CTA agrees on the outcome, so no one is left at a barrier
+        const bool landed = __syncthreads_and(mbar_wait(&s_bar[slot], (it / kFp8Stages) & 1));
+        if (!landed) {
+            if (tid == 0)
+                set_status(p.status, PA_ERR_TIMEOUT);
+            aborted = true;
+            break;
+        }
+        // one row per thread: 2 (K, V) x 4 pages x 16 rows = 128 rows per stage
+        static_assert(2 * kPagesPerStage * 16 == kThreads, "one row per thread");
+        if (it * kPagesPerStage + (tid / 16) % kPagesPerStage < n_pages)
+            convert_row(it, tid / (kPagesPerStage * 16), (tid / 16) % kPagesPerStage, tid % 16);
+        __syncthreads();  // the stage is dequantised; its codes can be replaced
+        if (tid == 0 && it + kFp8Stages < n_stages)
+            issue(it + kFp8Stages);
+        if (has_rows) {
+            for (int k = kg; k < kPagesPerStage; k += KG) {
+                const int pidx = it * kPagesPerStage + k;
+                if (pidx >= n_pages)
+                    break;
+                const int j0 = (page_lo + pidx) * 16;
+                if (j0 > lim_warp)
+                    continue;
+                const uint32_t kbase = smem_u32(s_work + k * L::kPage16);
+                const uint32_t vbase = smem_u32(s_work + kPagesPerStage * L::kPage16 + k * L::kPage16);
+                rows_page<D, BF16, true>(kbase, vbase, j0, lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, ~0u, ~0u,
+                                         base, ctx, sl2, s_scale + k * 16, s_scale + (kPagesPerStage + k) * 16);
+            }
+        }
+        __syncthreads();  // everyone is done with the work buffer before the next stage overwrites it
+    }
+    }
+    if (aborted) {
+        // let the copies still in flight land (bounded) before the CTA releases its shared memory
+        if (tid == 0)
+            for (int s = 0; s < kFp8Stages; ++s)
+                if (s_issued[s] > 0)
+                    mbar_wait(&s_bar[s], (s_issued[s] - 1) & 1, kWaitTimeoutNs / 10);
+        return;
+    }
+    rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_work), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0,
+                           g, split, n_splits, KG);
 }
 
 // One warp per (token, query head) row of a sequence with more than one split:
@@ -526,12 +863,33 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
 
 constexpr int kStages = 3;
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool TREE>
 static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
                        cudaStream_t stream)
 {
     using L = RowsSmem<D, kStages>;
-    auto kern = pa_attn_rows_kernel<D, BF16, kStages>;
+    auto kern = pa_attn_rows_kernel<D, BF16, kStages, TREE>;
+    static uint64_t configured = 0;  // one bit per device, per template instance
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return PA_ERR_CUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (!bit || !(configured & bit)) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured |= bit;
+    }
+    kern<<<grid, kThreads, L::kAlloc, stream>>>(tk, tv, rp);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int D, bool BF16>
+static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
+                           cudaStream_t stream)
+{
+    using L = Fp8Smem<D>;
+    auto kern = pa_attn_rows_fp8_kernel<D, BF16>;
     static uint64_t configured = 0;  // one bit per device, per template instance
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
@@ -643,10 +1001,13 @@ size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
 template <int D, bool BF16>
 static int run(const AttnArgs &a)
 {
+    const bool fp8 = a.key_scale != nullptr;
     CUtensorMap tk, tv;
-    int rc = make_cache_tmap(&tk, a.key_cache, a.num_blocks, a.H_kv, D, a.dtype);
+    int rc = fp8 ? make_cache_tmap_fp8(&tk, a.key_cache, a.num_blocks, a.H_kv, D)
+                 : make_cache_tmap(&tk, a.key_cache, a.num_blocks, a.H_kv, D, a.dtype);
     if (rc == PA_OK)
-        rc = make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
+        rc = fp8 ? make_cache_tmap_fp8(&tv, a.value_cache, a.num_blocks, a.H_kv, D)
+                 : make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
     if (rc != PA_OK)
         return rc;
     RowsParams rp{};
@@ -667,6 +1028,8 @@ static int run(const AttnArgs &a)
     rp.max_q_len = a.max_q_len;
     rp.scale_log2 = a.scale * 1.4426950408889634f;
     rp.tree = a.tree_mask;
+    rp.k_scale = a.key_scale;
+    rp.v_scale = a.value_scale;
     {
         const DecodePlan pl = decode_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx);
         rp.n_rg = pl.row_groups;
@@ -684,7 +1047,9 @@ static int run(const AttnArgs &a)
         dim3 grid(pl.max_splits, a.H_kv * pl.row_groups, a.B);
         rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
         if (rc == PA_OK)
-            rc = launch_rows<D, BF16>(rp, tk, tv, grid, a.stream);
+            rc = fp8       ? launch_rows_fp8<D, BF16>(rp, tk, tv, grid, a.stream)
+                 : rp.tree ? launch_rows<D, BF16, true>(rp, tk, tv, grid, a.stream)
+                           : launch_rows<D, BF16, false>(rp, tk, tv, grid, a.stream);
         if (rc == PA_OK && pl.max_splits > 1)
             rc = launch_merge<D, BF16>(rp, a.stream);
         return rc;

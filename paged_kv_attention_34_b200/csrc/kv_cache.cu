@@ -7,6 +7,8 @@
 // iopencloud "大模型推理加速技术全景" section 3.2 (16-token pages, per-request
 // page table); copy-on-write of refcounted blocks follows the zhihu roofline
 // page, "显存管理".
+#include <cuda_fp8.h>
+
 #include "pa_device.cuh"
 #include "pa_internal.h"
 
@@ -98,6 +100,69 @@ __global__ void __launch_bounds__(256) kv_block_swap_kernel(uint4 *__restrict__ 
             const uint4 vv = host_value[hi];
             key_cache[di] = kv;
             value_cache[di] = vv;
+        }
+    }
+}
+
+// FP8 cache write: one warp per (token, KV head) row of K and of V.  The row's scale is
+// amax / 448 (1 for an all-zero row) and every value becomes the E4M3 code nearest to value /
+// scale (saturated at +-448); both divisions are IEEE round-to-nearest, so the codes follow from
+// the 16-bit inputs alone.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) kv_cache_write_fp8_kernel(const void *__restrict__ k_new,
+                                                                 const void *__restrict__ v_new,
+                                                                 const int32_t *__restrict__ slot_mapping, int64_t T,
+                                                                 int H_kv, uint8_t *__restrict__ key_cache,
+                                                                 uint8_t *__restrict__ value_cache, float *key_scale,
+                                                                 float *value_scale, int64_t num_blocks, int32_t *status)
+{
+    constexpr int VPL = D / 32;  // values per lane (2 or 4)
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t r = blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5); r < T * H_kv; r += warps) {
+        const int64_t t = r / H_kv;
+        const int h = static_cast<int>(r % H_kv);
+        const int64_t slot = __ldg(slot_mapping + t);
+        if (slot < 0)
+            continue;  // padding token
+        if (slot >= num_blocks * 16) {
+            if (lane == 0)
+                set_status(status, PA_ERR_BOUNDS);
+            continue;
+        }
+        const int64_t row = ((slot / 16) * H_kv + h) * 16 + slot % 16;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+            const uint16_t *src = static_cast<const uint16_t *>(kv ? v_new : k_new) + (t * H_kv + h) * D + lane * VPL;
+            float x[VPL], amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) {
+                const uint16_t u = src[i];
+                if constexpr (BF16)
+                    x[i] = __bfloat162float(__ushort_as_bfloat16(u));
+                else
+                    x[i] = __half2float(__ushort_as_half(u));
+                amax = fmaxf(amax, fabsf(x[i]));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+            uint8_t code[VPL];
+#pragma unroll
+            for (int i = 0; i < VPL; i += 2) {
+                const float2 qv = make_float2(__fdiv_rn(x[i], sc), __fdiv_rn(x[i + 1], sc));
+                const __nv_fp8x2_storage_t pr = __nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
+                code[i] = static_cast<uint8_t>(pr & 0xffu);
+                code[i + 1] = static_cast<uint8_t>(pr >> 8);
+            }
+            uint8_t *dst = (kv ? value_cache : key_cache) + row * D + lane * VPL;
+            if constexpr (VPL == 4)
+                *reinterpret_cast<uint32_t *>(dst) = code[0] | (code[1] << 8) | (code[2] << 16) | (uint32_t(code[3]) << 24);
+            else
+                *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(code[0] | (code[1] << 8));
+            if (lane == 0)
+                (kv ? value_scale : key_scale)[row] = sc;
         }
     }
 }
@@ -210,6 +275,37 @@ extern "C" int pa_kv_block_swap(void *key_cache, void *value_cache, int64_t num_
     kv_block_swap_kernel<<<grid_for(n * chunks, threads), threads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), num_blocks, static_cast<uint4 *>(hk),
         static_cast<uint4 *>(hv), host_blocks, chunks, pairs, n, direction == PA_SWAP_OUT ? 1 : 0, status);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_kv_cache_write_fp8(const void *k_new, const void *v_new, const int32_t *slot_mapping, int64_t T,
+                                     uint8_t *key_cache, uint8_t *value_cache, float *key_scale, float *value_scale,
+                                     int64_t num_blocks, int H_kv, int d, pa_dtype dtype, int32_t *status, void *stream)
+{
+    if (T < 0 || num_blocks < 1 || H_kv < 1)
+        return PA_ERR_ARG;
+    if (dtype != PA_F16 && dtype != PA_BF16)
+        return PA_ERR_ARG;
+    if (d != 64 && d != 128)
+        return PA_ERR_UNSUPPORTED;
+    if (T == 0)
+        return PA_OK;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        !aligned4(key_scale) || !aligned4(value_scale) || !aligned4(slot_mapping) || (status && !aligned4(status)))
+        return PA_ERR_ALIGN;
+    const int threads = 256;
+    const int64_t warps_needed = T * H_kv;
+    const int grid = grid_for(warps_needed * 32, threads);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+#define PA_LAUNCH_WRITE8(DD, BB)                                                                                   \
+    kv_cache_write_fp8_kernel<DD, BB><<<grid, threads, 0, s>>>(k_new, v_new, slot_mapping, T, H_kv, key_cache,     \
+                                                               value_cache, key_scale, value_scale, num_blocks, status)
+    if (d == 128)
+        dtype == PA_BF16 ? PA_LAUNCH_WRITE8(128, true) : PA_LAUNCH_WRITE8(128, false);
+    else
+        dtype == PA_BF16 ? PA_LAUNCH_WRITE8(64, true) : PA_LAUNCH_WRITE8(64, false);
+#undef PA_LAUNCH_WRITE8
     count_launch();
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -62,6 +62,23 @@ int make_cache_tmap(CUtensorMap *map, const void *cache, int64_t num_blocks, int
     return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+// FP8 cache: the same rows of d one-byte codes; one box = a page (16 rows x d bytes), no swizzle.
+int make_cache_tmap_fp8(CUtensorMap *map, const void *cache, int64_t num_blocks, int H_kv, int d)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return PA_ERR_CUDA;
+    const int64_t rows = num_blocks * H_kv * 16;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(d), 16};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(cache), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
 int make_q_tmap(CUtensorMap *map, const void *q, int64_t T, int H_q, int d, int G, int tok, pa_dtype dtype)
 {
     auto fn = encode_fn();
@@ -165,6 +182,33 @@ extern "C" int pa_paged_attn_decode_tree(void *out, const void *q, const void *k
         if (!tree_mask)
             return PA_ERR_ARG;
         if (!aligned4(tree_mask))
+            return PA_ERR_ALIGN;
+    }
+    if (workspace_bytes < decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx))
+        return PA_ERR_WORKSPACE;
+    rc = reset_status(workspace, a.stream);
+    if (rc != PA_OK || B == 0 || T == 0)
+        return rc;
+    return launch_decode(a);
+}
+
+extern "C" int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t *key_cache,
+                                        const uint8_t *value_cache, const float *key_scale, const float *value_scale,
+                                        int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
+                                        const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int max_ctx,
+                                        int64_t T, int H_q, int H_kv, int d, float scale, pa_dtype dtype,
+                                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
+               context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
+               static_cast<cudaStream_t>(stream), nullptr, key_scale, value_scale};
+    int rc = check_attn(a, true);
+    if (rc != PA_OK)
+        return rc;
+    if (B > 0 && T > 0) {
+        if (!key_scale || !value_scale)
+            return PA_ERR_ARG;
+        if (!aligned4(key_scale) || !aligned4(value_scale))
             return PA_ERR_ALIGN;
     }
     if (workspace_bytes < decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx))

@@ -19,6 +19,7 @@ inline bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p
 // 2-D tensor map over a paged cache [num_blocks][H_kv][16][d] viewed as
 // rows of d elements; box = 64 elements x 16 rows, 128-byte swizzle.
 // Returns PA_OK or PA_ERR_CUDA / PA_ERR_ARG.
+int make_cache_tmap_fp8(CUtensorMap *map, const void *cache, int64_t num_blocks, int H_kv, int d);
 int make_cache_tmap(CUtensorMap *map, const void *cache, int64_t num_blocks, int H_kv, int d, pa_dtype dtype);
 
 // 3-D tensor map over Q [T][H_q][d] for query tiles of `tok` tokens x G heads of one
@@ -55,6 +56,8 @@ struct AttnArgs {
     size_t workspace_bytes;
     cudaStream_t stream;
     const int32_t *tree_mask = nullptr;  // decode only: per-token visibility bits of the new tokens
+    const float *key_scale = nullptr;    // FP8 cache (decode only): per-row scales, else nullptr
+    const float *value_scale = nullptr;
 };
 
 // Split-KV decode plan: pages per split and the number of splits.

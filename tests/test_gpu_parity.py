@@ -130,6 +130,104 @@ def test_prefill_fresh_prompts_exact_lengths():
     run_and_compare(w)
 
 
+# ---- FP8 (E4M3) KV cache ---------------------------------------------------------------------
+
+def _fp8_device_cache(w):
+    """The workload's cache (every stored row, then the step's new tokens) written into an FP8 cache on
+    the device: (codes K, codes V, scales K, scales V)."""
+    NB, H, _, d = w.key_cache.shape
+    kc8 = torch.zeros((NB, H, 16, d), dtype=torch.uint8, device="cuda")
+    vc8 = torch.zeros_like(kc8)
+    ks = torch.ones((NB, H, 16), dtype=torch.float32, device="cuda")
+    vs = torch.ones_like(ks)
+    rows_k = w.key_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous().cuda()
+    rows_v = w.value_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous().cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.kv_cache_write_fp8(rows_k, rows_v, torch.arange(NB * 16, dtype=torch.int32, device="cuda"), kc8, vc8, ks, vs,
+                          status=status)
+    pa.kv_cache_write_fp8(w.k_new.cuda(), w.v_new.cuda(), w.slot_mapping.cuda(), kc8, vc8, ks, vs, status=status)
+    torch.cuda.synchronize()
+    assert pa.read_status(status) == 0
+    return kc8, vc8, ks, vs
+
+
+def _fp8_decode(w, kc8, vc8, ks, vs):
+    call = next(c for c in DeviceStep(w).calls if c.kind == "decode")
+    out = pa.paged_attn_decode_fp8(call.q, kc8, vc8, ks, vs, call.bt, call.cu, call.ctx, call.max_ctx, w.scale,
+                                   workspace=call.ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(call.ws) == 0
+    return out
+
+
+FP8_CASES = [
+    (4, 1, 300, 2, 1, 128, W.F16),
+    (3, 4, 500, 2, 4, 128, W.BF16),
+    (3, 8, 400, 2, 8, 64, W.F16),
+    (5, 6, 2000, 2, 4, 128, W.BF16),  # several splits
+    (4, 3, 33, 2, 2, 64, W.BF16),     # tiny contexts, partial blocks
+]
+
+
+@pytest.mark.parametrize("idx", range(len(FP8_CASES)), ids=lambda i: _case_id(FP8_CASES[i]))
+def test_fp8_cache_and_decode_small(idx):
+    B, q_max, ctx_max, H_kv, G, d, dt = FP8_CASES[idx]
+    w = W.random_workload(800 + 7 * idx, B=B, q_max=q_max, ctx_max=ctx_max, H_kv=H_kv, G=G, d=d, dtype=dt,
+                          kind="decode")
+    kc8, vc8, ks, vs = _fp8_device_cache(w)
+    # the cache, byte for byte and scale for scale, as the oracle writes it
+    NB, H = w.key_cache.shape[:2]
+    okc, ovc = np.zeros((NB, H, 16, d), np.uint8), np.zeros((NB, H, 16, d), np.uint8)
+    oks, ovs = np.ones((NB, H, 16), np.float32), np.ones((NB, H, 16), np.float32)
+    rows_k = w.key_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous()
+    rows_v = w.value_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous()
+    dtc = oracle.dtype_code(w.dtype)
+    assert oracle.kv_cache_write_fp8(rows_k, rows_v, dtc, torch.arange(NB * 16, dtype=torch.int32), okc, ovc, oks,
+                                     ovs) == 0
+    assert oracle.kv_cache_write_fp8(w.k_new, w.v_new, dtc, w.slot_mapping, okc, ovc, oks, ovs) == 0
+    assert np.array_equal(kc8.cpu().numpy(), okc) and np.array_equal(vc8.cpu().numpy(), ovc)
+    assert np.array_equal(ks.cpu().numpy().view(np.uint32), oks.view(np.uint32))
+    assert np.array_equal(vs.cpu().numpy().view(np.uint32), ovs.view(np.uint32))
+    # attention over it
+    got = _fp8_decode(w, kc8, vc8, ks, vs).double().cpu().numpy()
+    ref = oracle.paged_attention_fp8(w.q, dtc, okc, ovc, oks, ovs, w.block_tables, w.cu_seqlens_q, w.context_lens,
+                                     w.H_kv, w.scale)
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref).max()
+    assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
+
+
+def test_fp8_decode_13b_layer_sampled():
+    # the 13B-shaped decode layer (64 sequences, 40 heads, contexts U[128, 4096]) over an FP8 cache
+    w = W.config2()
+    kc8, vc8, ks, vs = _fp8_device_cache(w)
+    out = _fp8_decode(w, kc8, vc8, ks, vs)
+    rows = sample_rows(w, 200, seed=6)
+    ref = oracle.paged_attention_fp8(w.q, oracle.dtype_code(w.dtype), kc8.cpu().numpy(), vc8.cpu().numpy(),
+                                     ks.cpu().numpy(), vs.cpu().numpy(), w.block_tables, w.cu_seqlens_q,
+                                     w.context_lens, w.H_kv, w.scale, rows=rows)
+    got = out.double().cpu().numpy().reshape(w.T * w.H_q, w.d)[rows]
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref).max()
+    assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
+
+
+def test_fp8_decode_rejects_missing_scales():
+    import ctypes
+
+    w = W.random_workload(5, B=2, q_max=1, ctx_max=40, H_kv=1, G=1, d=64, dtype=W.F16, kind="decode")
+    kc8, vc8, ks, vs = _fp8_device_cache(w)
+    call = DeviceStep(w).calls[0]
+    n0 = pa.launch_count()
+    rc = pa.lib().pa_paged_attn_decode_fp8(
+        ctypes.c_void_p(call.out.data_ptr()), ctypes.c_void_p(call.q.data_ptr()), ctypes.c_void_p(kc8.data_ptr()),
+        ctypes.c_void_p(vc8.data_ptr()), None, ctypes.c_void_p(vs.data_ptr()), kc8.shape[0],
+        ctypes.c_void_p(call.bt.data_ptr()), call.bt.shape[1], ctypes.c_void_p(call.cu.data_ptr()),
+        ctypes.c_void_p(call.ctx.data_ptr()), call.ctx.shape[0], call.max_ctx, call.q.shape[0], w.H_q, w.H_kv, w.d,
+        w.scale, 0, ctypes.c_void_p(call.ws.data_ptr()), call.ws.numel(), None)
+    assert rc == -1 and pa.launch_count() == n0
+
+
 # ---- tree-attention verification ---------------------------------------------------------
 
 def _tree_run(w, tm):
