@@ -160,10 +160,12 @@ def f64_to_e4m3(x: float, L=None) -> int:
 
 def kv_cache_write_fp8(k_new, v_new, dtype: int, slot_mapping, key_cache: np.ndarray, value_cache: np.ndarray,
                        key_scale: np.ndarray, value_scale: np.ndarray, L=None) -> int:
-    """FP8 cache write: codes uint8 [NB, H_kv, 16, d], scales float32 [NB, H_kv, 16]; in place."""
+    """FP8 cache write: K codes uint8 [NB, H_kv, 16, d], V codes uint8 [NB, H_kv, d, 16] (transposed
+    within the block), scales float32 [NB, H_kv, 16]; in place."""
     kn, vn = _u16(k_new), _u16(v_new)
     sm = _i32(slot_mapping)
     NB, H_kv, _, d = key_cache.shape
+    assert value_cache.shape == (NB, H_kv, d, 16)
     for a, dt in ((key_cache, np.uint8), (value_cache, np.uint8), (key_scale, np.float32), (value_scale, np.float32)):
         assert a.dtype == dt and a.flags.c_contiguous
     return (L or lib()).oracle_kv_cache_write_fp8(_p(kn), _p(vn), dtype, _p(sm), sm.shape[0], _p(key_cache),

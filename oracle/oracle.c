@@ -511,9 +511,10 @@ uint8_t oracle_f64_to_e4m3(double x)
     return sign | (uint8_t)best;
 }
 
-/* One row of d 16-bit values -> d codes and the row's scale: scale = amax / 448 (1 when amax is
- * 0), code_k = e4m3(x_k / scale), both divisions in float rounded to nearest, as the device does. */
-static float quant_row(const uint16_t *src, int dtype, int d, uint8_t *dst)
+/* One row of d 16-bit values -> d codes (code k at dst[k * stride]) and the row's scale:
+ * scale = amax / 448 (1 when amax is 0), code_k = e4m3(x_k / scale), both divisions in float
+ * rounded to nearest, as the device does. */
+static float quant_row(const uint16_t *src, int dtype, int d, uint8_t *dst, int64_t stride)
 {
     float amax = 0.0f;
     for (int k = 0; k < d; ++k) {
@@ -524,12 +525,14 @@ static float quant_row(const uint16_t *src, int dtype, int d, uint8_t *dst)
     float sc = amax > 0.0f ? amax / 448.0f : 1.0f;
     for (int k = 0; k < d; ++k) {
         float q = (float)widen(src[k], dtype) / sc;
-        dst[k] = oracle_f64_to_e4m3((double)q);
+        dst[k * stride] = oracle_f64_to_e4m3((double)q);
     }
     return sc;
 }
 
-/* kv_cache_write into the FP8 cache: codes [NB][H_kv][16][d], scales [NB][H_kv][16]. */
+/* kv_cache_write into the FP8 cache.  Per (block, KV head): K codes [16 slots][d], V codes
+ * transposed, [d][16 slots] (the value-cache layout of vLLM's paged attention kernel); scales
+ * [NB][H_kv][16] for each of K and V. */
 int64_t oracle_kv_cache_write_fp8(const uint16_t *k_new, const uint16_t *v_new, int dtype,
                                   const int32_t *slot_mapping, int64_t T, uint8_t *key_cache, uint8_t *value_cache,
                                   float *key_scale, float *value_scale, int64_t num_blocks, int H_kv, int d)
@@ -548,14 +551,16 @@ int64_t oracle_kv_cache_write_fp8(const uint16_t *k_new, const uint16_t *v_new, 
         for (int h = 0; h < H_kv; ++h) {
             int64_t row = (block * H_kv + h) * ORACLE_BLOCK + offset;
             int64_t src = (t * H_kv + h) * (int64_t)d;
-            key_scale[row] = quant_row(k_new + src, dtype, d, key_cache + row * d);
-            value_scale[row] = quant_row(v_new + src, dtype, d, value_cache + row * d);
+            uint8_t *vt = value_cache + (block * H_kv + h) * ORACLE_BLOCK * (int64_t)d + offset;
+            key_scale[row] = quant_row(k_new + src, dtype, d, key_cache + row * d, 1);
+            value_scale[row] = quant_row(v_new + src, dtype, d, vt, ORACLE_BLOCK);
         }
     }
     return bad;
 }
 
-/* Attention of one row over the FP8 cache: K_j = e4m3(code) * scale of its row, likewise V. */
+/* Attention of one row over the FP8 cache: K_j = e4m3(code) * scale of its row, likewise V (whose
+ * codes sit transposed in their block). */
 static int attention_row_fp8(double *out_row, const uint16_t *q, int dtype, const uint8_t *key_cache,
                              const uint8_t *value_cache, const float *key_scale, const float *value_scale,
                              const int32_t *block_tables, int max_blocks, int b, int i, int q_b, int ctx_b,
@@ -590,8 +595,9 @@ static int attention_row_fp8(double *out_row, const uint16_t *q, int dtype, cons
         int64_t block = block_tables[(int64_t)b * max_blocks + j / ORACLE_BLOCK];
         int64_t row = (block * H_kv + g) * ORACLE_BLOCK + j % ORACLE_BLOCK;
         double w = s[j] / z, vs = value_scale[row];
+        const uint8_t *vt = value_cache + (block * H_kv + g) * ORACLE_BLOCK * (int64_t)d + j % ORACLE_BLOCK;
         for (int k = 0; k < d; ++k)
-            out_row[k] += w * (oracle_e4m3_to_f64(value_cache[row * d + k]) * vs);
+            out_row[k] += w * (oracle_e4m3_to_f64(vt[k * ORACLE_BLOCK]) * vs);
     }
     return 0;
 }

@@ -229,11 +229,12 @@ def pin_e4m3_codec(L):
 
 
 def _fp8_case(seed, B=3, q_max=1, ctx_max=60, H_kv=2, G=2, d=32, dt=W.BF16):
-    """A small decode workload with its cache written to FP8 by the oracle (every context row)."""
+    """A small decode workload with its cache written to FP8 by the oracle (every context row);
+    V codes are [NB, H_kv, d, 16], transposed within each block."""
     w = W.random_workload(seed, B=B, q_max=q_max, ctx_max=ctx_max, H_kv=H_kv, G=G, d=d, dtype=dt, kind="decode")
     NB = w.key_cache.shape[0]
     kc8 = np.zeros((NB, H_kv, 16, d), np.uint8)
-    vc8 = np.zeros((NB, H_kv, 16, d), np.uint8)
+    vc8 = np.zeros((NB, H_kv, d, 16), np.uint8)
     ks = np.ones((NB, H_kv, 16), np.float32)
     vs = np.ones((NB, H_kv, 16), np.float32)
     # every stored row (the cached context and the step's new tokens) goes through the FP8 write
@@ -255,7 +256,7 @@ def pin_fp8_write(L):
     vn = (torch.randn((T, H, d), generator=g) * 30).bfloat16()
     vn[2, 1] = 0
     NB = 2
-    kc8, vc8 = np.zeros((NB, H, 16, d), np.uint8), np.zeros((NB, H, 16, d), np.uint8)
+    kc8, vc8 = np.zeros((NB, H, 16, d), np.uint8), np.zeros((NB, H, d, 16), np.uint8)
     ks, vs = np.zeros((NB, H, 16), np.float32), np.zeros((NB, H, 16), np.float32)
     slots = torch.tensor([0, 5, 17, 31, -1, 16], dtype=torch.int32)
     assert oracle.kv_cache_write_fp8(kn, vn, oracle.dtype_code(W.BF16), slots, kc8, vc8, ks, vs, L=L) == 0
@@ -263,7 +264,8 @@ def pin_fp8_write(L):
         if sl < 0:
             continue
         for h in range(H):
-            for new, c8, sc in ((kn, kc8, ks), (vn, vc8, vs)):
+            # a V row is a column of its block: V codes are [NB, H, d, 16]
+            for new, c8, sc in ((kn, kc8, ks), (vn, vc8.transpose(0, 1, 3, 2), vs)):
                 x = new[t, h].double()
                 amax = float(x.abs().max())
                 s_ref = np.float32(amax) / np.float32(448.0) if amax > 0 else np.float32(1.0)
@@ -274,7 +276,9 @@ def pin_fp8_write(L):
                 # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 for normals, absolute 2^-10 * scale below
                 bound = torch.maximum(x.abs() * 2.0 ** -4, torch.full_like(x, 2.0 ** -10 * float(s_ref)))
                 assert bool(((deq - x).abs() <= bound + 1e-12).all())
-    assert not vc8[1, 1, 1].any() and vs[1, 1, 1] == 1.0  # the zero row (token 2 -> slot 17)
+    assert not vc8[1, 1, :, 1].any() and vs[1, 1, 1] == 1.0  # the zero row (token 2 -> slot 17)
+    # writing one slot touches only that slot's column of the V block
+    assert not vc8[0, :, :, [c for c in range(16) if c not in (0, 5)]].any()
     assert oracle.kv_cache_write_fp8(kn[:1], vn[:1], oracle.dtype_code(W.BF16), torch.tensor([NB * 16], dtype=torch.int32), kc8, vc8,
                                      ks, vs, L=L) == 1
 
@@ -287,7 +291,8 @@ def pin_fp8_attention(L):
         got = oracle.paged_attention_fp8(w.q, oracle.dtype_code(w.dtype), kc8, vc8, ks, vs, w.block_tables,
                                          w.cu_seqlens_q, w.context_lens, w.H_kv, w.scale, L=L)
         deq = lambda c8, sc: (_e4m3_values(c8.reshape(-1)).reshape(c8.shape) * torch.from_numpy(sc).double()[..., None])
-        w2 = W.Workload(**{**vars(w), "key_cache": deq(kc8, ks), "value_cache": deq(vc8, vs),
+        vrows = np.ascontiguousarray(vc8.transpose(0, 1, 3, 2))  # back to [NB, H_kv, 16, d]
+        w2 = W.Workload(**{**vars(w), "key_cache": deq(kc8, ks), "value_cache": deq(vrows, vs),
                            "slot_mapping": torch.full_like(w.slot_mapping, -1)})
         ref = sdpa_reference(w2)
         err = np.abs(got - ref).max()

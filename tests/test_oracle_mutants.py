@@ -66,6 +66,8 @@ MUTANTS = {
                            "float sc = amax > 0.0f ? amax / 240.0f : 1.0f;"),
     "fp8_value_scale_from_keys": ("double w = s[j] / z, vs = value_scale[row];",
                                   "double w = s[j] / z, vs = key_scale[row];"),
+    "fp8_value_untransposed": ("out_row[k] += w * (oracle_e4m3_to_f64(vt[k * ORACLE_BLOCK]) * vs);",
+                               "out_row[k] += w * (oracle_e4m3_to_f64(vt[k]) * vs);"),
     "online_no_rescale": ("o[c] = alpha * o[c] + acc;", "o[c] = o[c] + acc;"),
     "merge_sign": ("double w = exp(lses[s] - m) / z;", "double w = exp(m - lses[s]) / z;"),
 }
