@@ -537,7 +537,7 @@ def leg_fp8(args, stream, device, hbm_peak, rank):
     call = st.calls[0]
     NB, H, _, d = st.key_cache.shape
     kc8 = torch.zeros((NB, H, 16, d), dtype=torch.uint8, device=device)
-    vc8 = torch.zeros_like(kc8)
+    vc8 = torch.zeros((NB, H, d, 16), dtype=torch.uint8, device=device)  # transposed within the block
     ks = torch.ones((NB, H, 16), dtype=torch.float32, device=device)
     vs = torch.ones_like(ks)
     rows_k = st.key_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous()

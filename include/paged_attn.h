@@ -185,11 +185,15 @@ int pa_paged_attn_decode_tree(void *out, const void *q, const void *key_cache, c
  * FP8 (E4M3) KV cache -- an 8-bit cache with one float scale per stored row
  * (the FP8 KV-cache option of the serving page; FP8 with scaling on the
  * interview Q&A page): half the HBM bytes of a 16-bit cache per key.
- *   key_cache, value_cache  uint8 [num_blocks][H_kv][16][d]: E4M3 codes
+ *   key_cache               uint8 [num_blocks][H_kv][16][d]: E4M3 codes
  *                           (OCP FP8: bias 7, 3 mantissa bits, no infinities,
  *                           largest finite 448)
+ *   value_cache             uint8 [num_blocks][H_kv][d][16]: E4M3 codes,
+ *                           transposed within each block (vLLM's value-cache
+ *                           layout), so a slot's row is a column of its block
  *   key_scale, value_scale  float [num_blocks][H_kv][16]: the row's scale;
- *                           the stored value is code x scale
+ *                           the stored value is code x scale (16-byte
+ *                           aligned for the decode call, else PA_ERR_ALIGN)
  * A row's scale is fixed when the row is written (amax / 448), so nothing
  * stored is ever requantised.
  *
@@ -204,9 +208,10 @@ int pa_kv_cache_write_fp8(const void *k_new, const void *v_new, const int32_t *s
 
 /*
  * pa_paged_attn_decode_fp8 -- pa_paged_attn_decode over the FP8 cache: the
- * same sizes, workspace, scheduling and errors; K and V are dequantised
- * (code x scale, rounded to `dtype`, the type of q and out) in shared memory
- * and the attention runs as in the 16-bit call.  NULL scales -> PA_ERR_ARG.
+ * same sizes, workspace, scheduling and errors.  The codes are widened exactly
+ * to `dtype` (the type of q and out; every E4M3 value is an f16 and a bf16
+ * value) in registers, and the row scales multiply the fp32 scores (K) and
+ * the probabilities before P V (V).  NULL scales -> PA_ERR_ARG.
  */
 int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t *key_cache, const uint8_t *value_cache,
                              const float *key_scale, const float *value_scale, int64_t num_blocks,

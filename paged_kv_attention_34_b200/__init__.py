@@ -276,8 +276,8 @@ def _fp8_cache(key_cache, value_cache, key_scale, value_scale):
     _cuda(key_cache, "key_cache", torch.uint8, 4)
     _cuda(value_cache, "value_cache", torch.uint8, 4)
     NB, H_kv, bs, d = key_cache.shape
-    if bs != 16 or tuple(value_cache.shape) != tuple(key_cache.shape):
-        raise ValueError("FP8 caches must be uint8 [NB, H_kv, 16, d], both the same shape")
+    if bs != 16 or tuple(value_cache.shape) != (NB, H_kv, d, 16):
+        raise ValueError("FP8 caches must be uint8: keys [NB, H_kv, 16, d], values [NB, H_kv, d, 16]")
     for name, t in (("key_scale", key_scale), ("value_scale", value_scale)):
         _cuda(t, name, torch.float32, 3)
         if tuple(t.shape) != (NB, H_kv, 16):
@@ -287,8 +287,9 @@ def _fp8_cache(key_cache, value_cache, key_scale, value_scale):
 
 def kv_cache_write_fp8(k_new, v_new, slot_mapping, key_cache, value_cache, key_scale, value_scale, status=None,
                        stream=None):
-    """Quantise k_new/v_new [T, H_kv, d] (16-bit) into the FP8 cache (uint8 codes [NB, H_kv, 16, d] and
-    float32 row scales [NB, H_kv, 16]) at slot_mapping [T]."""
+    """Quantise k_new/v_new [T, H_kv, d] (16-bit) into the FP8 cache (uint8 codes: keys [NB, H_kv, 16, d],
+    values transposed within the block [NB, H_kv, d, 16]; float32 row scales [NB, H_kv, 16]) at
+    slot_mapping [T]."""
     NB, H_kv, d = _fp8_cache(key_cache, value_cache, key_scale, value_scale)
     _cuda(k_new, "k_new", None, 3)
     _cuda(v_new, "v_new", k_new.dtype, 3)

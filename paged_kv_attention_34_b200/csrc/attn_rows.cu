@@ -531,34 +531,175 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---- FP8 (E4M3) cache -----------------------------------------------------------------------
-// The same split-KV decode over an 8-bit cache with one float scale per stored row.  TMA brings
-// each page's codes (16 rows x d bytes, one box for K and one for V) into a three-stage ring; per
-// stage the whole CTA converts the four pages' codes into their 16-bit values in one stage laid
-// out like the 16-bit cache's (128-byte swizzle) and stages the row scales, and the warps run
-// rows_page on it with the scales folded into the scores and into P.  Half the HBM bytes of the
-// 16-bit cache per key.
-constexpr int kFp8Stages = 3;
+// The split-KV decode over an 8-bit cache with one float scale per stored row.  Per (block, KV
+// head) the K codes are [16 keys][d] and the V codes [d][16 keys] (transposed, like vLLM's value
+// cache), so both reach the mma.sync operand fragments through plain shared-memory loads and are
+// widened to 16 bits in registers, with no dequantised copy of the page:
+//  - S = Q K^T sums over d in any order: k-step ks of lane quad kq takes the columns
+//    d = kq*(D/4) + 4ks + {0..3} (Q's fragments are built in the same order), so a lane reads
+//    D/4 contiguous code bytes of a key row;
+//  - the keys of a page sit in S's columns so that the four keys a lane quad holds in P (the A
+//    operand of P V) are 4kq .. 4kq+3: one 32-bit word of a transposed V row per n-tile.
+// The row scales of every page of the split are loaded into shared memory once; they multiply the
+// fp32 scores (K) and the probabilities before P V (V).  Pipeline and epilogue as the 16-bit
+// kernel: a four-stage TMA ring (one 16 x d-byte box per page for K and one for V), refilled by
+// the last warp done with a stage.
+constexpr int kFp8Stages = 4;
 
 template <int D>
 struct Fp8Smem {
-    static constexpr int kPage8 = 16 * D;                            // codes of one page
-    static constexpr int kStage8 = 2 * kPagesPerStage * kPage8;      // K pages then V pages
-    static constexpr int kPage16 = 16 * D * 2;
-    static constexpr int kStage16 = 2 * kPagesPerStage * kPage16;    // one dequantised stage
-    static constexpr int kQBytes = kRowsPerCta * D * 2;
-    static constexpr int kWork = ((kStage16 > RowsEpi<D>::kBytes ? kStage16 : RowsEpi<D>::kBytes) + 1023) / 1024 * 1024;
-    static_assert(kQBytes <= kWork, "Q is staged through the dequantised stage");
-    static constexpr int kWorkOff = 0;                               // dequantised stage / Q / epilogue
-    static constexpr int kRingOff = kWork;
-    static constexpr int kBarOff = kRingOff + kFp8Stages * kStage8;
-    static constexpr int kIssuedOff = kBarOff + 8 * kFp8Stages;
-    static constexpr int kCountOff = kIssuedOff + 4 * kFp8Stages;               // warps done with each stage
-    static constexpr int kFlagOff = kCountOff + 4 * kFp8Stages;                 // abort flag
-    static constexpr int kScaleOff = kFlagOff + 16;                             // [K, V][4 pages][16 rows]
-    static constexpr int kTableOff = kScaleOff + 4 * 2 * kPagesPerStage * 16;
-    static constexpr int kBytes = kTableOff + 4 * kMaxTablePages;
-    static constexpr int kAlloc = kBytes + 1024;
+    static constexpr int kPage = 16 * D;                       // codes of one page of K or of V
+    static constexpr int kStage = 2 * kPagesPerStage * kPage;  // K pages then V pages
+    static_assert(RowsEpi<D>::kBytes <= kFp8Stages * kStage, "the epilogue reuses the ring");
+    static constexpr int kRingOff = 0;
+    static constexpr int kScaleOff = kFp8Stages * kStage;          // [page of the split][K, V][16 keys]
+    static constexpr int kBarOff = kScaleOff + kMaxTablePages * 2 * 16 * 4;
+    static constexpr int kCountOff = kBarOff + 8 * kFp8Stages;     // warps done with each stage
+    static constexpr int kIssuedOff = kCountOff + 4 * kFp8Stages;  // loads issued into each stage
+    static constexpr int kTableOff = kIssuedOff + 4 * kFp8Stages;
+    static constexpr int kFlagOff = kTableOff + 4 * kMaxTablePages;
+    static constexpr int kBytes = kFlagOff + 16;
+    static constexpr int kAlloc = kBytes + 128;  // slack to align the base to 128 B
 };
+
+// Two E4M3 codes (the low 16 bits of `pair`) -> two 16-bit values; exact, as every E4M3 value is
+// an f16 and a bf16 value.
+template <bool BF16>
+__device__ __forceinline__ uint32_t widen_e4m3x2(uint32_t pair)
+{
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair & 0xffffu), __NV_E4M3);
+    if constexpr (BF16) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+        return pack2<true>(f.x, f.y);
+    } else {
+        return static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+    }
+}
+
+// One page of 16 keys for the 16 rows of a warp's m-tile, straight from the codes in shared memory
+// (kp: K [16][D], vp: V [D][16]) and the page's scales (sc: 16 for K, then 16 for V).  Rows and
+// state as rows_page; keys past `ctx` may hold anything (NaN codes, any scale) and are masked.
+template <int D, bool BF16>
+__device__ __forceinline__ void rows_page_fp8(const uint8_t *kp, const uint8_t *vp, const float *sc, int j0, int lane,
+                                              const uint32_t (&qa)[D / 16][4], float (&o)[D / 8][4], float &m_a,
+                                              float &m_b, float &l_a, float &l_b, int lim_a, int lim_b, int ctx,
+                                              float sl2)
+{
+    constexpr int KSTEPS = D / 16;  // k-steps of S = Q K^T
+    constexpr int NT = D / 8;       // n-tiles of O
+    constexpr int SPAN = D / 4;     // code bytes of a key row per lane quad
+    const int r = lane >> 2, kq = lane & 3;
+
+    // S (16 rows x 16 keys) = Q K^T.  Column r of n-tile t is key 4(r/2) + 2t + r%2; the k-steps
+    // alternate between two accumulators, which halves the chain of dependent MMAs.
+    float s[2][4], s2[2][4];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            s[t][i] = s2[t][i] = 0.f;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const uint8_t *row = kp + (4 * (r >> 1) + 2 * t + (r & 1)) * D + kq * SPAN;
+        uint32_t w[SPAN / 4];
+#pragma unroll
+        for (int i = 0; i < SPAN / 16; ++i) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(row + i * 16);
+            w[4 * i] = v.x;
+            w[4 * i + 1] = v.y;
+            w[4 * i + 2] = v.z;
+            w[4 * i + 3] = v.w;
+        }
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+            const uint32_t b0 = widen_e4m3x2<BF16>(w[ks]), b1 = widen_e4m3x2<BF16>(w[ks] >> 16);
+            if (ks & 1)
+                mma16816<BF16>(s2[t], qa[ks], b0, b1);
+            else
+                mma16816<BF16>(s[t], qa[ks], b0, b1);
+        }
+    }
+    // key scales, mask (causal / context end), log2 units, online softmax.  This lane's keys are
+    // 4kq + {0, 1} (n-tile 0) and 4kq + {2, 3} (n-tile 1).
+    const float4 kf4 = *reinterpret_cast<const float4 *>(sc + 4 * kq);
+    const float kf[4] = {kf4.x, kf4.y, kf4.z, kf4.w};
+    float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const int key = j0 + 4 * kq + 2 * t + c;
+            const float f = sl2 * kf[2 * t + c];
+            s[t][c] = key <= lim_a ? (s[t][c] + s2[t][c]) * f : -INFINITY;
+            s[t][2 + c] = key <= lim_b ? (s[t][2 + c] + s2[t][2 + c]) * f : -INFINITY;
+            mx_a = fmaxf(mx_a, s[t][c]);
+            mx_b = fmaxf(mx_b, s[t][2 + c]);
+        }
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+    const float base_a = mn_a == -INFINITY ? 0.f : mn_a;
+    const float base_b = mn_b == -INFINITY ? 0.f : mn_b;
+    const float al_a = fast_exp2(m_a - base_a), al_b = fast_exp2(m_b - base_b);
+    m_a = mn_a;
+    m_b = mn_b;
+    float ps_a = 0.f, ps_b = 0.f;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        s[t][0] = fast_exp2(s[t][0] - base_a);
+        s[t][1] = fast_exp2(s[t][1] - base_a);
+        s[t][2] = fast_exp2(s[t][2] - base_b);
+        s[t][3] = fast_exp2(s[t][3] - base_b);
+        ps_a += s[t][0] + s[t][1];
+        ps_b += s[t][2] + s[t][3];
+    }
+    l_a = l_a * al_a + ps_a;
+    l_b = l_b * al_b + ps_b;
+    if (__any_sync(0xffffffffu, al_a != 1.f || al_b != 1.f)) {
+#pragma unroll
+        for (int nd = 0; nd < NT; ++nd) {
+            o[nd][0] *= al_a;
+            o[nd][1] *= al_a;
+            o[nd][2] *= al_b;
+            o[nd][3] *= al_b;
+        }
+    }
+    // value scales into P, then P in the A layout of P V: logical keys 2kq + {0, 1} are n-tile 0's
+    // columns, 2kq + 8 + {0, 1} n-tile 1's, i.e. the lane's keys 4kq + {0, 1} and 4kq + {2, 3}
+    const float4 vf4 = *reinterpret_cast<const float4 *>(sc + 16 + 4 * kq);
+    const float vf[4] = {vf4.x, vf4.y, vf4.z, vf4.w};
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            s[t][c] *= vf[2 * t + c];
+            s[t][2 + c] *= vf[2 * t + c];
+        }
+    uint32_t pa_[4];
+    pa_[0] = pack2<BF16>(s[0][0], s[0][1]);
+    pa_[1] = pack2<BF16>(s[0][2], s[0][3]);
+    pa_[2] = pack2<BF16>(s[1][0], s[1][1]);
+    pa_[3] = pack2<BF16>(s[1][2], s[1][3]);
+
+    // codes of keys past the context end may be NaN: zero them (code 0 is +0)
+    uint32_t vmask = 0xffffffffu;
+    if (j0 + 16 > ctx) {
+        const int valid = ctx - j0;
+        vmask = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            vmask |= (4 * kq + i < valid ? 0xffu : 0u) << (8 * i);
+    }
+    // O (16 x D) += P (16 x 16 keys) V (16 keys x D): lane (r, kq) of n-tile nd reads the codes of
+    // keys 4kq .. 4kq+3 in V's row d = 8nd + r
+#pragma unroll
+    for (int nd = 0; nd < NT; ++nd) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(vp + (8 * nd + r) * 16 + 4 * kq) & vmask;
+        mma16816<BF16>(o[nd], pa_, widen_e4m3x2<BF16>(w), widen_e4m3x2<BF16>(w >> 16));
+    }
+}
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -566,19 +707,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const RowsParams p)
 {
     using L = Fp8Smem<D>;
-    constexpr int CH = D / 8;       // 16-byte chunks of a 16-bit row
+    constexpr int STAGES = kFp8Stages;
     constexpr int KSTEPS = D / 16;  // k-steps of S = Q K^T
     constexpr int NT = D / 8;       // n-tiles of O
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *s_work = smem + L::kWorkOff;
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint8_t *s_ring = smem + L::kRingOff;
+    float *s_scale = reinterpret_cast<float *>(smem + L::kScaleOff);
     uint64_t *s_bar = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    int *s_count = reinterpret_cast<int *>(smem + L::kCountOff);
     int *s_issued = reinterpret_cast<int *>(smem + L::kIssuedOff);
     int32_t *s_pages = reinterpret_cast<int32_t *>(smem + L::kTableOff);
-    float *s_scale = reinterpret_cast<float *>(smem + L::kScaleOff);
-    int *s_count = reinterpret_cast<int *>(smem + L::kCountOff);
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -600,7 +740,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (row0 >= R)
         return;
     const int rows_here = min(kRowsPerCta, R - row0);
-    const int base = ctx - qb;
     const int lim_cta = ctx - qb + (row0 + rows_here - 1) / G;
     const int pages_need = lim_cta / 16 + 1;
     const int pages_ctx = (ctx + 15) / 16;
@@ -616,71 +755,121 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int mt = warp / KG, kg = warp % KG;
     const bool has_rows = mt * 16 < rows_here;
 
-    // ---- set-up ----------------------------------------------------------------------------
+    // ---- set-up: barriers and the first loads, page ids and scales, Q fragments -------------
     const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
-    auto issue = [&](int st) {  // one thread
-        const int slot = st % kFp8Stages;
-        uint8_t *kb = s_ring + slot * L::kStage8;
-        uint8_t *vb = kb + kPagesPerStage * L::kPage8;
-        const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&s_bar[slot], np * 2 * L::kPage8);
-        s_issued[slot] += 1;
-        for (int k = 0; k < np; ++k) {
-            const int y = (s_pages[st * kPagesPerStage + k] * p.H_kv + g) * 16;
-            tma_load_2d(kb + k * L::kPage8, &tmap_k, 0, y, &s_bar[slot]);
-            tma_load_2d(vb + k * L::kPage8, &tmap_v, 0, y, &s_bar[slot]);
-        }
-    };
-    if (tid == 0) {
-        for (int s = 0; s < kFp8Stages; ++s) {
-            mbar_init(&s_bar[s], 1);
-            s_issued[s] = 0;
-            s_count[s] = 0;
-        }
-        *s_abort = 0;
-        fence_barrier_init();
-        prefetch_tmap(&tmap_k);
-        prefetch_tmap(&tmap_v);
-    }
-    for (int i = tid; i < n_pages; i += kThreads) {
-        int pg = __ldg(table + page_lo + i);
+    auto checked = [&](int pg) -> int {
         if (pg < 0 || pg >= p.num_blocks) {
             set_status(p.status, PA_ERR_BOUNDS);
-            pg = static_cast<int>(p.num_blocks);  // past the pool: TMA fills zeros, scale 0
+            pg = static_cast<int>(p.num_blocks);  // past the pool: TMA fills zeros, scales 0
         }
+        return pg;
+    };
+    auto load_page = [&](int slot, int k, int pg) {
+        uint8_t *kb = s_ring + slot * L::kStage;
+        const int y = (pg * p.H_kv + g) * 16;
+        tma_load_2d(kb + k * L::kPage, &tmap_k, 0, y, &s_bar[slot]);
+        tma_load_2d(kb + (kPagesPerStage + k) * L::kPage, &tmap_v, 0, y, &s_bar[slot]);
+    };
+    auto issue = [&](int st) {  // one thread; the page ids from the shared-memory copy
+        const int slot = st % STAGES;
+        const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&s_bar[slot], np * 2 * L::kPage);
+        s_issued[slot] += 1;
+        for (int k = 0; k < np; ++k)
+            load_page(slot, k, s_pages[st * kPagesPerStage + k]);
+    };
+    if (warp == 0) {
+        // every stage of the ring goes out at once: lane i reads the id of page i from the table
+        // in global memory and issues that page's two boxes
+        static_assert(STAGES * kPagesPerStage <= 32, "one lane per page of the first stages");
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&s_bar[s], 1);
+                s_count[s] = 0;
+                s_issued[s] = 0;
+            }
+            *s_abort = 0;
+            fence_barrier_init();
+            prefetch_tmap(&tmap_k);
+            prefetch_tmap(&tmap_v);
+        }
+        const int first = min(STAGES, n_stages);
+        const bool mine = lane < first * kPagesPerStage && lane < n_pages;
+        const int pg = mine ? checked(__ldg(table + page_lo + lane)) : 0;
+        __syncwarp();
+        if (lane == 0) {
+            for (int st = 0; st < first; ++st) {
+                mbar_arrive_expect_tx(&s_bar[st], min(kPagesPerStage, n_pages - st * kPagesPerStage) * 2 * L::kPage);
+                s_issued[st] += 1;
+            }
+        }
+        __syncwarp();
+        if (mine)
+            load_page(lane / kPagesPerStage, lane % kPagesPerStage, pg);
+    }
+    // page ids and the scales of the split's keys; keys past the context end (or of a bad page)
+    // get scale 0
+    for (int i = tid; i < n_pages; i += kThreads) {
+        const int pg = checked(__ldg(table + page_lo + i));
         s_pages[i] = pg;
-    }
-    for (int i = tid; i < kRowsPerCta * CH; i += kThreads) {
-        const int r = i / CH, c = i % CH;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < rows_here) {
-            const int ridx = row0 + r;
-            const int64_t t = q0 + ridx / G;
-            const int h = g * G + ridx % G;
-            v = __ldg(reinterpret_cast<const uint4 *>(p.q) + (t * p.H_q + h) * CH + c);
+        const int keys_left = ctx - (page_lo + i) * 16;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+            const float4 *src =
+                reinterpret_cast<const float4 *>((kv ? p.v_scale : p.k_scale) + ((int64_t)pg * p.H_kv + g) * 16);
+            float4 *dst = reinterpret_cast<float4 *>(s_scale + (i * 2 + kv) * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (pg < p.num_blocks)
+                    v = __ldg(src + j);
+                v.x = 4 * j < keys_left ? v.x : 0.f;
+                v.y = 4 * j + 1 < keys_left ? v.y : 0.f;
+                v.z = 4 * j + 2 < keys_left ? v.z : 0.f;
+                v.w = 4 * j + 3 < keys_left ? v.w : 0.f;
+                dst[j] = v;
+            }
         }
-        *reinterpret_cast<uint4 *>(s_work + r * (D * 2) + ((c ^ (r & 7)) << 4)) = v;
     }
-    __syncthreads();
-    if (tid == 0)
-        for (int st = 0; st < min(kFp8Stages, n_stages); ++st)
-            issue(st);
+
+    // This thread holds rows ra = lane/4 and rb = ra + 8 of its warp's m-tile.
     const int ra = mt * 16 + (lane >> 2), rb = ra + 8;
     const int lim_a = ra < rows_here ? ctx - qb + (row0 + ra) / G : -1;
     const int lim_b = rb < rows_here ? ctx - qb + (row0 + rb) / G : -1;
     const int lim_warp = has_rows ? ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G : -1;
+    // Q fragments in the column order of rows_page_fp8: qa[ks][0] = Q[ra][c0 + 4ks + {0, 1}] and
+    // qa[ks][2] = Q[ra][c0 + 4ks + {2, 3}] with c0 = (lane % 4) * D/4; [1] and [3] likewise for rb.
     uint32_t qa[KSTEPS][4];
-    if (has_rows) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int rr = half ? rb : ra;
+        uint32_t w[D / 8];
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i)
+            w[i] = 0u;
+        if (has_rows && rr < rows_here) {
+            const int ridx = row0 + rr;
+            const int64_t t = q0 + ridx / G;
+            const int h = g * G + ridx % G;
+            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.q) +
+                                                               ((t * p.H_q + h) * D + (lane & 3) * (D / 4)) * 2);
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) {
+                const uint4 v = __ldg(src + i);
+                w[4 * i] = v.x;
+                w[4 * i + 1] = v.y;
+                w[4 * i + 2] = v.z;
+                w[4 * i + 3] = v.w;
+            }
+        }
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
-            const int mi = lane >> 3, rr = lane & 7;
-            const int r = mt * 16 + (mi & 1) * 8 + rr;
-            const int c = 2 * ks + (mi >> 1);
-            ldsm_x4(smem_u32(s_work + r * (D * 2) + ((c ^ (r & 7)) << 4)), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+            qa[ks][half] = w[2 * ks];
+            qa[ks][2 + half] = w[2 * ks + 1];
         }
     }
-    __syncthreads();  // Q is in registers: the work buffer takes the dequantised stages
+    __syncthreads();  // page ids, scales and barriers are set
     float o[NT][4];
 #pragma unroll
     for (int i = 0; i < NT; ++i)
@@ -688,121 +877,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
     const float sl2 = p.scale_log2;
 
-    // Convert row `row` of page `k` of stage `it` (kv 0 = K, 1 = V): the codes become their values in
-    // the 16-bit type (exact: every E4M3 value is an f16 and a bf16 value), in 8-byte pieces from a
-    // per-thread offset (spreading the banks), into the work buffer laid out like the 16-bit cache's;
-    // the row's scale goes to shared memory (0 past the context end, whose rows may hold anything).
-    auto convert_row = [&](int it, int kv, int k, int row) {
-        const int pidx = it * kPagesPerStage + k;
-        const int pg = s_pages[pidx];
-        const float *scales = kv ? p.v_scale : p.k_scale;
-        const bool live = pg < p.num_blocks && (page_lo + pidx) * 16 + row < ctx;
-        s_scale[(kv * kPagesPerStage + k) * 16 + row] =
-            live ? __ldg(scales + ((int64_t)pg * p.H_kv + g) * 16 + row) : 0.f;
-        const uint8_t *src = s_ring + (it % kFp8Stages) * L::kStage8 + kv * kPagesPerStage * L::kPage8 +
-                             k * L::kPage8 + row * D;
-        uint8_t *dst = s_work + kv * kPagesPerStage * L::kPage16 + k * L::kPage16;
-#pragma unroll
-        for (int i = 0; i < CH; ++i) {
-            const int ch = (i + row) % CH;
-            const uint2 codes = *reinterpret_cast<const uint2 *>(src + ch * 8);
-            uint32_t w[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t word = q < 2 ? codes.x : codes.y;
-                const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((word >> (16 * (q & 1))) & 0xffffu);
-                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-                if constexpr (BF16) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
-                    w[q] = pack2<true>(f.x, f.y);
-                } else {
-                    w[q] = static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
-                }
-            }
-            *reinterpret_cast<uint4 *>(dst + (ch >> 3) * 2048 + row * 128 + (((ch & 7) ^ (row & 7)) << 4)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    };
-
-    bool aborted = false;
-    if (MT == 1) {
-        // ---- one m-tile: warp w owns page w of every stage (converts it, then computes it), no CTA
-        // barrier; the last warp done with a stage refills it (as the 16-bit kernel) ------------
-        static_assert(kPagesPerStage == 4, "one page per warp");
-        for (int it = 0; it < n_stages; ++it) {
-            const int slot = it % kFp8Stages;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_bar[slot], (it / kFp8Stages) & 1));
-            if (!ok) {
-                *s_abort = 1;
-                set_status(p.status, PA_ERR_TIMEOUT);
-            }
-            const int k = warp, pidx = it * kPagesPerStage + k;
-            if (ok && pidx < n_pages) {
-                convert_row(it, lane >> 4, k, lane & 15);
-                __syncwarp();
-                const int j0 = (page_lo + pidx) * 16;
-                if (has_rows && j0 <= lim_warp)
-                    rows_page<D, BF16, true>(smem_u32(s_work + k * L::kPage16),
-                                             smem_u32(s_work + kPagesPerStage * L::kPage16 + k * L::kPage16), j0,
-                                             lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, ~0u, ~0u, base, ctx, sl2,
-                                             s_scale + k * 16, s_scale + (kPagesPerStage + k) * 16);
-            }
-            __syncwarp();
-            if (lane == 0 && atomicAdd(&s_count[slot], 1) == 3) {
-                s_count[slot] = 0;
-                if (it + kFp8Stages < n_stages && !*s_abort)
-                    issue(it + kFp8Stages);
-            }
-            if (*s_abort)
-                break;
-        }
-        __syncthreads();
-        aborted = *s_abort != 0;
-    } else {
-    // ---- several m-tiles: the CTA converts each stage together, then computes it -----------
+    // ---- main loop over stages (as the 16-bit kernel) ------------------------------------------
     for (int it = 0; it < n_stages; ++it) {
-        const int slot = it % kFp8Stages;
-        // every thread waits; the CTA agrees on the outcome, so no one is left at a barrier
-        const bool landed = __syncthreads_and(mbar_wait(&s_bar[slot], (it / kFp8Stages) & 1));
-        if (!landed) {
-            if (tid == 0)
-                set_status(p.status, PA_ERR_TIMEOUT);
-            aborted = true;
-            break;
+        const int slot = it % STAGES;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&s_bar[slot], (it / STAGES) & 1));
+        if (!ok) {
+            *s_abort = 1;
+            set_status(p.status, PA_ERR_TIMEOUT);
         }
-        // one row per thread: 2 (K, V) x 4 pages x 16 rows = 128 rows per stage
-        static_assert(2 * kPagesPerStage * 16 == kThreads, "one row per thread");
-        if (it * kPagesPerStage + (tid / 16) % kPagesPerStage < n_pages)
-            convert_row(it, tid / (kPagesPerStage * 16), (tid / 16) % kPagesPerStage, tid % 16);
-        __syncthreads();  // the stage is dequantised; its codes can be replaced
-        if (tid == 0 && it + kFp8Stages < n_stages)
-            issue(it + kFp8Stages);
-        if (has_rows) {
+        if (ok && has_rows) {
+            const uint8_t *st = s_ring + slot * L::kStage;
             for (int k = kg; k < kPagesPerStage; k += KG) {
                 const int pidx = it * kPagesPerStage + k;
                 if (pidx >= n_pages)
                     break;
                 const int j0 = (page_lo + pidx) * 16;
                 if (j0 > lim_warp)
-                    continue;
-                const uint32_t kbase = smem_u32(s_work + k * L::kPage16);
-                const uint32_t vbase = smem_u32(s_work + kPagesPerStage * L::kPage16 + k * L::kPage16);
-                rows_page<D, BF16, true>(kbase, vbase, j0, lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, ~0u, ~0u,
-                                         base, ctx, sl2, s_scale + k * 16, s_scale + (kPagesPerStage + k) * 16);
+                    continue;  // every row of this warp is causally masked on this page
+                rows_page_fp8<D, BF16>(st + k * L::kPage, st + (kPagesPerStage + k) * L::kPage, s_scale + pidx * 32,
+                                       j0, lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, ctx, sl2);
             }
         }
-        __syncthreads();  // everyone is done with the work buffer before the next stage overwrites it
+        // the last warp done with this slot refills it
+        __syncwarp();
+        if (lane == 0 && atomicAdd(&s_count[slot], 1) == 3) {
+            s_count[slot] = 0;
+            if (it + STAGES < n_stages && !*s_abort)
+                issue(it + STAGES);
+        }
+        if (*s_abort)
+            break;
     }
-    }
-    if (aborted) {
+    __syncthreads();
+    if (*s_abort) {
         // let the copies still in flight land (bounded) before the CTA releases its shared memory
         if (tid == 0)
-            for (int s = 0; s < kFp8Stages; ++s)
+            for (int s = 0; s < STAGES; ++s)
                 if (s_issued[s] > 0)
                     mbar_wait(&s_bar[s], (s_issued[s] - 1) & 1, kWaitTimeoutNs / 10);
         return;
     }
-    rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_work), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0,
+    rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_ring), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0,
                            g, split, n_splits, KG);
 }
 

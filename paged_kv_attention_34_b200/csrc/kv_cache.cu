@@ -156,11 +156,20 @@ __global__ void __launch_bounds__(256) kv_cache_write_fp8_kernel(const void *__r
                 code[i] = static_cast<uint8_t>(pr & 0xffu);
                 code[i + 1] = static_cast<uint8_t>(pr >> 8);
             }
-            uint8_t *dst = (kv ? value_cache : key_cache) + row * D + lane * VPL;
-            if constexpr (VPL == 4)
-                *reinterpret_cast<uint32_t *>(dst) = code[0] | (code[1] << 8) | (code[2] << 16) | (uint32_t(code[3]) << 24);
-            else
-                *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(code[0] | (code[1] << 8));
+            if (kv) {
+                // V codes are transposed within the block ([d][16 slots]): this row is a column
+                uint8_t *dst = value_cache + ((slot / 16) * H_kv + h) * 16 * D + (lane * VPL) * 16 + slot % 16;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i)
+                    dst[i * 16] = code[i];
+            } else {
+                uint8_t *dst = key_cache + row * D + lane * VPL;
+                if constexpr (VPL == 4)
+                    *reinterpret_cast<uint32_t *>(dst) =
+                        code[0] | (code[1] << 8) | (code[2] << 16) | (uint32_t(code[3]) << 24);
+                else
+                    *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(code[0] | (code[1] << 8));
+            }
             if (lane == 0)
                 (kv ? value_scale : key_scale)[row] = sc;
         }

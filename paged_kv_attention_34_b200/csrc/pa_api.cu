@@ -208,7 +208,7 @@ extern "C" int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t 
     if (B > 0 && T > 0) {
         if (!key_scale || !value_scale)
             return PA_ERR_ARG;
-        if (!aligned4(key_scale) || !aligned4(value_scale))
+        if (!aligned16(key_scale) || !aligned16(value_scale))
             return PA_ERR_ALIGN;
     }
     if (workspace_bytes < decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx))

@@ -137,7 +137,7 @@ def _fp8_device_cache(w):
     the device: (codes K, codes V, scales K, scales V)."""
     NB, H, _, d = w.key_cache.shape
     kc8 = torch.zeros((NB, H, 16, d), dtype=torch.uint8, device="cuda")
-    vc8 = torch.zeros_like(kc8)
+    vc8 = torch.zeros((NB, H, d, 16), dtype=torch.uint8, device="cuda")  # transposed within the block
     ks = torch.ones((NB, H, 16), dtype=torch.float32, device="cuda")
     vs = torch.ones_like(ks)
     rows_k = w.key_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous().cuda()
@@ -177,7 +177,7 @@ def test_fp8_cache_and_decode_small(idx):
     kc8, vc8, ks, vs = _fp8_device_cache(w)
     # the cache, byte for byte and scale for scale, as the oracle writes it
     NB, H = w.key_cache.shape[:2]
-    okc, ovc = np.zeros((NB, H, 16, d), np.uint8), np.zeros((NB, H, 16, d), np.uint8)
+    okc, ovc = np.zeros((NB, H, 16, d), np.uint8), np.zeros((NB, H, d, 16), np.uint8)
     oks, ovs = np.ones((NB, H, 16), np.float32), np.ones((NB, H, 16), np.float32)
     rows_k = w.key_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous()
     rows_v = w.value_cache.permute(0, 2, 1, 3).reshape(NB * 16, H, d).contiguous()
