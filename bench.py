@@ -357,6 +357,7 @@ def run_ours(args):
             "mixed_step": leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank),
             "tree_verify": leg_tree(args, stream, device, hbm_peak, rank),
             "fp8_cache": leg_fp8(args, stream, device, hbm_peak, rank),
+            "shared_prefix": leg_shared(args, stream, device, hbm_peak, rank),
             "block_swap": leg_swap(args, stream, device, rank),
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -531,7 +532,7 @@ def leg_fp8(args, stream, device, hbm_peak, rank):
     from paged_kv_attention_34_b200 import workloads as W
     from paged_kv_attention_34_b200.step import DeviceStep, attn_bytes
 
-    w = W.config2(seed=shard_seed(34_002, rank), fill="zero")
+    w = W.config2(seed=shard_seed(34_002, rank), fill="zero", B=args.batch)
     with torch.cuda.stream(stream):
         st = DeviceStep(w, device=device)
     call = st.calls[0]
@@ -567,7 +568,7 @@ def leg_fp8(args, stream, device, hbm_peak, rank):
     ctx_tokens = sum(int(c) for c in w.ctx_lens)
     b8 = b16 - ctx_tokens * 2 * H * d * 2 + ctx_tokens * 2 * H * (d + 4)
     gbs = b8 / (ms["fp8"] * 1e-3) / 1e9
-    return {"workload": "FP8 (E4M3) KV cache, 13B-shaped decode layer: B 64, 40/40 heads, d 128, fp16 Q, "
+    return {"workload": f"FP8 (E4M3) KV cache, 13B-shaped decode layer: B {args.batch}, 40/40 heads, d 128, fp16 Q, "
                         "ctx U[128,4096]",
             "decode_GB/s": round(gbs, 1), "frac": round(gbs / hbm_peak, 4), "bytes": b8,
             "decode_ms": round(ms["fp8"], 5), "decode_16bit_ms": round(ms["16bit"], 5),
@@ -610,6 +611,71 @@ def leg_tree(args, stream, device, hbm_peak, rank):
             "decode_GB/s": round(gbs, 1), "frac": round(gbs / hbm_peak, 4), "bytes": b,
             "decode_ms": round(per[1], 5), "per_call_ms": {"kv_cache_write": round(per[0], 5),
                                                            "paged_attn_decode_tree": round(per[1], 5)}}
+
+
+def leg_shared(args, stream, device, hbm_peak, rank):
+    """Shared-prefix decode: 64 requests in 4 groups of 16 sharing a 4096-token prompt (256 blocks),
+    own suffixes U[16, 512], on the 13B-shaped layer (40/40 heads, d 128, fp16); the shared-prefix
+    decode against the plain decode of the same tables.  Algorithmic bytes: every distinct key's K
+    and V (each prompt once), Q, O, tables.  Also the long-context GQA config (16 sequences sharing
+    2048 tokens of 32768) through both calls."""
+    import torch
+
+    from paged_kv_attention_34_b200 import paged_attn_decode, paged_attn_decode_shared_prefix
+    from paged_kv_attention_34_b200 import shared_prefix_workspace_bytes
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import DeviceStep, attn_bytes
+
+    def run(w, starts, P):
+        with torch.cuda.stream(stream):
+            st = DeviceStep(w, device=device)
+            st.copy_blocks()
+            st.write()
+        call = st.calls[0]
+        gs = torch.tensor(starts, dtype=torch.int32, device=device)
+        pb = torch.tensor(P, dtype=torch.int32, device=device)
+        max_gt = max(sum(w.q_lens[starts[v]:starts[v + 1]]) for v in range(len(P)))
+        ws = torch.zeros(shared_prefix_workspace_bytes(w.T, w.B, w.H_q, w.H_kv, w.d, call.max_ctx, len(P), max(P),
+                                                       max_gt), dtype=torch.uint8, device=device)
+        out2 = torch.empty_like(call.out)
+
+        def shared():
+            paged_attn_decode_shared_prefix(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, gs, pb,
+                                            call.max_ctx, max(P), max_gt, w.scale, out=out2, workspace=ws)
+
+        def plain():
+            paged_attn_decode(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, call.max_ctx,
+                              w.scale, out=call.out, workspace=call.ws)
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                shared()
+                plain()
+        torch.cuda.synchronize()
+        _, per = time_calls([shared, plain], max(args.steps, 5), stream)
+        if any(st.statuses()) or read_status_of(ws):
+            raise RuntimeError("device status")
+        dev = (out2.float() - call.out.float()).abs().max().item()
+        b = attn_bytes(w)
+        return {"shared_ms": round(per[0], 5), "plain_ms": round(per[1], 5),
+                "speedup_vs_plain": round(per[1] / per[0], 3), "unique_bytes": b,
+                "unique_GB/s": round(b / (per[0] * 1e-3) / 1e9, 1),
+                "frac": round(b / (per[0] * 1e-3) / 1e9 / hbm_peak, 4), "max_abs_diff_vs_plain": round(dev, 6)}
+
+    w = W.shared_prefix_batch(seed=shard_seed(34_106, rank), fill="zero")
+    res = {"workload": "shared-prefix decode: 64 requests = 4 prompts (4096 tokens) x 16, own suffixes U[16,512], "
+                       "40/40 heads, d 128, fp16",
+           **run(w, w.notes["group_start"], w.notes["prefix_blocks"])}
+    w4 = W.config4(seed=shard_seed(34_004, rank), fill="zero")
+    res["gqa_config"] = {"workload": W.CONFIG_NAMES[4],
+                         **run(w4, [0, w4.B], [w4.notes["shared_tokens"] // 16])}
+    return res
+
+
+def read_status_of(ws):
+    from paged_kv_attention_34_b200 import read_status
+
+    return read_status(ws)
 
 
 def leg_swap(args, stream, device, rank, n_blocks=512):
@@ -784,6 +850,8 @@ def run_one_leg(args):
         res = leg_tree(args, stream, device, hbm, 0)
     elif args.only == "fp8":
         res = leg_fp8(args, stream, device, hbm, 0)
+    elif args.only == "shared":
+        res = leg_shared(args, stream, device, hbm, 0)
     else:
         res = leg_mixed(args, stream, device, hbm, bf16, 0)
     print(json.dumps({"leg": args.only, **res}), flush=True)
@@ -798,7 +866,7 @@ def main(argv=None):
     ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
-    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap", "tree", "fp8"], default=None,
+    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap", "tree", "fp8", "shared"], default=None,
                     help="run one leg alone and print its JSON object (profiling runs)")
     ap.add_argument("--batch", type=int, default=64,
                     help="sequences of the headline decode workload (64 = the 13B-shaped layer; smaller for profiling)")

@@ -182,6 +182,56 @@ int pa_paged_attn_decode_tree(void *out, const void *q, const void *key_cache, c
                               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Shared-prefix decode -- pa_paged_attn_decode for batches in which groups of
+ * sequences share the blocks of a common prompt prefix (page-level sharing of
+ * one prompt prefix by several requests: iopencloud "大模型推理加速技术全景"
+ * section 3.2; refcounted shared blocks on the PagedAttention section of the
+ * fourth page).  The shared blocks are read once per (group, KV head) for all
+ * the group's query rows, instead of once per sequence; each sequence's own
+ * keys (after the prefix) are read as in pa_paged_attn_decode, and the two
+ * partial softmaxes are merged by log-sum-exp.  The result is the attention of
+ * pa_paged_attn_decode over the same tables (the pages only say that blocks
+ * are shared; reading them once and merging is this library's reading of it).
+ *
+ * pa_shared_prefix_workspace_bytes -- workspace for these sizes (status word,
+ * sequence order, per-sequence prefix lengths, the prefix partials and the
+ * sequences' own split partials).  Pure host function; 0 for invalid sizes.
+ */
+size_t pa_shared_prefix_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx, int n_groups,
+                                        int max_prefix_blocks, int max_group_tokens);
+
+/*
+ * pa_paged_attn_decode_shared_prefix -- sizes, layouts and errors of
+ * pa_paged_attn_decode, plus:
+ *   group_start        int32 [n_groups + 1], device: group v is the sequences
+ *                      group_start[v] .. group_start[v+1]-1 (consecutive runs,
+ *                      group_start[0] = 0, group_start[n_groups] = B; a
+ *                      sequence sharing nothing is a group of its own with 0
+ *                      prefix blocks)
+ *   prefix_blocks      int32 [n_groups], device: the first prefix_blocks[v]
+ *                      entries of the block tables of group v are the shared
+ *                      blocks (whole blocks, before every new token)
+ *   max_prefix_blocks  host bound on prefix_blocks (<= max_blocks_per_seq)
+ *   max_group_tokens   host bound on the new tokens of one group (sizes the
+ *                      prefix pass: rows = tokens x H_q/H_kv per KV head)
+ * A sequence whose table does not start with its group leader's prefix
+ * blocks, or whose new tokens start inside the prefix, is computed over its
+ * own table alone (same result, no sharing).  Groups that are not a partition
+ * of the sequences into consecutive runs, prefix_blocks outside
+ * 0..max_blocks_per_seq, or a group with more new tokens than
+ * max_group_tokens set PA_ERR_ARG in the status word (every sequence is then
+ * computed alone).  Launches: a one-CTA plan kernel, the sequence order, the
+ * attention kernel (prefix CTAs first, then the sequences'), the merge.
+ */
+int pa_paged_attn_decode_shared_prefix(void *out, const void *q, const void *key_cache, const void *value_cache,
+                                       int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
+                                       const int32_t *cu_seqlens_q, const int32_t *context_lens, int B, int max_ctx,
+                                       int64_t T, int H_q, int H_kv, int d, float scale, pa_dtype dtype,
+                                       const int32_t *group_start, const int32_t *prefix_blocks, int n_groups,
+                                       int max_prefix_blocks, int max_group_tokens, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/*
  * FP8 (E4M3) KV cache -- an 8-bit cache with one float scale per stored row
  * (the FP8 KV-cache option of the serving page; FP8 with scaling on the
  * interview Q&A page): half the HBM bytes of a 16-bit cache per key.

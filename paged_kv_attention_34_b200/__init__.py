@@ -70,6 +70,11 @@ def _declare(L):
     L.pa_paged_attn_decode_tree.restype = I
     L.pa_paged_attn_decode_tree.argtypes = [P, P, P, P, I64, P, I, P, P, P, I, I, I64, I, I, I, c.c_float, I, P, SZ,
                                             P]
+    L.pa_shared_prefix_workspace_bytes.restype = SZ
+    L.pa_shared_prefix_workspace_bytes.argtypes = [I64, I, I, I, I, I, I, I, I]
+    L.pa_paged_attn_decode_shared_prefix.restype = I
+    L.pa_paged_attn_decode_shared_prefix.argtypes = [P, P, P, P, I64, P, I, P, P, I, I, I64, I, I, I, c.c_float, I,
+                                                     P, P, I, I, I, P, SZ, P]
     L.pa_prefill_workspace_bytes.restype = SZ
     L.pa_prefill_workspace_bytes.argtypes = [I, I, I, I, I]
     L.pa_paged_attn_prefill.restype = I
@@ -348,6 +353,42 @@ def paged_attn_decode_tree(q, key_cache, value_cache, block_tables, cu_seqlens_q
     )
     _check(rc, "pa_paged_attn_decode_tree")
     paged_attn_decode_tree.last_workspace = ws
+    return out
+
+
+def shared_prefix_workspace_bytes(T: int, B: int, H_q: int, H_kv: int, d: int, max_ctx: int, n_groups: int,
+                                  max_prefix_blocks: int, max_group_tokens: int) -> int:
+    n = lib().pa_shared_prefix_workspace_bytes(T, B, H_q, H_kv, d, max_ctx, n_groups, max_prefix_blocks,
+                                               max_group_tokens)
+    if n == 0:
+        raise ValueError("invalid sizes for pa_shared_prefix_workspace_bytes")
+    return int(n)
+
+
+def paged_attn_decode_shared_prefix(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens,
+                                    group_start, prefix_blocks, max_ctx: int, max_prefix_blocks: int,
+                                    max_group_tokens: int, scale: float, out=None, workspace=None, stream=None):
+    """Decode where groups of consecutive sequences share the first prefix_blocks[v] blocks of their
+    tables (group v = sequences group_start[v] .. group_start[v+1]-1, int32 device tensors): the
+    shared blocks are read once per group, then merged with each sequence's own keys; returns out."""
+    out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
+                                               context_lens, out)
+    _cuda(group_start, "group_start", torch.int32, 1)
+    _cuda(prefix_blocks, "prefix_blocks", torch.int32, 1)
+    n_groups = prefix_blocks.shape[0]
+    if group_start.shape[0] != n_groups + 1:
+        raise ValueError(f"group_start must be int32 [{n_groups + 1}]")
+    nbytes = shared_prefix_workspace_bytes(T, B, H_q, H_kv, d, max_ctx, n_groups, max_prefix_blocks,
+                                           max_group_tokens)
+    ws = _workspace(workspace, nbytes, q.device)
+    rc = lib().pa_paged_attn_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
+        _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_ctx), T, H_q, H_kv, d, float(scale), _dtype_code(q),
+        _ptr(group_start), _ptr(prefix_blocks), n_groups, int(max_prefix_blocks), int(max_group_tokens), _ptr(ws),
+        ws.numel(), ctypes.c_void_p(_stream(stream)),
+    )
+    _check(rc, "pa_paged_attn_decode_shared_prefix")
+    paged_attn_decode_shared_prefix.last_workspace = ws
     return out
 
 

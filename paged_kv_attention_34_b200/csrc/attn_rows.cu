@@ -37,6 +37,13 @@ constexpr int kPagesPerStage = 4;
 constexpr int kMaxTablePages = 256;  // page ids of one split (split_pages <= this)
 constexpr int kThreads = 128;
 
+// What the rows of a decode CTA see: causal (the new tokens in order), a tree-verification mask
+// over the new tokens, or the shared-prefix pass (causal sequence CTAs plus prefix CTAs whose
+// rows see every prefix key).
+constexpr int kModeCausal = 0;
+constexpr int kModeTree = 1;
+constexpr int kModeShared = 2;
+
 struct RowsParams {
     const void *q;
     void *out;
@@ -49,6 +56,13 @@ struct RowsParams {
     const int32_t *tree;   // [T] tree verification: bit j = the token sees new token j; nullptr = causal
     const float *k_scale;  // FP8 cache: [num_blocks][H_kv][16] scale of every stored K row
     const float *v_scale;  // ... and V row
+    // shared-prefix decode
+    const int32_t *group_start;    // [n_groups + 1] the sequences of group v: [group_start[v], group_start[v+1])
+    const int32_t *prefix_blocks;  // [n_groups] blocks shared by group v at the head of its tables
+    int32_t *seq_prefix;           // [B] prefix blocks of each sequence's group (set by the plan kernel)
+    int n_groups;
+    int prefix_split_pages;  // pages per split of a prefix
+    int prefix_slots;        // workspace slots of the prefix splits (the sequences' own splits follow)
     int32_t *status;
     int64_t num_blocks;
     int64_t T;
@@ -233,12 +247,12 @@ __device__ __forceinline__ void rows_page(uint32_t kbase, uint32_t vbase, int j0
 
 // Epilogue of a rows CTA: merge the warps of each m-tile (several warps on different pages of the
 // same rows, like splits) through shared memory `e_o` (at least RowsEpi<D>::kBytes), normalise,
-// and store the rows: straight to `out` when the sequence has one split, else the normalised
-// partial and its log2-sum-exp to the workspace.
+// and store the rows: straight to `out` when `final_out`, else the normalised partial and its
+// log2-sum-exp to workspace slot `slot`.
 template <int D, bool BF16>
 __device__ __forceinline__ void rows_epilogue(float *e_o, const RowsParams &p, const float (&o)[D / 8][4], float m_a,
                                               float m_b, float l_a, float l_b, bool has_rows, int rows_here,
-                                              int row0, int q0, int g, int split, int n_splits, int KG)
+                                              int row0, int q0, int g, int slot, bool final_out, int KG)
 {
     constexpr int NT = D / 8;
     constexpr int kEpiStride = RowsEpi<D>::kStride;
@@ -266,7 +280,6 @@ __device__ __forceinline__ void rows_epilogue(float *e_o, const RowsParams &p, c
         }
     }
     __syncthreads();
-    const bool final_out = n_splits == 1;
     for (int i = tid; i < rows_here * (D / 4); i += kThreads) {
         const int r = i / (D / 4), c4 = i % (D / 4);
         const int mtr = r >> 4, lr = r & 15;
@@ -295,7 +308,7 @@ __device__ __forceinline__ void rows_epilogue(float *e_o, const RowsParams &p, c
             store4<BF16>(static_cast<uint8_t *>(p.out) + (orow * D + c4 * 4) * 2, acc.x * inv, acc.y * inv,
                          acc.z * inv, acc.w * inv);
         } else {
-            const int64_t prow = (int64_t)split * p.T * p.H_q + orow;
+            const int64_t prow = (int64_t)slot * p.T * p.H_q + orow;
             *reinterpret_cast<float4 *>(p.ws_o + prow * D + c4 * 4) =
                 make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
             if (c4 == 0)
@@ -304,7 +317,7 @@ __device__ __forceinline__ void rows_epilogue(float *e_o, const RowsParams &p, c
     }
 }
 
-template <int D, bool BF16, int STAGES, bool TREE>
+template <int D, bool BF16, int STAGES, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     pa_attn_rows_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const RowsParams p)
@@ -328,33 +341,80 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // ---- which (sequence, KV head, row group, split) --------------------------------
-    const int b = __ldg(p.order + blockIdx.z);
+    // Shared-prefix mode: grid z < n_groups is the prefix of group z -- every token of the
+    // group's sequences against the group's shared blocks, read once for all of them (no mask:
+    // the prefix precedes every new token); z >= n_groups is one sequence's own keys, from the
+    // first block after its group's prefix.
     const int split = blockIdx.x;
     const int g = blockIdx.y / p.n_rg, rg = blockIdx.y % p.n_rg;
-    const int q0 = __ldg(p.cu_seqlens + b), q1 = __ldg(p.cu_seqlens + b + 1);
-    const int qb = q1 - q0, ctx = __ldg(p.context_lens + b);
-    if (!seq_ok(qb, ctx, p, q1)) {
-        if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
-            set_status(p.status, PA_ERR_SEQ);
-        return;
+    int q0, q1, ctx, page_base = 0, sp = p.split_pages, slot0 = 0;
+    bool prefix_cta = false;
+    const int32_t *table;
+    if constexpr (MODE == kModeShared) {
+        const int sp_pre = p.prefix_split_pages;
+        if (static_cast<int>(blockIdx.z) < p.n_groups) {
+            // the group's arrays were checked by the plan kernel (status); clamp them here so a
+            // bad call stays inside its buffers
+            const int v = blockIdx.z;
+            const int s0 = min(max(__ldg(p.group_start + v), 0), p.B);
+            const int s1 = min(max(__ldg(p.group_start + v + 1), s0), p.B);
+            if (s0 >= s1)
+                return;
+            q0 = __ldg(p.cu_seqlens + s0);
+            q1 = max(__ldg(p.cu_seqlens + s1), q0);
+            ctx = min(max(__ldg(p.prefix_blocks + v), 0), min(p.max_blocks, p.prefix_slots * sp_pre)) * 16;
+            table = p.block_tables + (int64_t)s0 * p.max_blocks;
+            sp = p.prefix_split_pages;
+            prefix_cta = true;
+            if (q0 < 0 || q1 > p.T || ctx == 0)
+                return;
+        } else {
+            const int b = __ldg(p.order + (blockIdx.z - p.n_groups));
+            q0 = __ldg(p.cu_seqlens + b);
+            q1 = __ldg(p.cu_seqlens + b + 1);
+            ctx = __ldg(p.context_lens + b);
+            if (!seq_ok(q1 - q0, ctx, p, q1)) {
+                if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+                    set_status(p.status, PA_ERR_SEQ);
+                return;
+            }
+            table = p.block_tables + (int64_t)b * p.max_blocks;
+            page_base = min(max(__ldg(p.seq_prefix + b), 0), (ctx - (q1 - q0)) / 16);
+            slot0 = p.prefix_slots;
+        }
+    } else {
+        const int b = __ldg(p.order + blockIdx.z);
+        q0 = __ldg(p.cu_seqlens + b);
+        q1 = __ldg(p.cu_seqlens + b + 1);
+        ctx = __ldg(p.context_lens + b);
+        if (!seq_ok(q1 - q0, ctx, p, q1)) {
+            if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+                set_status(p.status, PA_ERR_SEQ);
+            return;
+        }
+        table = p.block_tables + (int64_t)b * p.max_blocks;
     }
+    const int qb = q1 - q0;
     const int G = p.G;
     const int R = G * qb;
     const int row0 = rg * kRowsPerCta;
     if (row0 >= R)
         return;
     const int rows_here = min(kRowsPerCta, R - row0);
-    constexpr bool tree = TREE;  // p.tree is set exactly when TREE is
+    constexpr bool tree = MODE == kModeTree;  // p.tree is set exactly in this mode
     const int base = ctx - qb;  // first new token of the sequence
-    // last key any row here sees (a tree row may see every new token)
-    const int lim_cta = tree ? ctx - 1 : ctx - qb + (row0 + rows_here - 1) / G;
+    // rows that see every key: tree rows (their mask decides among the new tokens) and the rows
+    // of a shared prefix
+    const bool see_all = tree || prefix_cta;
+    // last key any row here sees
+    const int lim_cta = see_all ? ctx - 1 : ctx - qb + (row0 + rows_here - 1) / G;
     const int pages_need = lim_cta / 16 + 1;
     const int pages_ctx = (ctx + 15) / 16;
-    const int n_splits = (pages_ctx + p.split_pages - 1) / p.split_pages;
+    const int n_splits = (pages_ctx - page_base + sp - 1) / sp;
     if (split >= n_splits)
         return;
-    const int page_lo = split * p.split_pages;
-    const int page_hi = min(page_lo + p.split_pages, pages_need);
+    const int page_lo = page_base + split * sp;
+    const int page_hi = min(page_lo + sp, pages_need);
     const int n_pages = max(0, page_hi - page_lo);
     const int n_stages = (n_pages + kPagesPerStage - 1) / kPagesPerStage;
 
@@ -365,7 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_rows = mt * 16 < rows_here;
 
     // ---- set-up: barriers and the first loads, page ids, Q tile ---------------------------
-    const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
     auto checked = [&](int pg) -> int {
         if (pg < 0 || pg >= p.num_blocks) {
             set_status(p.status, PA_ERR_BOUNDS);
@@ -453,12 +512,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // causal rows see keys up to their own position with every bit set; tree rows see up to the
     // last key with their own mask.
     const int ra = mt * 16 + (lane >> 2), rb = ra + 8;
-    const int lim_a = ra < rows_here ? (tree ? ctx - 1 : ctx - qb + (row0 + ra) / G) : -1;
-    const int lim_b = rb < rows_here ? (tree ? ctx - 1 : ctx - qb + (row0 + rb) / G) : -1;
+    const int lim_a = ra < rows_here ? (see_all ? ctx - 1 : ctx - qb + (row0 + ra) / G) : -1;
+    const int lim_b = rb < rows_here ? (see_all ? ctx - 1 : ctx - qb + (row0 + rb) / G) : -1;
     const uint32_t bits_a = tree && ra < rows_here ? static_cast<uint32_t>(__ldg(p.tree + q0 + (row0 + ra) / G)) : ~0u;
     const uint32_t bits_b = tree && rb < rows_here ? static_cast<uint32_t>(__ldg(p.tree + q0 + (row0 + rb) / G)) : ~0u;
     const int lim_warp =
-        has_rows ? (tree ? ctx - 1 : ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G) : -1;
+        has_rows ? (see_all ? ctx - 1 : ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G) : -1;
 
     uint32_t qa[KSTEPS][4];
     if (has_rows) {
@@ -501,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     continue;  // every row of this warp is causally masked on this page
                 const uint32_t kbase = smem_u32(kst + k * L::kPageBytes);
                 const uint32_t vbase = smem_u32(vst + k * L::kPageBytes);
-                rows_page<D, BF16, false, TREE>(kbase, vbase, j0, lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, bits_a, bits_b,
+                rows_page<D, BF16, false, MODE == kModeTree>(kbase, vbase, j0, lane, qa, o, m_a, m_b, l_a, l_b, lim_a, lim_b, bits_a, bits_b,
                                    base, ctx, sl2);
             }
         }
@@ -526,8 +585,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- epilogue ---------------------------------------------------------------------------
+    // a shared-prefix pass always leaves partials for the merge: prefix splits in slots
+    // [0, prefix_slots), a sequence's own splits after them
     rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_stage), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0, g,
-                           split, n_splits, KG);
+                           slot0 + split, MODE != kModeShared && n_splits == 1, KG);
 }
 
 // ---- FP8 (E4M3) cache -----------------------------------------------------------------------
@@ -918,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_ring), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0,
-                           g, split, n_splits, KG);
+                           g, split, n_splits == 1, KG);
 }
 
 // One warp per (token, query head) row of a sequence with more than one split:
@@ -937,19 +998,29 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
     if (!seq_ok(q1 - q0, ctx, p, q1))
         return;
     const int pages_ctx = (ctx + 15) / 16;
-    const int ns = (pages_ctx + p.split_pages - 1) / p.split_pages;
-    if (ns <= 1)
+    // shared-prefix decode: the prefix's splits sit in slots [0, nps), the sequence's own splits
+    // from prefix_slots on, and every row goes through the merge
+    const bool shared = p.seq_prefix != nullptr;
+    int nps = 0, own_lo = 0, own_slot = 0;
+    if (shared) {
+        own_lo = min(max(__ldg(p.seq_prefix + b), 0), (ctx - (q1 - q0)) / 16);
+        nps = (own_lo + p.prefix_split_pages - 1) / p.prefix_split_pages;
+        own_slot = p.prefix_slots;
+    }
+    const int ns = nps + (pages_ctx - own_lo + p.split_pages - 1) / p.split_pages;
+    if (!shared && ns <= 1)
         return;
+    auto slot = [&](int s) -> int64_t { return s < nps ? s : own_slot + (s - nps); };
     const int64_t stride = p.T * p.H_q;
     float M = -INFINITY;
     for (int s = lane; s < ns; s += 32)
-        M = fmaxf(M, p.ws_lse[s * stride + row]);
+        M = fmaxf(M, p.ws_lse[slot(s) * stride + row]);
 #pragma unroll
     for (int o = 16; o; o >>= 1)
         M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Z = 0.f;
     for (int s = lane; s < ns; s += 32) {
-        const float l = p.ws_lse[s * stride + row];
+        const float l = p.ws_lse[slot(s) * stride + row];
         Z += l == -INFINITY ? 0.f : fast_exp2(l - M);
     }
 #pragma unroll
@@ -960,11 +1031,11 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
     if (lane < LANES) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s = 0; s < ns; ++s) {
-            const float l = p.ws_lse[s * stride + row];
+            const float l = p.ws_lse[slot(s) * stride + row];
             if (l == -INFINITY)
                 continue;
             const float w = fast_exp2(l - M) * invZ;
-            const float4 v = *reinterpret_cast<const float4 *>(p.ws_o + (s * stride + row) * D + lane * 4);
+            const float4 v = *reinterpret_cast<const float4 *>(p.ws_o + (slot(s) * stride + row) * D + lane * 4);
             acc.x += w * v.x;
             acc.y += w * v.y;
             acc.z += w * v.z;
@@ -974,16 +1045,70 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
     }
 }
 
+// Shared-prefix decode, before the rows kernel: seq_prefix[b] = the prefix blocks of sequence b's
+// group, or 0 where the shared pass must not be used for b -- its table does not start with the
+// group leader's prefix blocks, or the prefix reaches its new tokens; such a sequence is computed
+// over its own table alone (the result is the same).  Malformed groups (not a partition of the
+// sequences into consecutive runs, a prefix outside the table, more new tokens than the rows
+// planned for a group, a prefix longer than the planned bound) set PA_ERR_ARG and turn every
+// sequence into the unshared case.
+__global__ void __launch_bounds__(1024) pa_shared_plan_kernel(const RowsParams p)
+{
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0)
+        bad = __ldg(p.group_start) != 0 || __ldg(p.group_start + p.n_groups) != p.B;
+    __syncthreads();
+    for (int v = tid; v < p.n_groups; v += blockDim.x) {
+        const int s0 = __ldg(p.group_start + v), s1 = __ldg(p.group_start + v + 1);
+        const int P = __ldg(p.prefix_blocks + v);
+        if (s0 < 0 || s1 < s0 || s1 > p.B || P < 0 || P > p.max_blocks || P > p.prefix_slots * p.prefix_split_pages)
+            bad = 1;
+        else if (s1 > s0 && (int64_t)(__ldg(p.cu_seqlens + s1) - __ldg(p.cu_seqlens + s0)) * p.G >
+                                (int64_t)p.n_rg * kRowsPerCta)
+            bad = 1;
+    }
+    __syncthreads();
+    if (bad) {
+        if (tid == 0)
+            set_status(p.status, PA_ERR_ARG);
+        for (int b = tid; b < p.B; b += blockDim.x)
+            p.seq_prefix[b] = 0;
+        return;
+    }
+    for (int b = tid; b < p.B; b += blockDim.x) {
+        // b's group: the last v with group_start[v] <= b (groups may be empty)
+        int lo = 0, hi = p.n_groups - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (__ldg(p.group_start + mid) <= b)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        const int s0 = __ldg(p.group_start + lo);
+        const int P = __ldg(p.prefix_blocks + lo);
+        const int q_b = __ldg(p.cu_seqlens + b + 1) - __ldg(p.cu_seqlens + b);
+        int use = (int64_t)P * 16 <= (int64_t)__ldg(p.context_lens + b) - q_b ? P : 0;
+        const int32_t *mine = p.block_tables + (int64_t)b * p.max_blocks;
+        const int32_t *lead = p.block_tables + (int64_t)s0 * p.max_blocks;
+        for (int i = 0; i < use; ++i)
+            if (__ldg(mine + i) != __ldg(lead + i))
+                use = 0;
+        p.seq_prefix[b] = use;
+    }
+}
+
 // ---- host side ------------------------------------------------------------------------------
 
 constexpr int kStages = 3;
 
-template <int D, bool BF16, bool TREE>
+template <int D, bool BF16, int MODE>
 static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
                        cudaStream_t stream)
 {
     using L = RowsSmem<D, kStages>;
-    auto kern = pa_attn_rows_kernel<D, BF16, kStages, TREE>;
+    auto kern = pa_attn_rows_kernel<D, BF16, kStages, MODE>;
     static uint64_t configured = 0;  // one bit per device, per template instance
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
@@ -1113,6 +1238,36 @@ size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
     return bytes;
 }
 
+SharedPlan shared_plan(int B, int H_q, int H_kv, int d, int max_ctx, int n_groups, int max_prefix_blocks,
+                       int max_group_tokens)
+{
+    SharedPlan sp;
+    sp.own = decode_plan(B, H_q, H_kv, d, max_ctx);
+    const int G = H_q / H_kv;
+    const int rg_prefix = max(1, (max_group_tokens * G + kRowsPerCta - 1) / kRowsPerCta);
+    sp.row_groups = max(sp.own.row_groups, rg_prefix);
+    // prefix splits: about one wave of prefix CTAs (two per SM), at least 16 pages each
+    const int64_t units = (int64_t)max(n_groups, 1) * H_kv * rg_prefix;
+    const int64_t slots = (int64_t)sm_count() * 2;
+    const int64_t want = (slots + units - 1) / units;  // >= 1
+    int64_t len = max_prefix_blocks > 0 ? (max_prefix_blocks + want - 1) / want : 16;
+    len = (len + kPagesPerStage - 1) / kPagesPerStage * kPagesPerStage;
+    len = len < 16 ? 16 : (len > kMaxTablePages ? kMaxTablePages : len);
+    sp.prefix_split_pages = static_cast<int>(len);
+    sp.prefix_slots = max_prefix_blocks > 0 ? static_cast<int>((max_prefix_blocks + len - 1) / len) : 0;
+    return sp;
+}
+
+// Workspace of the shared-prefix decode: status, sequence order, seq_prefix, then the partials of
+// the prefix splits and of the sequences' own splits (every row is merged).
+size_t shared_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx, int n_groups,
+                              int max_prefix_blocks, int max_group_tokens)
+{
+    const SharedPlan sp = shared_plan(B, H_q, H_kv, d, max_ctx, n_groups, max_prefix_blocks, max_group_tokens);
+    const size_t rows = static_cast<size_t>(sp.prefix_slots + sp.own.max_splits) * static_cast<size_t>(T) * H_q;
+    return PA_STATUS_BYTES + 2 * seq_order_bytes(B) + rows * d * sizeof(float) + rows * sizeof(float) + 256;
+}
+
 template <int D, bool BF16>
 static int run(const AttnArgs &a)
 {
@@ -1145,6 +1300,40 @@ static int run(const AttnArgs &a)
     rp.tree = a.tree_mask;
     rp.k_scale = a.key_scale;
     rp.v_scale = a.value_scale;
+    if (a.group_start) {
+        const SharedPlan sp = shared_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx, a.n_groups, a.max_prefix_blocks,
+                                          a.max_group_tokens);
+        rp.n_rg = sp.row_groups;
+        rp.split_pages = sp.own.split_pages;
+        rp.prefix_split_pages = sp.prefix_split_pages;
+        rp.prefix_slots = sp.prefix_slots;
+        rp.n_groups = a.n_groups;
+        rp.group_start = a.group_start;
+        rp.prefix_blocks = a.prefix_blocks;
+        uint8_t *ws = static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES;
+        int32_t *order = reinterpret_cast<int32_t *>(ws);
+        int32_t *seq_prefix = reinterpret_cast<int32_t *>(ws + seq_order_bytes(a.B));
+        rp.order = order;
+        rp.seq_prefix = seq_prefix;
+        const size_t rows = static_cast<size_t>(sp.prefix_slots + sp.own.max_splits) * static_cast<size_t>(a.T) * a.H_q;
+        uint8_t *part = ws + 2 * seq_order_bytes(a.B);
+        rp.ws_o = reinterpret_cast<float *>(part);
+        rp.ws_lse = reinterpret_cast<float *>(part + rows * D * sizeof(float));
+        const int64_t z = (int64_t)a.n_groups + a.B;
+        if (z > 65535 || (int64_t)a.H_kv * sp.row_groups > 65535)
+            return PA_ERR_UNSUPPORTED;
+        dim3 grid(max(sp.own.max_splits, sp.prefix_slots), a.H_kv * sp.row_groups, static_cast<unsigned>(z));
+        pa_shared_plan_kernel<<<1, 1024, 0, a.stream>>>(rp);
+        count_launch();
+        rc = cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+        if (rc == PA_OK)
+            rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
+        if (rc == PA_OK)
+            rc = launch_rows<D, BF16, kModeShared>(rp, tk, tv, grid, a.stream);
+        if (rc == PA_OK)
+            rc = launch_merge<D, BF16>(rp, a.stream);
+        return rc;
+    }
     {
         const DecodePlan pl = decode_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx);
         rp.n_rg = pl.row_groups;
@@ -1163,8 +1352,8 @@ static int run(const AttnArgs &a)
         rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
         if (rc == PA_OK)
             rc = fp8       ? launch_rows_fp8<D, BF16>(rp, tk, tv, grid, a.stream)
-                 : rp.tree ? launch_rows<D, BF16, true>(rp, tk, tv, grid, a.stream)
-                           : launch_rows<D, BF16, false>(rp, tk, tv, grid, a.stream);
+                 : rp.tree ? launch_rows<D, BF16, kModeTree>(rp, tk, tv, grid, a.stream)
+                           : launch_rows<D, BF16, kModeCausal>(rp, tk, tv, grid, a.stream);
         if (rc == PA_OK && pl.max_splits > 1)
             rc = launch_merge<D, BF16>(rp, a.stream);
         return rc;

@@ -192,6 +192,54 @@ extern "C" int pa_paged_attn_decode_tree(void *out, const void *q, const void *k
     return launch_decode(a);
 }
 
+extern "C" size_t pa_shared_prefix_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx,
+                                                    int n_groups, int max_prefix_blocks, int max_group_tokens)
+{
+    if (T < 0 || B < 0 || H_q < 1 || H_kv < 1 || (d != 64 && d != 128) || max_ctx < 0 || H_q % H_kv ||
+        n_groups < 1 || max_prefix_blocks < 0 || max_group_tokens < 0)
+        return 0;
+    return shared_workspace_bytes(T, B, H_q, H_kv, d, max_ctx, n_groups, max_prefix_blocks, max_group_tokens);
+}
+
+extern "C" int pa_paged_attn_decode_shared_prefix(void *out, const void *q, const void *key_cache,
+                                                  const void *value_cache, int64_t num_blocks,
+                                                  const int32_t *block_tables, int max_blocks_per_seq,
+                                                  const int32_t *cu_seqlens_q, const int32_t *context_lens, int B,
+                                                  int max_ctx, int64_t T, int H_q, int H_kv, int d, float scale,
+                                                  pa_dtype dtype, const int32_t *group_start,
+                                                  const int32_t *prefix_blocks, int n_groups, int max_prefix_blocks,
+                                                  int max_group_tokens, void *workspace, size_t workspace_bytes,
+                                                  void *stream)
+{
+    AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
+               context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
+               static_cast<cudaStream_t>(stream)};
+    a.group_start = group_start;
+    a.prefix_blocks = prefix_blocks;
+    a.n_groups = n_groups;
+    a.max_prefix_blocks = max_prefix_blocks;
+    a.max_group_tokens = max_group_tokens;
+    int rc = check_attn(a, true);
+    if (rc != PA_OK)
+        return rc;
+    if (n_groups < 1 || n_groups > B + 1 || max_prefix_blocks < 0 || max_prefix_blocks > max_blocks_per_seq ||
+        max_group_tokens < 0 || (int64_t)max_group_tokens > T)
+        return PA_ERR_ARG;
+    if (B > 0 && T > 0) {
+        if (!group_start || !prefix_blocks)
+            return PA_ERR_ARG;
+        if (!aligned4(group_start) || !aligned4(prefix_blocks))
+            return PA_ERR_ALIGN;
+    }
+    if (workspace_bytes <
+        shared_workspace_bytes(T, B, H_q, H_kv, d, max_ctx, n_groups, max_prefix_blocks, max_group_tokens))
+        return PA_ERR_WORKSPACE;
+    rc = reset_status(workspace, a.stream);
+    if (rc != PA_OK || B == 0 || T == 0)
+        return rc;
+    return launch_decode(a);
+}
+
 extern "C" int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t *key_cache,
                                         const uint8_t *value_cache, const float *key_scale, const float *value_scale,
                                         int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,

@@ -58,6 +58,13 @@ struct AttnArgs {
     const int32_t *tree_mask = nullptr;  // decode only: per-token visibility bits of the new tokens
     const float *key_scale = nullptr;    // FP8 cache (decode only): per-row scales, else nullptr
     const float *value_scale = nullptr;
+    // shared-prefix decode (decode only): groups of consecutive sequences whose tables start
+    // with the same prefix_blocks[v] blocks; nullptr = none
+    const int32_t *group_start = nullptr;    // [n_groups + 1] device
+    const int32_t *prefix_blocks = nullptr;  // [n_groups] device
+    int n_groups = 0;
+    int max_prefix_blocks = 0;  // host bound on prefix_blocks[v]
+    int max_group_tokens = 0;   // host bound on the new tokens of one group
 };
 
 // Split-KV decode plan: pages per split and the number of splits.
@@ -68,6 +75,18 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx);
 size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx);
+
+// Shared-prefix decode plan: the decode plan of the sequences' own keys plus the prefix pass.
+struct SharedPlan {
+    DecodePlan own;
+    int row_groups;          // per KV head: covers a sequence's rows and a group's rows
+    int prefix_split_pages;  // pages per split of a prefix
+    int prefix_slots;        // workspace slots of the prefix splits
+};
+SharedPlan shared_plan(int B, int H_q, int H_kv, int d, int max_ctx, int n_groups, int max_prefix_blocks,
+                       int max_group_tokens);
+size_t shared_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx, int n_groups,
+                              int max_prefix_blocks, int max_group_tokens);
 
 // Sequence order by decreasing page count (one CTA, on `stream`): order[r] = the sequence of rank r.
 // The workspace holds it right after the status area, seq_order_bytes(B) bytes.

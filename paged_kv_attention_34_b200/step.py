@@ -129,7 +129,13 @@ def attn_bytes(w: Workload, call_kind: Optional[str] = None) -> int:
             total += ctx * 2 * w.H_kv * w.d * esz  # K and V rows
             total += w.q_lens[b] * w.H_q * w.d * esz * 2  # Q in, O out
             total += ((ctx + 15) // 16) * 4 + 4 + 4  # table entries, ctx, cu
-        if shared_tokens:
+        if "group_start" in w.notes:  # groups of sequences sharing their first prefix_blocks[v] blocks
+            st, P = w.notes["group_start"], w.notes["prefix_blocks"]
+            for v in range(len(P)):
+                n = len(range(max(st[v], c.seq_lo), min(st[v + 1], c.seq_hi)))
+                if n > 1:
+                    total -= (n - 1) * P[v] * 16 * 2 * w.H_kv * w.d * esz
+        elif shared_tokens:
             n = c.seq_hi - c.seq_lo
             total -= (n - 1) * shared_tokens * 2 * w.H_kv * w.d * esz
     return total

@@ -505,6 +505,46 @@ def tree_verify(seed: int = 34_105, fill: str = "nan", B: int = 64, q: int = 8) 
     )
 
 
+def share_prefixes(w: Workload, group_sizes: List[int], prefix_blocks: List[int]) -> Workload:
+    """Make consecutive runs of sequences share prompt-prefix blocks, in place: group v is the next
+    group_sizes[v] sequences, and the first prefix_blocks[v] entries of each member's table are
+    pointed at its first sequence's blocks (whose contents then stand for the shared prompt; the
+    members' own former prefix blocks stay in the pool unused).  A prefix must end before every
+    member's new tokens.  Returns w with notes group_start / prefix_blocks."""
+    assert sum(group_sizes) == w.B and len(group_sizes) == len(prefix_blocks)
+    starts = [0]
+    for n in group_sizes:
+        starts.append(starts[-1] + n)
+    for v, P in enumerate(prefix_blocks):
+        lead = starts[v]
+        for b in range(lead, starts[v + 1]):
+            assert P * BLOCK_SIZE <= w.ctx_lens[b] - w.q_lens[b], (b, P)
+            if b != lead:
+                w.block_tables[b, :P] = w.block_tables[lead, :P]
+    w.shared_blocks = sum(P for v, P in enumerate(prefix_blocks) if group_sizes[v] > 1)
+    w.notes = {**w.notes, "group_start": starts, "prefix_blocks": list(prefix_blocks)}
+    return w
+
+
+def shared_prefix_batch(seed: int = 34_106, fill: str = "nan", B: int = 64, n_groups: int = 4,
+                        prefix_tokens: int = 4096, suffix=(16, 512), q_max: int = 1, H_q: int = 40, H_kv: int = 40,
+                        d: int = 128, dtype: torch.dtype = F16) -> Workload:
+    """Decode batch of requests that share prompts: B sequences in n_groups consecutive groups of
+    (nearly) equal size; each group shares a prefix_tokens-token prompt (whole blocks), and each
+    sequence has its own suffix of U[suffix] tokens after it, the last q_b of them new this step.
+    Defaults: the 13B-shaped decode layer (40/40 heads, d 128, fp16) with 4 prompts of 4096 tokens
+    and 16 requests each."""
+    assert prefix_tokens % BLOCK_SIZE == 0
+    g = _gen(seed + 1_000_000)
+    q_lens = [int(x) for x in torch.randint(1, q_max + 1, (B,), generator=g)]
+    suf = _uniform_int(g, suffix[0], suffix[1], B)
+    ctx = [prefix_tokens + max(sb, qb) for sb, qb in zip(suf, q_lens)]
+    w = build_workload("shared_prefix", q_lens=q_lens, ctx_lens=ctx, H_q=H_q, H_kv=H_kv, d=d, dtype=dtype,
+                       seed=seed, calls=[AttnCall("decode", 0, B)], fill=fill)
+    sizes = [B // n_groups + (1 if v < B % n_groups else 0) for v in range(n_groups)]
+    return share_prefixes(w, sizes, [prefix_tokens // BLOCK_SIZE] * n_groups)
+
+
 def make_config(idx: int, **kw) -> Workload:
     return {1: config1, 2: config2, 3: config3, 4: config4, 5: config5}[idx](**kw)
 

@@ -329,6 +329,44 @@ def pin_tree_verify(L):
     assert np.abs(got - sdpa_reference(w, tree_mask=solo)).max() < 1e-12
 
 
+def pin_shared_prefix(L):
+    """Groups of sequences sharing prompt-prefix blocks: the oracle over the aliased tables == fp64
+    SDPA on the gathered keys, and for every row the attention over the group's shared keys merged
+    by log-sum-exp with the attention over the sequence's own keys is the whole -- the decomposition
+    that the shared-prefix decode computes (the prefix once per group, then the merge)."""
+    w = W.shared_prefix_batch(seed=61, B=5, n_groups=2, prefix_tokens=48, suffix=(3, 40), q_max=3, H_q=4, H_kv=2,
+                              d=16)
+    starts, P = w.notes["group_start"], w.notes["prefix_blocks"]
+    for v in range(len(P)):
+        for b in range(starts[v], starts[v + 1]):
+            assert torch.equal(w.block_tables[b, : P[v]], w.block_tables[starts[v], : P[v]])
+    got, kc, vc = oracle_step(w, L)
+    assert np.abs(got - sdpa_reference(w)).max() < 1e-12
+    G = w.H_q // w.H_kv
+    kd = torch.from_numpy(kc.view(np.float16)).double()
+    vd = torch.from_numpy(vc.view(np.float16)).double()
+    cu = w.cu_seqlens_q.tolist()
+    for b in range(w.B):
+        v = max(i for i in range(len(P)) if starts[i] <= b)
+        n_pre = P[v] * 16
+        ctx, qb = w.ctx_lens[b], w.q_lens[b]
+        K = gather_contiguous(kd, w.block_tables[b], ctx)
+        V = gather_contiguous(vd, w.block_tables[b], ctx)
+        for i in range(qb):
+            t = cu[b] + i
+            last = ctx - qb + i
+            for h in range(w.H_q):
+                q = w.q[t, h].double().numpy()
+                kh, vh = K[h // G].numpy(), V[h // G].numpy()
+                parts, lses = [], []
+                for lo, hi in ((0, n_pre), (n_pre, last + 1)):
+                    o, l_ = oracle.attention_partial(q, kh, vh, lo, hi, w.scale, L=L)
+                    parts.append(o)
+                    lses.append(l_)
+                merged, _ = oracle.lse_merge(np.stack(parts), np.array(lses), L=L)
+                assert np.abs(merged - got[t, h]).max() < 1e-13, (b, i, h)
+
+
 def pin_dense_three_pass(L):
     """Paged oracle == the standard three-pass attention on contiguous data."""
     w = W.random_workload(11, B=2, q_max=5, ctx_max=37, H_kv=2, G=2, d=16, dtype=W.F16, kind="decode")
@@ -588,6 +626,7 @@ ALL_PINS = [
     pin_fp8_attention,
     pin_sdpa_library,
     pin_tree_verify,
+    pin_shared_prefix,
     pin_dense_three_pass,
     pin_block_permutation,
     pin_paged_equals_contiguous,

@@ -143,6 +143,25 @@ def test_prefill_rejects_bad_args(L):
     assert call(wsb=8) == -4
 
 
+def test_shared_prefix_rejects_bad_args(L):
+    f = L.pa_paged_attn_decode_shared_prefix
+
+    def call(n_groups=2, max_pb=4, max_gt=2, gs=_fake(), pb=_fake(), wsb=1 << 20, B=2, T=2):
+        return f(_fake(), _fake(), _fake(), _fake(), 16, _fake(), 8, _fake(), _fake(), B, 100, T, 8, 2, 128, 0.1, 1,
+                 gs, pb, n_groups, max_pb, max_gt, _fake(), wsb, None)
+
+    n0 = pa.launch_count()
+    assert call(n_groups=0) == -1
+    assert call(max_pb=9) == -1     # more prefix blocks than a table holds
+    assert call(max_gt=3) == -1     # more new tokens in a group than in the batch
+    assert call(gs=None) == -1
+    assert call(pb=None) == -1
+    assert call(gs=_fake(0x10002)) == -3
+    assert call(wsb=64) == -4
+    assert call(n_groups=4) == -1   # more groups than B + 1
+    assert pa.launch_count() == n0
+
+
 def test_workspace_queries(L):
     # one split needs the status word and the sequence order (B int32 in 256-byte units);
     # long contexts need partials
@@ -156,6 +175,11 @@ def test_workspace_queries(L):
     assert pa.decode_workspace_bytes(16, 16, 64, 8, 128, 65536) >= big
     assert L.pa_decode_workspace_bytes(1, 1, 6, 4, 128, 10) == 0  # invalid GQA ratio
     assert pa.prefill_workspace_bytes(8, 40, 40, 128, 2048) >= pa.PA_STATUS_BYTES
+    # shared-prefix decode: status, order and per-sequence prefix areas, then every row's partials
+    sh = pa.shared_prefix_workspace_bytes(64, 64, 40, 40, 128, 4608, 4, 256, 16)
+    assert sh >= pa.PA_STATUS_BYTES + 2 * 256 + 64 * 40 * 129 * 4
+    assert pa.shared_prefix_workspace_bytes(64, 64, 40, 40, 128, 4608, 4, 512, 16) >= sh  # longer prefixes
+    assert L.pa_shared_prefix_workspace_bytes(64, 64, 40, 40, 128, 4608, 0, 256, 16) == 0  # no group
 
 
 def test_binding_refuses_cpu_tensors():

@@ -508,3 +508,109 @@ def test_prefill_schedules_heaviest_work_first():
     keys = np.array([min(tiles(int(e)), 4095) for e in order])
     assert np.all(np.diff(keys) <= 0)
     assert keys[0] == max(tiles(e) for e in range(n_pairs * B))
+
+
+# ---- shared-prefix decode -------------------------------------------------------------------
+
+def _groups_of(w):
+    """(group_start, prefix_blocks, max_prefix_blocks, max_group_tokens) from share_prefixes' notes."""
+    starts, P = w.notes["group_start"], w.notes["prefix_blocks"]
+    tokens = [sum(w.q_lens[starts[v] : starts[v + 1]]) for v in range(len(P))]
+    return (torch.tensor(starts, dtype=torch.int32, device="cuda"), torch.tensor(P, dtype=torch.int32, device="cuda"),
+            max(P), max(tokens))
+
+
+def _shared_run(w, groups=None):
+    """Block copies and cache write, then the shared-prefix decode; returns (output, status word)."""
+    gs, pb, max_pb, max_gt = groups if groups is not None else _groups_of(w)
+    st = DeviceStep(w)
+    st.copy_blocks()
+    st.write()
+    call = st.calls[0]
+    n_ws = pa.shared_prefix_workspace_bytes(call.q.shape[0], w.B, w.H_q, w.H_kv, w.d, call.max_ctx, pb.shape[0],
+                                            max_pb, max_gt)
+    ws = torch.zeros(n_ws, dtype=torch.uint8, device="cuda")
+    out = pa.paged_attn_decode_shared_prefix(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, gs, pb,
+                                             call.max_ctx, max_pb, max_gt, w.scale, out=call.out, workspace=ws)
+    torch.cuda.synchronize()
+    assert st.statuses()[0] == 0
+    return out, pa.read_status(ws)
+
+
+# (B, n_groups, prefix tokens, own suffix range, q_max, H_q, H_kv, d, dtype)
+SHARED_CASES = [
+    (8, 3, 64, (1, 40), 3, 8, 2, 64, W.F16),          # ragged verify rows, GQA 4
+    (6, 2, 256, (16, 300), 1, 4, 4, 128, W.BF16),     # MHA decode
+    (16, 1, 2048, (1, 100), 2, 32, 8, 128, W.BF16),   # one group, long prefix (several prefix splits), 2 row groups
+    (20, 4, 512, (1, 2000), 1, 16, 2, 128, W.F16),    # long own keys: several splits of their own
+    (3, 3, 32, (5, 9), 4, 2, 1, 64, W.BF16),          # one sequence per group
+]
+
+
+def _shared_id(c):
+    return "B{}g{}p{}q{}h{}/{}d{}{}".format(c[0], c[1], c[2], c[4], c[5], c[6], c[7], "bf16" if c[8] == W.BF16 else "f16")
+
+
+@pytest.mark.parametrize("idx", range(len(SHARED_CASES)), ids=lambda i: _shared_id(SHARED_CASES[i]))
+def test_shared_prefix_small(idx):
+    B, n_groups, pre, suf, q_max, H_q, H_kv, d, dt = SHARED_CASES[idx]
+    w = W.shared_prefix_batch(seed=700 + idx, B=B, n_groups=n_groups, prefix_tokens=pre, suffix=suf, q_max=q_max,
+                              H_q=H_q, H_kv=H_kv, d=d, dtype=dt)
+    out, status = _shared_run(w)
+    assert status == 0
+    ref, _, _ = oracle_step(w, oracle.lib())
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref).max()
+    assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
+
+
+def test_shared_prefix_falls_back_where_tables_differ():
+    # one group over sequences that share nothing (each owns its 4 prefix blocks): every member's
+    # table differs from the leader's, so each is computed over its own table (same result, status OK)
+    w = W.shared_prefix_batch(seed=71, B=5, n_groups=5, prefix_tokens=64, suffix=(1, 60), q_max=2, H_q=4, H_kv=2,
+                              d=64, dtype=W.F16)
+    groups = (torch.tensor([0, w.B], dtype=torch.int32, device="cuda"),
+              torch.tensor([4], dtype=torch.int32, device="cuda"), 4, w.T)
+    out, status = _shared_run(w, groups)
+    assert status == 0
+    ref, _, _ = oracle_step(w, oracle.lib())
+    assert np.abs(out.double().cpu().numpy() - ref).max() <= TOL[w.dtype]
+
+
+def test_shared_prefix_rejects_malformed_groups_and_stays_correct():
+    w = W.shared_prefix_batch(seed=72, B=6, n_groups=2, prefix_tokens=64, suffix=(4, 50), q_max=2, H_q=4, H_kv=2,
+                              d=64, dtype=W.BF16)
+    _, _, max_pb, max_gt = _groups_of(w)
+    bad = (torch.tensor([0, 4, 2, 6], dtype=torch.int32, device="cuda"),  # not increasing
+           torch.tensor([4, 4, 4], dtype=torch.int32, device="cuda"), max_pb, max_gt)
+    out, status = _shared_run(w, bad)
+    assert status == -1  # PA_ERR_ARG: every sequence computed alone
+    ref, _, _ = oracle_step(w, oracle.lib())
+    assert np.abs(out.double().cpu().numpy() - ref).max() <= TOL[w.dtype]
+
+
+def test_shared_prefix_4_prompts_13b_layer_sampled():
+    # 64 requests in 4 groups sharing a 4096-token prompt, own suffixes U[16, 512]; 40/40 heads, d 128
+    w = W.shared_prefix_batch()
+    out, status = _shared_run(w)
+    assert status == 0
+    rows = sample_rows(w, 256, seed=8)
+    ref, _, _ = oracle_step(w, oracle.lib(), rows=rows)
+    got = out.double().cpu().numpy().reshape(w.T * w.H_q, w.d)[rows]
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= TOL[w.dtype]
+
+
+def test_shared_prefix_on_the_gqa_shared_prefix_config_sampled():
+    # the long-context GQA decode (16 sequences sharing 128 blocks = 2048 tokens, one block copy)
+    w = W.config4()
+    n_shared = w.notes["shared_tokens"] // 16
+    groups = (torch.tensor([0, w.B], dtype=torch.int32, device="cuda"),
+              torch.tensor([n_shared], dtype=torch.int32, device="cuda"), n_shared, w.T)
+    out, status = _shared_run(w, groups)
+    assert status == 0
+    rows = sample_rows(w, 256, seed=9)
+    ref, _, _ = oracle_step(w, oracle.lib(), rows=rows)
+    got = out.double().cpu().numpy().reshape(w.T * w.H_q, w.d)[rows]
+    assert np.abs(got - ref).max() <= TOL[w.dtype]
