@@ -607,14 +607,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // the last warp done with a stage.
 constexpr int kFp8Stages = 4;
 
-template <int D>
+// NARROW: no scale table (each warp loads its page's scales into registers one stage ahead), so
+// three CTAs fit on an SM.
+template <int D, bool NARROW>
 struct Fp8Smem {
     static constexpr int kPage = 16 * D;                       // codes of one page of K or of V
     static constexpr int kStage = 2 * kPagesPerStage * kPage;  // K pages then V pages
     static_assert(RowsEpi<D>::kBytes <= kFp8Stages * kStage, "the epilogue reuses the ring");
     static constexpr int kRingOff = 0;
     static constexpr int kScaleOff = kFp8Stages * kStage;          // [page of the split][K, V][16 keys]
-    static constexpr int kBarOff = kScaleOff + kMaxTablePages * 2 * 16 * 4;
+    static constexpr int kBarOff = kScaleOff + (NARROW ? 0 : kMaxTablePages * 2 * 16 * 4);
     static constexpr int kCountOff = kBarOff + 8 * kFp8Stages;     // warps done with each stage
     static constexpr int kIssuedOff = kCountOff + 4 * kFp8Stages;  // loads issued into each stage
     static constexpr int kTableOff = kIssuedOff + 4 * kFp8Stages;
@@ -762,12 +764,198 @@ __device__ __forceinline__ void rows_page_fp8(const uint8_t *kp, const uint8_t *
     }
 }
 
+// FP8 page step with the keys on the MMA's M side, for CTAs of at most 8 query rows (single-token
+// decode with G <= 8), where the 16-row m-tile of rows_page_fp8 would be mostly padding:
+// S^T = K Q^T (m = 16 keys, n = 8 rows, k = 16 columns of d) and O^T += V^T P^T (m = 16 columns
+// of d, n = 8 rows, k = 16 keys) -- half the MMAs per page, and V^T's operand is one 32-bit word
+// of a transposed V row.  A-row g of S^T is key 2g and A-row g + 8 key 2g + 1; the d order of the
+// k-steps is rows_page_fp8's.  kf, vf: the K and V scales of keys 2g, 2g + 1 (0 past the context
+// end).  State per lane (g = lane/4, t = lane%4): rows 2t and 2t + 1, their
+// running max m (uniform over the 8 lanes of a t) and partial sum l (summed over g at the end),
+// and O^T rows d = 16 mt + g, 16 mt + g + 8.
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ void narrow_page_fp8(const uint8_t *kp, const uint8_t *vp, float2 kf, float2 vf, int j0, int lane,
+                                                const uint32_t (&qb)[D / 16][2], float (&o)[D / 16][4], float (&m)[2],
+                                                float (&l)[2], const int (&lim)[2], int ctx, float sl2)
+{
+    constexpr int KSTEPS = D / 16;  // k-steps of S^T
+    constexpr int MT = D / 16;      // m-tiles of O^T
+    constexpr int SPAN = D / 4;     // code bytes of a key row per lane quad
+    const int g = lane >> 2, t = lane & 3;
+
+    // S^T (16 keys x 8 rows); the k-steps alternate between two accumulators
+    float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+        const uint8_t *r0 = kp + (2 * g) * D + t * SPAN;
+        const uint8_t *r1 = r0 + D;
+        uint32_t w0[SPAN / 4], w1[SPAN / 4];
+#pragma unroll
+        for (int i = 0; i < SPAN / 16; ++i) {
+            const uint4 a = *reinterpret_cast<const uint4 *>(r0 + i * 16);
+            const uint4 b = *reinterpret_cast<const uint4 *>(r1 + i * 16);
+            w0[4 * i] = a.x;
+            w0[4 * i + 1] = a.y;
+            w0[4 * i + 2] = a.z;
+            w0[4 * i + 3] = a.w;
+            w1[4 * i] = b.x;
+            w1[4 * i + 1] = b.y;
+            w1[4 * i + 2] = b.z;
+            w1[4 * i + 3] = b.w;
+        }
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ++ks) {
+            const uint32_t a[4] = {widen_e4m3x2<BF16>(w0[ks]), widen_e4m3x2<BF16>(w1[ks]),
+                                   widen_e4m3x2<BF16>(w0[ks] >> 16), widen_e4m3x2<BF16>(w1[ks] >> 16)};
+            if (ks & 1)
+                mma16816<BF16>(s2, a, qb[ks][0], qb[ks][1]);
+            else
+                mma16816<BF16>(s, a, qb[ks][0], qb[ks][1]);
+        }
+    }
+    // x0 = (key 2g, row 2t), x1 = (2g, 2t+1), x2 = (2g+1, 2t), x3 = (2g+1, 2t+1): key scales,
+    // mask, log2 units; max over the page's keys (this lane's two, then the 8 lanes of its t)
+    const int key0 = j0 + 2 * g, key1 = key0 + 1;
+    const float x0 = key0 <= lim[0] ? (s[0] + s2[0]) * (sl2 * kf.x) : -INFINITY;
+    const float x1 = key0 <= lim[1] ? (s[1] + s2[1]) * (sl2 * kf.x) : -INFINITY;
+    const float x2 = key1 <= lim[0] ? (s[2] + s2[2]) * (sl2 * kf.y) : -INFINITY;
+    const float x3 = key1 <= lim[1] ? (s[3] + s2[3]) * (sl2 * kf.y) : -INFINITY;
+    float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+    const float b0 = mn0 == -INFINITY ? 0.f : mn0;
+    const float b1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float al0 = fast_exp2(m[0] - b0), al1 = fast_exp2(m[1] - b1);
+    m[0] = mn0;
+    m[1] = mn1;
+    const float p0 = fast_exp2(x0 - b0), p1 = fast_exp2(x1 - b1);
+    const float p2 = fast_exp2(x2 - b0), p3 = fast_exp2(x3 - b1);
+    l[0] = l[0] * al0 + p0 + p2;
+    l[1] = l[1] * al1 + p1 + p3;
+    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            o[mt][0] *= al0;
+            o[mt][1] *= al1;
+            o[mt][2] *= al0;
+            o[mt][3] *= al1;
+        }
+    }
+    // value scales into P, packed per row as (key 2g, key 2g + 1); P^T's operand for lane (g, t)
+    // is row g's keys 4t, 4t + 1 (held by lane (2t, g/2)) and 4t + 2, 4t + 3 (lane (2t + 1, g/2))
+    const uint32_t pk0 = pack2<BF16>(p0 * vf.x, p2 * vf.y);  // row 2t
+    const uint32_t pk1 = pack2<BF16>(p1 * vf.x, p3 * vf.y);  // row 2t + 1
+    const int src = (2 * t) * 4 + (g >> 1);
+    const uint32_t u0 = __shfl_sync(0xffffffffu, pk0, src), u1 = __shfl_sync(0xffffffffu, pk1, src);
+    const uint32_t v0 = __shfl_sync(0xffffffffu, pk0, src + 4), v1 = __shfl_sync(0xffffffffu, pk1, src + 4);
+    const uint32_t pb0 = (g & 1) ? u1 : u0, pb1 = (g & 1) ? v1 : v0;
+
+    // codes of keys past the context end may be NaN: zero them (code 0 is +0)
+    uint32_t vmask = 0xffffffffu;
+    if (j0 + 16 > ctx) {
+        const int valid = ctx - j0;
+        vmask = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            vmask |= (4 * t + i < valid ? 0xffu : 0u) << (8 * i);
+    }
+    // O^T += V^T P^T: m-tile mt holds d = 16 mt + g (A rows g) and 16 mt + g + 8; the word of V
+    // row d at bytes 4t .. 4t + 3 is keys 4t .. 4t + 3 = MMA k indices 2t, 2t+1, 2t+8, 2t+9
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const uint32_t wa = *reinterpret_cast<const uint32_t *>(vp + (16 * mt + g) * 16 + 4 * t) & vmask;
+        const uint32_t wb = *reinterpret_cast<const uint32_t *>(vp + (16 * mt + g + 8) * 16 + 4 * t) & vmask;
+        const uint32_t a[4] = {widen_e4m3x2<BF16>(wa), widen_e4m3x2<BF16>(wb), widen_e4m3x2<BF16>(wa >> 16),
+                               widen_e4m3x2<BF16>(wb >> 16)};
+        mma16816<BF16>(o[mt], a, pb0, pb1);
+    }
+}
+
+// Epilogue of a narrow FP8 CTA: the four warps (different pages of the same <= 8 rows) merge
+// through shared memory `e` (at least NarrowEpi<D>::kBytes) like splits; then as rows_epilogue.
+template <int D>
+struct NarrowEpi {
+    static constexpr int kStride = D + 4;  // floats per (warp, row) of O
+    static constexpr int kBytes = (4 * 8 * kStride + 2 * 4 * 8) * 4;
+};
+
+template <int D, bool BF16>
+__device__ __forceinline__ void narrow_epilogue(float *e, const RowsParams &p, const float (&o)[D / 16][4],
+                                                const float (&m)[2], float (&l)[2], int rows_here, int row0, int q0,
+                                                int g, int slot, bool final_out)
+{
+    constexpr int S = NarrowEpi<D>::kStride;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gr = lane >> 2, t = lane & 3;
+    const int G = p.G;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        l[0] += __shfl_xor_sync(0xffffffffu, l[0], off);
+        l[1] += __shfl_xor_sync(0xffffffffu, l[1], off);
+    }
+    float *e_o = e;                   // [4 warps][8 rows][S]
+    float *e_m = e + 4 * 8 * S;       // [4][8]
+    float *e_l = e_m + 32;            // [4][8]
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+        const int d0 = 16 * mt + gr;
+        e_o[(warp * 8 + 2 * t) * S + d0] = o[mt][0];
+        e_o[(warp * 8 + 2 * t + 1) * S + d0] = o[mt][1];
+        e_o[(warp * 8 + 2 * t) * S + d0 + 8] = o[mt][2];
+        e_o[(warp * 8 + 2 * t + 1) * S + d0 + 8] = o[mt][3];
+    }
+    if (gr == 0) {
+        e_m[warp * 8 + 2 * t] = m[0];
+        e_m[warp * 8 + 2 * t + 1] = m[1];
+        e_l[warp * 8 + 2 * t] = l[0];
+        e_l[warp * 8 + 2 * t + 1] = l[1];
+    }
+    __syncthreads();
+    for (int i = tid; i < rows_here * (D / 4); i += kThreads) {
+        const int r = i / (D / 4), c4 = i % (D / 4);
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            M = fmaxf(M, e_m[w * 8 + r]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float Lsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float mw = e_m[w * 8 + r];
+            const float wt = mw == -INFINITY ? 0.f : fast_exp2(mw - M);
+            Lsum += wt * e_l[w * 8 + r];
+            const float4 v = *reinterpret_cast<const float4 *>(e_o + (w * 8 + r) * S + c4 * 4);
+            acc.x += wt * v.x;
+            acc.y += wt * v.y;
+            acc.z += wt * v.z;
+            acc.w += wt * v.w;
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        const int ridx = row0 + r;
+        const int64_t tok = q0 + ridx / G;
+        const int h = g * G + ridx % G;
+        const int64_t orow = tok * p.H_q + h;
+        if (final_out) {
+            store4<BF16>(static_cast<uint8_t *>(p.out) + (orow * D + c4 * 4) * 2, acc.x * inv, acc.y * inv,
+                         acc.z * inv, acc.w * inv);
+        } else {
+            const int64_t prow = (int64_t)slot * p.T * p.H_q + orow;
+            *reinterpret_cast<float4 *>(p.ws_o + prow * D + c4 * 4) =
+                make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+            if (c4 == 0)
+                p.ws_lse[prow] = Lsum > 0.f ? M + log2f(Lsum) : -INFINITY;
+        }
+    }
+}
+
+template <int D, bool BF16, bool NARROW>
+__global__ void __launch_bounds__(kThreads, NARROW ? 3 : 1)
     pa_attn_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                             const RowsParams p)
 {
-    using L = Fp8Smem<D>;
+    using L = Fp8Smem<D, NARROW>;
     constexpr int STAGES = kFp8Stages;
     constexpr int KSTEPS = D / 16;  // k-steps of S = Q K^T
     constexpr int NT = D / 8;       // n-tiles of O
@@ -815,6 +1003,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int KG = 4 / MT;
     const int mt = warp / KG, kg = warp % KG;
     const bool has_rows = mt * 16 < rows_here;
+    if (NARROW && rows_here > 8) {  // the host picks this variant for single-token decode with G <= 8 only
+        if (tid == 0)
+            set_status(p.status, PA_ERR_UNSUPPORTED);
+        return;
+    }
 
     // ---- set-up: barriers and the first loads, page ids and scales, Q fragments -------------
     const int32_t *table = p.block_tables + (int64_t)b * p.max_blocks;
@@ -874,6 +1067,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i < n_pages; i += kThreads) {
         const int pg = checked(__ldg(table + page_lo + i));
         s_pages[i] = pg;
+        if constexpr (NARROW)
+            continue;
         const int keys_left = ctx - (page_lo + i) * 16;
 #pragma unroll
         for (int kv = 0; kv < 2; ++kv) {
@@ -901,10 +1096,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lim_warp = has_rows ? ctx - qb + (row0 + min(mt * 16 + 15, rows_here - 1)) / G : -1;
     // Q fragments in the column order of rows_page_fp8: qa[ks][0] = Q[ra][c0 + 4ks + {0, 1}] and
     // qa[ks][2] = Q[ra][c0 + 4ks + {2, 3}] with c0 = (lane % 4) * D/4; [1] and [3] likewise for rb.
-    uint32_t qa[KSTEPS][4];
+    // The narrow variant's B operand (Q^T) is the same two words of row lane/4: qn[ks][0], [1].
+    uint32_t qa[KSTEPS][4], qn[KSTEPS][2];
+    int lim_n[2];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const int rr = half ? rb : ra;
+    for (int i = 0; i < 2; ++i) {
+        const int r = 2 * (lane & 3) + i;
+        lim_n[i] = r < rows_here ? ctx - qb + (row0 + r) / G : -1;
+    }
+#pragma unroll
+    for (int half = 0; half < (NARROW ? 1 : 2); ++half) {
+        const int rr = NARROW ? (lane >> 2) : (half ? rb : ra);
         uint32_t w[D / 8];
 #pragma unroll
         for (int i = 0; i < D / 8; ++i)
@@ -926,8 +1128,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
-            qa[ks][half] = w[2 * ks];
-            qa[ks][2 + half] = w[2 * ks + 1];
+            if constexpr (NARROW) {
+                qn[ks][0] = w[2 * ks];
+                qn[ks][1] = w[2 * ks + 1];
+            } else {
+                qa[ks][half] = w[2 * ks];
+                qa[ks][2 + half] = w[2 * ks + 1];
+            }
         }
     }
     __syncthreads();  // page ids, scales and barriers are set
@@ -936,7 +1143,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < NT; ++i)
         o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    float on[D / 16][4], m_n[2] = {-INFINITY, -INFINITY}, l_n[2] = {0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i)
+        on[i][0] = on[i][1] = on[i][2] = on[i][3] = 0.f;
     const float sl2 = p.scale_log2;
+
+    // narrow: the scales of keys 2g, 2g + 1 of this warp's page of a stage, loaded a stage ahead
+    auto load_scales = [&](int pidx, float2 &kf, float2 &vf) {
+        kf = vf = make_float2(0.f, 0.f);
+        if (pidx < n_pages) {
+            const int pg = s_pages[pidx];
+            const int key0 = (page_lo + pidx) * 16 + 2 * (lane >> 2);
+            if (pg < p.num_blocks) {
+                const int64_t at = ((int64_t)pg * p.H_kv + g) * 16 + 2 * (lane >> 2);
+                kf = __ldg(reinterpret_cast<const float2 *>(p.k_scale + at));
+                vf = __ldg(reinterpret_cast<const float2 *>(p.v_scale + at));
+            }
+            if (key0 >= ctx)
+                kf.x = vf.x = 0.f;
+            if (key0 + 1 >= ctx)
+                kf.y = vf.y = 0.f;
+        }
+    };
+    float2 kf_next = make_float2(0.f, 0.f), vf_next = make_float2(0.f, 0.f);
+    if constexpr (NARROW)
+        load_scales(kg, kf_next, vf_next);
 
     // ---- main loop over stages (as the 16-bit kernel) ------------------------------------------
     for (int it = 0; it < n_stages; ++it) {
@@ -946,7 +1178,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             *s_abort = 1;
             set_status(p.status, PA_ERR_TIMEOUT);
         }
-        if (ok && has_rows) {
+        if constexpr (NARROW) {
+            // one page per warp per stage (KG = 4)
+            const float2 kf = kf_next, vf = vf_next;
+            load_scales((it + 1) * kPagesPerStage + kg, kf_next, vf_next);
+            const int pidx = it * kPagesPerStage + kg;
+            const int j0 = (page_lo + pidx) * 16;
+            if (ok && has_rows && pidx < n_pages && j0 <= lim_warp) {
+                const uint8_t *st = s_ring + slot * L::kStage;
+                narrow_page_fp8<D, BF16>(st + kg * L::kPage, st + (kPagesPerStage + kg) * L::kPage, kf, vf, j0, lane,
+                                         qn, on, m_n, l_n, lim_n, ctx, sl2);
+            }
+        } else if (ok && has_rows) {
             const uint8_t *st = s_ring + slot * L::kStage;
             for (int k = kg; k < kPagesPerStage; k += KG) {
                 const int pidx = it * kPagesPerStage + k;
@@ -978,8 +1221,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait(&s_bar[s], (s_issued[s] - 1) & 1, kWaitTimeoutNs / 10);
         return;
     }
-    rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_ring), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0,
-                           g, split, n_splits == 1, KG);
+    static_assert(NarrowEpi<D>::kBytes <= kFp8Stages * L::kStage, "the epilogue reuses the ring");
+    if constexpr (NARROW)
+        narrow_epilogue<D, BF16>(reinterpret_cast<float *>(s_ring), p, on, m_n, l_n, rows_here, row0, q0, g, split,
+                                 n_splits == 1);
+    else
+        rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_ring), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0,
+                               q0, g, split, n_splits == 1, KG);
 }
 
 // One warp per (token, query head) row of a sequence with more than one split:
@@ -1124,12 +1372,12 @@ static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtens
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool NARROW>
 static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
                            cudaStream_t stream)
 {
-    using L = Fp8Smem<D>;
-    auto kern = pa_attn_rows_fp8_kernel<D, BF16>;
+    using L = Fp8Smem<D, NARROW>;
+    auto kern = pa_attn_rows_fp8_kernel<D, BF16, NARROW>;
     static uint64_t configured = 0;  // one bit per device, per template instance
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
@@ -1351,7 +1599,9 @@ static int run(const AttnArgs &a)
         dim3 grid(pl.max_splits, a.H_kv * pl.row_groups, a.B);
         rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
         if (rc == PA_OK)
-            rc = fp8       ? launch_rows_fp8<D, BF16>(rp, tk, tv, grid, a.stream)
+            // single-token decode with at most 8 query heads per KV head: keys on the MMA's M side
+            rc = fp8 && a.T == a.B && rp.G <= 8 ? launch_rows_fp8<D, BF16, true>(rp, tk, tv, grid, a.stream)
+                 : fp8     ? launch_rows_fp8<D, BF16, false>(rp, tk, tv, grid, a.stream)
                  : rp.tree ? launch_rows<D, BF16, kModeTree>(rp, tk, tv, grid, a.stream)
                            : launch_rows<D, BF16, kModeCausal>(rp, tk, tv, grid, a.stream);
         if (rc == PA_OK && pl.max_splits > 1)

@@ -166,6 +166,12 @@ FP8_CASES = [
     (3, 8, 400, 2, 8, 64, W.F16),
     (5, 6, 2000, 2, 4, 128, W.BF16),  # several splits
     (4, 3, 33, 2, 2, 64, W.BF16),     # tiny contexts, partial blocks
+    # single-token decode with G <= 8 takes the keys-on-M variant
+    (6, 1, 700, 2, 8, 128, W.BF16),
+    (5, 1, 3000, 1, 4, 64, W.F16),    # several splits
+    (4, 1, 40, 4, 2, 128, W.F16),     # tiny contexts
+    (3, 1, 17, 2, 1, 64, W.BF16),     # one full block and one key
+    (2, 1, 600, 1, 16, 128, W.BF16),  # G 16: the 16-row variant again
 ]
 
 
