@@ -606,20 +606,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 // kernel: a four-stage TMA ring (one 16 x d-byte box per page for K and one for V), refilled by
 // the last warp done with a stage.
 constexpr int kFp8Stages = 4;
+constexpr int kNarrowStages = 3;     // narrow variant: a shallower ring ...
+constexpr int kNarrowCtasPerSm = 4;  // ... and more CTAs on an SM
+
+// Epilogue buffer of a narrow FP8 CTA: O^T, max and sum of every warp's 8 rows.
+template <int D>
+struct NarrowEpi {
+    static constexpr int kStride = D + 4;  // floats per (warp, row) of O
+    static constexpr int kBytes = (4 * 8 * kStride + 2 * 4 * 8) * 4;
+};
 
 // NARROW: no scale table (each warp loads its page's scales into registers one stage ahead), so
 // three CTAs fit on an SM.
 template <int D, bool NARROW>
 struct Fp8Smem {
+    static constexpr int kStages = NARROW ? kNarrowStages : kFp8Stages;
     static constexpr int kPage = 16 * D;                       // codes of one page of K or of V
     static constexpr int kStage = 2 * kPagesPerStage * kPage;  // K pages then V pages
-    static_assert(RowsEpi<D>::kBytes <= kFp8Stages * kStage, "the epilogue reuses the ring");
+    static_assert(NARROW || RowsEpi<D>::kBytes <= kStages * kStage, "the epilogue reuses the ring");
+    static_assert(NarrowEpi<D>::kBytes <= kStages * kStage, "the epilogue reuses the ring");
     static constexpr int kRingOff = 0;
-    static constexpr int kScaleOff = kFp8Stages * kStage;          // [page of the split][K, V][16 keys]
+    static constexpr int kScaleOff = kStages * kStage;          // [page of the split][K, V][16 keys]
     static constexpr int kBarOff = kScaleOff + (NARROW ? 0 : kMaxTablePages * 2 * 16 * 4);
-    static constexpr int kCountOff = kBarOff + 8 * kFp8Stages;     // warps done with each stage
-    static constexpr int kIssuedOff = kCountOff + 4 * kFp8Stages;  // loads issued into each stage
-    static constexpr int kTableOff = kIssuedOff + 4 * kFp8Stages;
+    static constexpr int kCountOff = kBarOff + 8 * kStages;     // warps done with each stage
+    static constexpr int kIssuedOff = kCountOff + 4 * kStages;  // loads issued into each stage
+    static constexpr int kTableOff = kIssuedOff + 4 * kStages;
     static constexpr int kFlagOff = kTableOff + 4 * kMaxTablePages;
     static constexpr int kBytes = kFlagOff + 16;
     static constexpr int kAlloc = kBytes + 128;  // slack to align the base to 128 B
@@ -876,11 +887,6 @@ __device__ __forceinline__ void narrow_page_fp8(const uint8_t *kp, const uint8_t
 
 // Epilogue of a narrow FP8 CTA: the four warps (different pages of the same <= 8 rows) merge
 // through shared memory `e` (at least NarrowEpi<D>::kBytes) like splits; then as rows_epilogue.
-template <int D>
-struct NarrowEpi {
-    static constexpr int kStride = D + 4;  // floats per (warp, row) of O
-    static constexpr int kBytes = (4 * 8 * kStride + 2 * 4 * 8) * 4;
-};
 
 template <int D, bool BF16>
 __device__ __forceinline__ void narrow_epilogue(float *e, const RowsParams &p, const float (&o)[D / 16][4],
@@ -951,12 +957,12 @@ __device__ __forceinline__ void narrow_epilogue(float *e, const RowsParams &p, c
 }
 
 template <int D, bool BF16, bool NARROW>
-__global__ void __launch_bounds__(kThreads, NARROW ? 3 : 1)
+__global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
     pa_attn_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                             const RowsParams p)
 {
     using L = Fp8Smem<D, NARROW>;
-    constexpr int STAGES = kFp8Stages;
+    constexpr int STAGES = L::kStages;
     constexpr int KSTEPS = D / 16;  // k-steps of S = Q K^T
     constexpr int NT = D / 8;       // n-tiles of O
 
@@ -1221,7 +1227,6 @@ __global__ void __launch_bounds__(kThreads, NARROW ? 3 : 1)
                     mbar_wait(&s_bar[s], (s_issued[s] - 1) & 1, kWaitTimeoutNs / 10);
         return;
     }
-    static_assert(NarrowEpi<D>::kBytes <= kFp8Stages * L::kStage, "the epilogue reuses the ring");
     if constexpr (NARROW)
         narrow_epilogue<D, BF16>(reinterpret_cast<float *>(s_ring), p, on, m_n, l_n, rows_here, row0, q0, g, split,
                                  n_splits == 1);
