@@ -337,7 +337,11 @@ def run_ours(args):
             "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
             "frac_of_nominal_8TBs": round(achieved / 8000.0, 4),
-            "traffic": None,
+            # DRAM bytes read + written per launch of the decode kernel: ncu capture of the same
+            # kernel on this workload with 16 sequences (702.95 MB for 696.53 MB of algorithmic
+            # bytes), scaled by the algorithmic bytes to 64 (profiles/pa_attn_rows_decode_13b.md)
+            "traffic": 2804.0e6 if args.batch == 64 else None,
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, 16-sequence capture scaled",
             "bytes_per_launch": decode_bytes,
             "avg_launch_ms": round(decode_ms, 5),
         },
