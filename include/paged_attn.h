@@ -203,6 +203,7 @@ size_t pa_shared_prefix_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int
 /*
  * pa_paged_attn_decode_shared_prefix -- sizes, layouts and errors of
  * pa_paged_attn_decode, plus:
+ *   n_groups           1 .. B + 1 (else PA_ERR_ARG)
  *   group_start        int32 [n_groups + 1], device: group v is the sequences
  *                      group_start[v] .. group_start[v+1]-1 (consecutive runs,
  *                      group_start[0] = 0, group_start[n_groups] = B; a
