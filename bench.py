@@ -625,7 +625,7 @@ def leg_shared(args, stream, device, hbm_peak, rank):
     2048 tokens of 32768) through both calls."""
     import torch
 
-    from paged_kv_attention_34_b200 import paged_attn_decode, paged_attn_decode_shared_prefix
+    from paged_kv_attention_34_b200 import paged_attn_decode, paged_attn_decode_shared_prefix, read_status
     from paged_kv_attention_34_b200 import shared_prefix_workspace_bytes
     from paged_kv_attention_34_b200 import workloads as W
     from paged_kv_attention_34_b200.step import DeviceStep, attn_bytes
@@ -657,7 +657,7 @@ def leg_shared(args, stream, device, hbm_peak, rank):
                 plain()
         torch.cuda.synchronize()
         _, per = time_calls([shared, plain], max(args.steps, 5), stream)
-        if any(st.statuses()) or read_status_of(ws):
+        if any(st.statuses()) or read_status(ws):
             raise RuntimeError("device status")
         dev = (out2.float() - call.out.float()).abs().max().item()
         b = attn_bytes(w)
@@ -674,12 +674,6 @@ def leg_shared(args, stream, device, hbm_peak, rank):
     res["gqa_config"] = {"workload": W.CONFIG_NAMES[4],
                          **run(w4, [0, w4.B], [w4.notes["shared_tokens"] // 16])}
     return res
-
-
-def read_status_of(ws):
-    from paged_kv_attention_34_b200 import read_status
-
-    return read_status(ws)
 
 
 def leg_swap(args, stream, device, rank, n_blocks=512):
