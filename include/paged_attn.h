@@ -328,6 +328,18 @@ int pa_paged_attn_prefill(void *out, const void *q, const void *key_cache, const
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * pa_selftest_wait_timeout -- exercise the failure path that every kernel of
+ * this library shares (no counterpart on the pages): one warp waits on an
+ * mbarrier phase that nothing completes, bounded by `timeout_ns` of
+ * %globaltimer, then records PA_ERR_TIMEOUT in *status (if it still holds
+ * PA_OK) and returns; the context stays usable.  No fault, trap or endless
+ * loop is involved.
+ *   status      int32, device memory, owned by the caller (set it to PA_OK first)
+ *   timeout_ns  1 .. 100,000,000 (0.1 s); else PA_ERR_ARG, nothing launched
+ */
+int pa_selftest_wait_timeout(int32_t *status, uint64_t timeout_ns, void *stream);
+
+/*
  * pa_read_status -- copy the device status word at the start of `workspace`
  * (or any device int32 given to the write/copy calls) into *host_status.
  * This call synchronises `stream`.  Returns PA_OK or PA_ERR_CUDA.

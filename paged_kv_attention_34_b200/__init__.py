@@ -79,6 +79,8 @@ def _declare(L):
     L.pa_prefill_workspace_bytes.argtypes = [I, I, I, I, I]
     L.pa_paged_attn_prefill.restype = I
     L.pa_paged_attn_prefill.argtypes = [P, P, P, P, I64, P, I, P, P, I, I, I, I64, I, I, I, c.c_float, I, P, SZ, P]
+    L.pa_selftest_wait_timeout.restype = I
+    L.pa_selftest_wait_timeout.argtypes = [P, c.c_uint64, P]
     L.pa_read_status.restype = I
     L.pa_read_status.argtypes = [P, P, P]
     L.pa_strerror.restype = c.c_char_p
@@ -407,6 +409,14 @@ def paged_attn_prefill(q, key_cache, value_cache, block_tables, cu_seqlens_q, co
     _check(rc, "pa_paged_attn_prefill")
     paged_attn_prefill.last_workspace = ws
     return out
+
+
+def selftest_wait_timeout(status: torch.Tensor, timeout_ns: int, stream=None) -> None:
+    """Launch the bounded-wait self-test: a wait on a barrier that nothing completes gives up after
+    timeout_ns and records PA_ERR_TIMEOUT in status (int32 device tensor)."""
+    _cuda(status, "status", torch.int32, None)
+    rc = lib().pa_selftest_wait_timeout(_ptr(status), int(timeout_ns), ctypes.c_void_p(_stream(stream)))
+    _check(rc, "pa_selftest_wait_timeout")
 
 
 def read_status(workspace: torch.Tensor, stream=None) -> int:

@@ -162,6 +162,16 @@ def test_shared_prefix_rejects_bad_args(L):
     assert pa.launch_count() == n0
 
 
+def test_selftest_wait_timeout_rejects_bad_args(L):
+    f = L.pa_selftest_wait_timeout
+    n0 = pa.launch_count()
+    assert f(None, 1000, None) == -1
+    assert f(_fake(0x10002), 1000, None) == -1  # misaligned status word
+    assert f(_fake(), 0, None) == -1
+    assert f(_fake(), 100_000_001, None) == -1  # more than 0.1 s
+    assert pa.launch_count() == n0
+
+
 def test_workspace_queries(L):
     # one split needs the status word and the sequence order (B int32 in 256-byte units);
     # long contexts need partials

@@ -386,6 +386,25 @@ def test_inconsistent_sequence_is_reported():
     assert st.statuses()[1] == -8  # PA_ERR_SEQ
 
 
+def test_bounded_wait_runs_out_and_reports_timeout():
+    # the failure path every kernel shares: a wait on a barrier that nothing completes gives up
+    # after its limit, records PA_ERR_TIMEOUT (-6) in the status word and returns; the first error
+    # sticks, and the context stays usable (a decode right after is correct)
+    import time
+
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    pa.selftest_wait_timeout(status, 2_000_000)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert pa.read_status(status) == -6
+    status.fill_(-7)
+    pa.selftest_wait_timeout(status, 1_000_000)
+    assert pa.read_status(status) == -7
+    w = W.random_workload(3, B=2, q_max=1, ctx_max=50, H_kv=1, G=2, d=64, dtype=W.F16, kind="decode")
+    run_and_compare(w)
+
+
 def test_block_copy_bitexact_random():
     g = torch.Generator().manual_seed(3)
     NB, H, d = 40, 4, 128
