@@ -405,6 +405,78 @@ def test_bounded_wait_runs_out_and_reports_timeout():
     run_and_compare(w)
 
 
+_CANARY = 0x7BAD  # an int16 pattern no kernel writes (a large finite fp16 / bf16 value)
+
+
+def _padded(like, pad=4096):
+    """(buffer with `pad` canary elements on each side, a view shaped like `like` inside it)."""
+    n = like.numel()
+    buf = torch.full((n + 2 * pad,), _CANARY, dtype=torch.int16, device=like.device)
+    return buf, buf[pad : pad + n].view(like.dtype).view(like.shape)
+
+
+def _canaries_intact(buf, n, pad=4096):
+    return bool((buf[:pad] == _CANARY).all()) and bool((buf[pad + n :] == _CANARY).all())
+
+
+def test_outputs_and_workspaces_stay_inside_their_buffers():
+    # canary padding around every output and workspace (the pool's compute-sanitizer is closed):
+    # decode, prefill, the FP8 decode and the shared-prefix decode write only inside them
+    w = W.shared_prefix_batch(seed=90, B=6, n_groups=2, prefix_tokens=64, suffix=(1, 300), q_max=3, H_q=8,
+                              H_kv=2, d=128, dtype=W.BF16)
+    st = DeviceStep(w)
+    st.copy_blocks()
+    st.write()
+    call = st.calls[0]
+    n = call.out.numel()
+
+    def ws_padded(nbytes, pad=4096):
+        buf = torch.full((nbytes + 2 * pad,), 0x5A, dtype=torch.uint8, device="cuda")
+        return buf, buf[pad : pad + nbytes]
+
+    def ws_intact(buf, nbytes, pad=4096):
+        return bool((buf[:pad] == 0x5A).all()) and bool((buf[pad + nbytes :] == 0x5A).all())
+
+    # decode
+    ob, out = _padded(call.out)
+    wb, ws = ws_padded(call.ws.numel())
+    pa.paged_attn_decode(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, call.max_ctx, w.scale,
+                         out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0 and _canaries_intact(ob, n) and ws_intact(wb, call.ws.numel())
+    # shared-prefix decode
+    starts, P = w.notes["group_start"], w.notes["prefix_blocks"]
+    gs = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    pb = torch.tensor(P, dtype=torch.int32, device="cuda")
+    max_gt = max(sum(w.q_lens[starts[v] : starts[v + 1]]) for v in range(len(P)))
+    nbytes = pa.shared_prefix_workspace_bytes(w.T, w.B, w.H_q, w.H_kv, w.d, call.max_ctx, len(P), max(P), max_gt)
+    ob, out = _padded(call.out)
+    wb, ws = ws_padded(nbytes)
+    pa.paged_attn_decode_shared_prefix(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, gs, pb,
+                                       call.max_ctx, max(P), max_gt, w.scale, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0 and _canaries_intact(ob, n) and ws_intact(wb, nbytes)
+    # FP8 decode over the same keys
+    kc8, vc8, ks, vs = _fp8_device_cache(w)
+    ob, out = _padded(call.out)
+    wb, ws = ws_padded(call.ws.numel())
+    pa.paged_attn_decode_fp8(call.q, kc8, vc8, ks, vs, call.bt, call.cu, call.ctx, call.max_ctx, w.scale, out=out,
+                             workspace=ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0 and _canaries_intact(ob, n) and ws_intact(wb, call.ws.numel())
+    # prefill (chunks with earlier context)
+    wp = W.random_workload(91, B=3, q_max=150, ctx_max=300, H_kv=2, G=4, d=128, dtype=W.BF16, kind="prefill")
+    sp = DeviceStep(wp)
+    sp.write()
+    pc = sp.calls[0]
+    ob, out = _padded(pc.out)
+    wb, ws = ws_padded(pc.ws.numel())
+    pa.paged_attn_prefill(pc.q, sp.key_cache, sp.value_cache, pc.bt, pc.cu, pc.ctx, pc.max_q_len, pc.max_ctx,
+                          wp.scale, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert pa.read_status(ws) == 0 and _canaries_intact(ob, pc.out.numel()) and ws_intact(wb, pc.ws.numel())
+
+
 def test_block_copy_bitexact_random():
     g = torch.Generator().manual_seed(3)
     NB, H, d = 40, 4, 128
