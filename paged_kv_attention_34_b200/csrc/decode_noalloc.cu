@@ -60,6 +60,7 @@ extern "C" int pa_paged_attn_decode_noalloc(void *out, const void *q, const void
                                             int max_ctx, int64_t T, int H_q, int H_kv, int d, float scale,
                                             pa_dtype dtype, int32_t *status, void *stream)
 {
+    pa::CallRange range(__func__);
     const size_t need = pa_decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx);
     if (need == 0)
         return PA_ERR_ARG;

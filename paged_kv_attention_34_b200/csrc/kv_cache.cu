@@ -191,6 +191,7 @@ extern "C" int pa_kv_cache_write(const void *k_new, const void *v_new, const int
                                  void *key_cache, void *value_cache, int64_t num_blocks, int H_kv, int d,
                                  pa_dtype dtype, int32_t *status, void *stream)
 {
+    CallRange range(__func__);
     if (T < 0 || num_blocks < 1 || H_kv < 1)
         return PA_ERR_ARG;
     if (dtype != PA_F16 && dtype != PA_BF16)
@@ -223,6 +224,7 @@ extern "C" int pa_kv_cache_write(const void *k_new, const void *v_new, const int
 extern "C" int pa_kv_block_copy(void *key_cache, void *value_cache, int64_t num_blocks, int H_kv, int d,
                                 pa_dtype dtype, const int32_t *pairs, int64_t n, int32_t *status, void *stream)
 {
+    CallRange range(__func__);
     if (n < 0 || num_blocks < 1 || H_kv < 1)
         return PA_ERR_ARG;
     if (dtype != PA_F16 && dtype != PA_BF16)
@@ -261,6 +263,7 @@ extern "C" int pa_kv_block_swap(void *key_cache, void *value_cache, int64_t num_
                                 void *host_value, int64_t host_blocks, int H_kv, int d, pa_dtype dtype,
                                 const int32_t *pairs, int64_t n, int direction, int32_t *status, void *stream)
 {
+    CallRange range(__func__);
     if (n < 0 || num_blocks < 1 || host_blocks < 1 || H_kv < 1)
         return PA_ERR_ARG;
     if (dtype != PA_F16 && dtype != PA_BF16)
@@ -292,6 +295,7 @@ extern "C" int pa_kv_cache_write_fp8(const void *k_new, const void *v_new, const
                                      uint8_t *key_cache, uint8_t *value_cache, float *key_scale, float *value_scale,
                                      int64_t num_blocks, int H_kv, int d, pa_dtype dtype, int32_t *status, void *stream)
 {
+    CallRange range(__func__);
     if (T < 0 || num_blocks < 1 || H_kv < 1)
         return PA_ERR_ARG;
     if (dtype != PA_F16 && dtype != PA_BF16)

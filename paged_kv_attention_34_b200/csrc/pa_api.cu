@@ -151,6 +151,7 @@ extern "C" int pa_paged_attn_decode(void *out, const void *q, const void *key_ca
                                     int64_t T, int H_q, int H_kv, int d, float scale, pa_dtype dtype,
                                     void *workspace, size_t workspace_bytes, void *stream)
 {
+    CallRange range(__func__);
     AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
                context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
                static_cast<cudaStream_t>(stream)};
@@ -172,6 +173,7 @@ extern "C" int pa_paged_attn_decode_tree(void *out, const void *q, const void *k
                                          int d, float scale, pa_dtype dtype, void *workspace, size_t workspace_bytes,
                                          void *stream)
 {
+    CallRange range(__func__);
     AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
                context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
                static_cast<cudaStream_t>(stream), tree_mask};
@@ -211,6 +213,7 @@ extern "C" int pa_paged_attn_decode_shared_prefix(void *out, const void *q, cons
                                                   int max_group_tokens, void *workspace, size_t workspace_bytes,
                                                   void *stream)
 {
+    CallRange range(__func__);
     AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
                context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
                static_cast<cudaStream_t>(stream)};
@@ -247,6 +250,7 @@ extern "C" int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t 
                                         int64_t T, int H_q, int H_kv, int d, float scale, pa_dtype dtype,
                                         void *workspace, size_t workspace_bytes, void *stream)
 {
+    CallRange range(__func__);
     AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
                context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
                static_cast<cudaStream_t>(stream), nullptr, key_scale, value_scale};
@@ -280,6 +284,7 @@ extern "C" int pa_paged_attn_prefill(void *out, const void *q, const void *key_c
                                      int max_q_len, int max_ctx, int64_t T, int H_q, int H_kv, int d, float scale,
                                      pa_dtype dtype, void *workspace, size_t workspace_bytes, void *stream)
 {
+    CallRange range(__func__);
     AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
                context_lens, B, max_q_len, max_ctx, T, H_q, H_kv, d, scale, dtype, workspace, workspace_bytes,
                static_cast<cudaStream_t>(stream)};
@@ -296,6 +301,7 @@ extern "C" int pa_paged_attn_prefill(void *out, const void *q, const void *key_c
 
 extern "C" int pa_read_status(const void *workspace, int32_t *host_status, void *stream)
 {
+    CallRange range(__func__);
     if (!workspace || !host_status)
         return PA_ERR_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

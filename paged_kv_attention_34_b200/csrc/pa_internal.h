@@ -7,7 +7,19 @@
 
 #include "../../include/paged_attn.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace pa {
+
+// An NVTX range around one library call, named after its entry point, for timelines in the
+// profilers; free when no profiler is attached (NVTX v3 is header-only and looks for a tool on
+// first use).
+struct CallRange {
+    explicit CallRange(const char *name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange &) = delete;
+    CallRange &operator=(const CallRange &) = delete;
+};
 
 // Counts every kernel launch of the library (pa_launch_count).
 void count_launch(uint64_t n = 1);

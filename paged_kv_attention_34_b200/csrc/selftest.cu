@@ -27,6 +27,7 @@ using namespace pa;
 
 extern "C" int pa_selftest_wait_timeout(int32_t *status, uint64_t timeout_ns, void *stream)
 {
+    CallRange range(__func__);
     if (!aligned4(status) || timeout_ns == 0 || timeout_ns > 100000000ull)
         return PA_ERR_ARG;
     pa_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status, timeout_ns);
