@@ -50,6 +50,9 @@ if ROOT not in sys.path:
 
 METRIC = "paged decode attn HBM GB/s & prefill attn TFLOPS, as % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# ncu DRAM bytes (read + written) / algorithmic bytes of the 16-bit decode kernel, captured on the
+# 13B-shaped decode layer with 16 sequences: 702.95 MB / 696.53 MB
+TRAFFIC_RATIO_DECODE_13B = 702.95 / 696.53
 HEADLINE = "LLaMA-2-13B-shaped decode layer: B 64, q_len 1, 40/40 heads, d 128, fp16, ctx U[128,4096], block 16"
 
 
@@ -337,10 +340,11 @@ def run_ours(args):
             "unit": "GB/s",
             "frac": round(achieved / hbm_peak, 4),
             "frac_of_nominal_8TBs": round(achieved / 8000.0, 4),
-            # DRAM bytes read + written per launch of the decode kernel: ncu capture of the same
-            # kernel on this workload with 16 sequences (702.95 MB for 696.53 MB of algorithmic
-            # bytes), scaled by the algorithmic bytes to 64 (profiles/pa_attn_rows_decode_13b.md)
-            "traffic": 2804.0e6 if args.batch == 64 else None,
+            # DRAM bytes read + written per launch of the decode kernel: an ncu capture of the same
+            # kernel on this workload with 16 sequences measured 1.0092 x its algorithmic bytes (the
+            # padding rows of last partial blocks); the same ratio applied to this run's algorithmic
+            # bytes.  Only for the captured shape (fp16, 40/40 heads, contexts U[128, 4096]).
+            "traffic": round(TRAFFIC_RATIO_DECODE_13B * decode_bytes) if w.name == "cfg2" else None,
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, 16-sequence capture scaled",
             "bytes_per_launch": decode_bytes,
             "avg_launch_ms": round(decode_ms, 5),

@@ -276,8 +276,8 @@ int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t *key_cache,
  * allocate device memory when they call, such as plugins inside an engine that
  * owns all device memory and forbids allocation while work is enqueued, or
  * latency-critical code that cannot take cudaMalloc's implicit synchronisation
- * or a possible allocation failure mid-step.  Same arguments and results as
- * pa_paged_attn_decode, except:
+ * or a possible allocation failure mid-step.  Same arguments, argument checks,
+ * error codes and results as pa_paged_attn_decode, except:
  *   - the scratch (status word + split partials) is a fixed array of
  *     PA_DECODE_NOALLOC_SCRATCH_BYTES inside the library; every GPU that loads
  *     it holds that memory until the process exits;
@@ -345,6 +345,16 @@ int pa_selftest_wait_timeout(int32_t *status, uint64_t timeout_ns, void *stream)
  * This call synchronises `stream`.  Returns PA_OK or PA_ERR_CUDA.
  */
 int pa_read_status(const void *workspace, int32_t *host_status, void *stream);
+
+/*
+ * pa_get_status -- the device status word at the start of `workspace` (or any
+ * device int32 given to the write/copy calls), returned directly.  It first
+ * waits for all work on the current device (every stream), so it suits a
+ * check after a step, not the middle of a pipeline (pa_read_status waits for
+ * one stream only).  Returns the word (PA_OK or a device-detected pa_status),
+ * or PA_ERR_ARG for NULL, PA_ERR_CUDA if the runtime fails.
+ */
+int pa_get_status(const void *workspace);
 
 /* pa_strerror -- static text for a pa_status value. */
 const char *pa_strerror(int code);

@@ -83,6 +83,8 @@ def _declare(L):
     L.pa_selftest_wait_timeout.argtypes = [P, c.c_uint64, P]
     L.pa_read_status.restype = I
     L.pa_read_status.argtypes = [P, P, P]
+    L.pa_get_status.restype = I
+    L.pa_get_status.argtypes = [P]
     L.pa_strerror.restype = c.c_char_p
     L.pa_strerror.argtypes = [I]
     L.pa_launch_count.restype = c.c_uint64
@@ -229,7 +231,7 @@ def prefill_workspace_bytes(B: int, H_q: int, H_kv: int, d: int, max_q_len: int)
     return int(n)
 
 
-def _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, out):
+def _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_lens, out, stream=None):
     _cuda(q, "q", ndim=3)
     dt = q.dtype
     _cuda(key_cache, "key_cache", dt, 4)
@@ -245,7 +247,7 @@ def _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_
     if cu_seqlens_q.shape[0] != B + 1 or block_tables.shape[0] != B:
         raise ValueError("cu_seqlens_q must have B+1 entries and block_tables B rows")
     if out is None:
-        out = torch.empty_like(q)
+        out = _bind_to_stream(torch.empty_like(q), stream)
     else:
         _cuda(out, "out", dt, 3)
         if out.shape != q.shape:
@@ -253,9 +255,18 @@ def _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q, context_
     return out, T, H_q, d, NB, H_kv, B
 
 
-def _workspace(ws, nbytes, device):
+def _bind_to_stream(t: torch.Tensor, stream) -> torch.Tensor:
+    """A tensor allocated here (workspace, output) is used by kernels on `stream`; when that is not
+    the current stream, tell the caching allocator, so the memory is not handed out again on the
+    current stream while those kernels may still run."""
+    if stream is not None and stream != torch.cuda.current_stream(t.device):
+        t.record_stream(stream)
+    return t
+
+
+def _workspace(ws, nbytes, device, stream=None):
     if ws is None:
-        return torch.empty(nbytes, dtype=torch.uint8, device=device)
+        return _bind_to_stream(torch.empty(nbytes, dtype=torch.uint8, device=device), stream)
     _cuda(ws, "workspace", torch.uint8, 1)
     if ws.numel() < nbytes:
         raise ValueError(f"workspace too small: {ws.numel()} < {nbytes}")
@@ -266,9 +277,9 @@ def paged_attn_decode(q, key_cache, value_cache, block_tables, cu_seqlens_q, con
                       scale: float, out=None, workspace=None, stream=None):
     """Split-KV decode for 1..8 query tokens per sequence; returns out [T, H_q, d]."""
     out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
-                                               context_lens, out)
+                                               context_lens, out, stream)
     nbytes = decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx)
-    ws = _workspace(workspace, nbytes, q.device)
+    ws = _workspace(workspace, nbytes, q.device, stream)
     rc = lib().pa_paged_attn_decode(
         _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
         _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_ctx), T, H_q, H_kv, d, float(scale),
@@ -324,9 +335,9 @@ def paged_attn_decode_fp8(q, key_cache, value_cache, key_scale, value_scale, blo
     _cuda(context_lens, "context_lens", torch.int32, 1)
     B = context_lens.shape[0]
     if out is None:
-        out = torch.empty_like(q)
+        out = _bind_to_stream(torch.empty_like(q), stream)
     nbytes = decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx)
-    ws = _workspace(workspace, nbytes, q.device)
+    ws = _workspace(workspace, nbytes, q.device, stream)
     rc = lib().pa_paged_attn_decode_fp8(
         _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(key_scale), _ptr(value_scale), NB,
         _ptr(block_tables), block_tables.shape[1], _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_ctx), T, H_q,
@@ -342,12 +353,12 @@ def paged_attn_decode_tree(q, key_cache, value_cache, block_tables, cu_seqlens_q
     """Tree-attention verification: decode where token t sees the cached keys before its sequence's
     new tokens and new token j when bit j of tree_mask[t] (int32 [T]) is set; returns out."""
     out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
-                                               context_lens, out)
+                                               context_lens, out, stream)
     _cuda(tree_mask, "tree_mask", torch.int32, 1)
     if tree_mask.shape[0] != T:
         raise ValueError(f"tree_mask must be int32 [{T}]")
     nbytes = decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx)
-    ws = _workspace(workspace, nbytes, q.device)
+    ws = _workspace(workspace, nbytes, q.device, stream)
     rc = lib().pa_paged_attn_decode_tree(
         _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
         _ptr(cu_seqlens_q), _ptr(context_lens), _ptr(tree_mask), B, int(max_ctx), T, H_q, H_kv, d, float(scale),
@@ -374,7 +385,7 @@ def paged_attn_decode_shared_prefix(q, key_cache, value_cache, block_tables, cu_
     tables (group v = sequences group_start[v] .. group_start[v+1]-1, int32 device tensors): the
     shared blocks are read once per group, then merged with each sequence's own keys; returns out."""
     out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
-                                               context_lens, out)
+                                               context_lens, out, stream)
     _cuda(group_start, "group_start", torch.int32, 1)
     _cuda(prefix_blocks, "prefix_blocks", torch.int32, 1)
     n_groups = prefix_blocks.shape[0]
@@ -382,7 +393,7 @@ def paged_attn_decode_shared_prefix(q, key_cache, value_cache, block_tables, cu_
         raise ValueError(f"group_start must be int32 [{n_groups + 1}]")
     nbytes = shared_prefix_workspace_bytes(T, B, H_q, H_kv, d, max_ctx, n_groups, max_prefix_blocks,
                                            max_group_tokens)
-    ws = _workspace(workspace, nbytes, q.device)
+    ws = _workspace(workspace, nbytes, q.device, stream)
     rc = lib().pa_paged_attn_decode_shared_prefix(
         _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
         _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_ctx), T, H_q, H_kv, d, float(scale), _dtype_code(q),
@@ -398,9 +409,9 @@ def paged_attn_prefill(q, key_cache, value_cache, block_tables, cu_seqlens_q, co
                        max_ctx: int, scale: float, out=None, workspace=None, stream=None):
     """Causal varlen prefill over the paged cache; returns out [T, H_q, d]."""
     out, T, H_q, d, NB, H_kv, B = _attn_common(q, key_cache, value_cache, block_tables, cu_seqlens_q,
-                                               context_lens, out)
+                                               context_lens, out, stream)
     nbytes = prefill_workspace_bytes(B, H_q, H_kv, d, max_q_len)
-    ws = _workspace(workspace, nbytes, q.device)
+    ws = _workspace(workspace, nbytes, q.device, stream)
     rc = lib().pa_paged_attn_prefill(
         _ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), NB, _ptr(block_tables), block_tables.shape[1],
         _ptr(cu_seqlens_q), _ptr(context_lens), B, int(max_q_len), int(max_ctx), T, H_q, H_kv, d, float(scale),
@@ -426,3 +437,13 @@ def read_status(workspace: torch.Tensor, stream=None) -> int:
     rc = lib().pa_read_status(_ptr(workspace), ctypes.byref(val), ctypes.c_void_p(_stream(stream)))
     _check(rc, "pa_read_status")
     return int(val.value)
+
+
+def get_status(workspace: torch.Tensor) -> int:
+    """Device status word at the start of a workspace (or a status tensor), after waiting for all
+    work on the current device.  Raises only if the runtime fails."""
+    _cuda(workspace, "workspace")
+    rc = int(lib().pa_get_status(_ptr(workspace)))
+    if rc == -5:  # the kernels never record PA_ERR_CUDA: this is the runtime failing
+        _check(rc, "pa_get_status")
+    return rc

@@ -61,6 +61,13 @@ extern "C" int pa_paged_attn_decode_noalloc(void *out, const void *q, const void
                                             pa_dtype dtype, int32_t *status, void *stream)
 {
     pa::CallRange range(__func__);
+    // the same size and shape checks as pa_paged_attn_decode, so both return the same code
+    pa::AttnArgs a{out, q, key_cache, value_cache, num_blocks, block_tables, max_blocks_per_seq, cu_seqlens_q,
+                   context_lens, B, 8, max_ctx, T, H_q, H_kv, d, scale, dtype, nullptr, 0,
+                   static_cast<cudaStream_t>(stream)};
+    const int shape_rc = pa::check_attn_shape(a, true);
+    if (shape_rc != PA_OK)
+        return shape_rc;
     const size_t need = pa_decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx);
     if (need == 0)
         return PA_ERR_ARG;

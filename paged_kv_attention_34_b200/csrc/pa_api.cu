@@ -102,10 +102,10 @@ int reset_status(void *workspace, cudaStream_t stream)
     return cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-// Checks shared by decode and prefill.  Largest TMA row coordinate used is
-// (num_blocks + 1) * H_kv * 16 (one past the pool marks a bad block id), which
-// must stay below 2^31.
-static int check_attn(const AttnArgs &a, bool decode)
+// Size and shape checks shared by decode and prefill (no pointer is looked at).  Largest TMA
+// row coordinate used is (num_blocks + 1) * H_kv * 16 (one past the pool marks a bad block id),
+// which must stay below 2^31.
+int check_attn_shape(const AttnArgs &a, bool decode)
 {
     if (a.B < 0 || a.T < 0 || a.H_q < 1 || a.H_kv < 1 || a.num_blocks < 1 || a.max_blocks < 1 || a.max_ctx < 0)
         return PA_ERR_ARG;
@@ -119,6 +119,15 @@ static int check_attn(const AttnArgs &a, bool decode)
         return PA_ERR_UNSUPPORTED;
     if (!decode && a.max_q_len < 1)
         return PA_ERR_ARG;
+    return PA_OK;
+}
+
+// Every host-side check of decode and prefill: sizes and shapes, then workspace and pointers.
+static int check_attn(const AttnArgs &a, bool decode)
+{
+    const int rc = check_attn_shape(a, decode);
+    if (rc != PA_OK)
+        return rc;
     if (!a.workspace)
         return PA_ERR_WORKSPACE;
     if (!aligned16(a.workspace))
@@ -308,6 +317,18 @@ extern "C" int pa_read_status(const void *workspace, int32_t *host_status, void 
     if (cudaMemcpyAsync(host_status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return PA_ERR_CUDA;
     return cudaStreamSynchronize(s) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+extern "C" int pa_get_status(const void *workspace)
+{
+    CallRange range(__func__);
+    if (!workspace)
+        return PA_ERR_ARG;
+    int32_t word = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpy(&word, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return PA_ERR_CUDA;
+    return word;
 }
 
 extern "C" const char *pa_strerror(int code)

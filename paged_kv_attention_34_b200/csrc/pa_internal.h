@@ -38,6 +38,11 @@ int make_cache_tmap(CUtensorMap *map, const void *cache, int64_t num_blocks, int
 // KV head: dims (d, H_q, T), box (64, G, tok), 128-byte swizzle.
 int make_q_tmap(CUtensorMap *map, const void *q, int64_t T, int H_q, int d, int G, int tok, pa_dtype dtype);
 
+// The size and shape checks of decode and prefill, before any pointer or workspace check:
+// PA_OK, PA_ERR_ARG or PA_ERR_UNSUPPORTED.
+struct AttnArgs;
+int check_attn_shape(const AttnArgs &a, bool decode);
+
 // Reset the status word at the start of a workspace on `stream`.
 int reset_status(void *workspace, cudaStream_t stream);
 

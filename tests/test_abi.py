@@ -130,6 +130,32 @@ def test_decode_rejects_bad_args(L):
     assert _decode(L, dt=3) == -1
 
 
+def test_noalloc_decode_returns_the_same_codes_as_decode(L):
+    """The allocation-free decode runs the same size and shape checks as the regular one, before
+    its scratch-size check; none of these calls reaches the device."""
+    f = L.pa_paged_attn_decode_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p]
+
+    def noalloc(B=2, T=2, H_q=8, H_kv=2, d=128, max_ctx=100, NB=16, dt=1):
+        return f(_fake(), _fake(), _fake(), _fake(), NB, _fake(), 8, _fake(), _fake(), B, max_ctx, T, H_q, H_kv, d,
+                 0.1, dt, None, None)
+
+    n0 = pa.launch_count()
+    for bad in (dict(d=96), dict(H_q=3, H_kv=2), dict(H_q=6, H_kv=4), dict(B=-1), dict(T=-1), dict(H_kv=0),
+                dict(NB=0), dict(dt=3), dict(max_ctx=-1), dict(NB=(1 << 31) // 32)):
+        assert noalloc(**bad) == _decode(L, **bad), bad
+        assert noalloc(**bad) in (-1, -2), bad
+    assert pa.launch_count() == n0
+
+
+def test_get_status_rejects_null(L):
+    assert L.pa_get_status(None) == -1
+
+
 def test_prefill_rejects_bad_args(L):
     f = L.pa_paged_attn_prefill
 
