@@ -179,10 +179,28 @@ class ClockSampler:
 
 # ---- timing helpers ----------------------------------------------------------------------------------
 
-def time_calls(fn_list, steps, stream):
+def pctl(xs, q):
+    """q-th percentile (0..100) of a list, linear interpolation between order statistics."""
+    ys = sorted(xs)
+    if not ys:
+        return None
+    pos = (len(ys) - 1) * q / 100.0
+    lo = int(math.floor(pos))
+    hi = min(lo + 1, len(ys) - 1)
+    return ys[lo] + (ys[hi] - ys[lo]) * (pos - lo)
+
+
+def stats_ms(xs):
+    """mean / p10 / p50 / p90 of per-step durations (ms)."""
+    return {"mean": round(sum(xs) / len(xs), 5), "p10": round(pctl(xs, 10), 5), "p50": round(pctl(xs, 50), 5),
+            "p90": round(pctl(xs, 90), 5), "n": len(xs)}
+
+
+def time_calls(fn_list, steps, stream, per_step=None):
     """Run `steps` iterations of the step; per-call CUDA-event durations on `stream`.
 
-    Returns (total_ms, [avg_ms per call]) with the total bracketed by events."""
+    Returns (total_ms, [avg_ms per call]) with the total bracketed by events; when `per_step` is a
+    list, it receives, for every step, the list of that step's call durations."""
     import torch
 
     n = len(fn_list)
@@ -198,7 +216,10 @@ def time_calls(fn_list, steps, stream):
                 evs[s][i][1].record(stream)
         end.record(stream)
     end.synchronize()
-    per = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(steps)) / steps for i in range(n)]
+    durs = [[evs[s][i][0].elapsed_time(evs[s][i][1]) for i in range(n)] for s in range(steps)]
+    if per_step is not None:
+        per_step.extend(durs)
+    per = [sum(durs[s][i] for s in range(steps)) / steps for i in range(n)]
     return start.elapsed_time(end), per
 
 
@@ -240,10 +261,13 @@ def bench_leg(w, steps, warmup, stream, device):
             for fn in fns:
                 fn()
     torch.cuda.synchronize()
-    total, per = time_calls(fns, steps, stream)
+    durs = []
+    total, per = time_calls(fns, steps, stream, durs)
     stat = st.statuses()
     if any(stat):
         raise RuntimeError(f"{w.name}: device status {stat}")
+    st.call_stats = {name: stats_ms([d[i] for d in durs]) for i, name in enumerate(names)}
+    st.step_stats = stats_ms([sum(d) for d in durs])
     return st, dict(zip(names, per)), total / steps
 
 
@@ -288,7 +312,8 @@ def run_ours(args):
     with ClockSampler(local_rank) as clk:
         # per-call durations (CUDA events around every call), then the timed steps themselves with
         # events only at the two ends, so the step time carries no per-call event overhead
-        _, per = time_calls(fns, args.steps, stream)
+        durs = []
+        _, per = time_calls(fns, args.steps, stream, durs)
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
@@ -352,6 +377,10 @@ def run_ours(args):
         "gpu_launches": n_launch,
         "e2e": e2e,
         "per_call_ms": {"kv_cache_write": round(per[0], 5), "paged_attn_decode": round(per[1], 5)},
+        # per-step distributions from the pass with events around every call (the step time above
+        # comes from the pass with events only at its ends)
+        "step_ms_stats": stats_ms([sum(d) for d in durs]),
+        "decode_ms_stats": stats_ms([d[1] for d in durs]),
     }
     clk_sum = clk.summary()
     result["clocks"] = clk_sum if clk_sum else {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
@@ -370,6 +399,8 @@ def run_ours(args):
         }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        if not args.no_legs:
+            result["cpu_baseline"]["per_config"] = cpu_baseline_configs(args.cpu_seconds / 2)
     del st
     if world > 1:
         barrier()
@@ -511,6 +542,7 @@ def leg_prefill(args, stream, device, bf16_peak, peak_src, rank):
         "kv_cache_write": {"GB/s": round(wb / (per["kv_cache_write"] * 1e-3) / 1e9, 1), "bytes": wb,
                            "avg_launch_ms": round(per["kv_cache_write"], 5)},
         "tokens_per_s": round(w.T / (step_ms * 1e-3), 1),
+        "prefill_ms_stats": st.call_stats["paged_attn_prefill"],
     }
 
 
@@ -526,6 +558,7 @@ def leg_gqa(args, stream, device, hbm_peak, rank):
     return {"workload": W.CONFIG_NAMES[4], "decode_GB/s": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
             "unique_bytes": b, "decode_ms": round(ms, 5), "step_ms": round(step_ms, 5),
             "per_call_ms": {k: round(v, 5) for k, v in per.items()},
+            "decode_ms_stats": st.call_stats["paged_attn_decode"], "step_ms_stats": st.step_stats,
             "note": "shared prefix counted once; its blocks may stay in L2 across sequences"}
 
 
@@ -735,7 +768,8 @@ def leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank):
     return {"workload": W.CONFIG_NAMES[5], "frac": round(sum(t_roof.values()) / sum(meas.values()), 4),
             "per_call_ms": {k: round(v, 5) for k, v in per.items()},
             "per_call_frac": {k: round(t_roof[k] / meas[k], 4) for k in t_roof},
-            "tokens_per_s": round(w.T / (step_ms * 1e-3), 1), "step_ms": round(step_ms, 5)}
+            "tokens_per_s": round(w.T / (step_ms * 1e-3), 1), "step_ms": round(step_ms, 5),
+            "step_ms_stats": st.step_stats}
 
 
 # ---- the CPU oracle ---------------------------------------------------------------------------------------------
@@ -783,6 +817,73 @@ def cpu_baseline(w, seconds: float):
     rate, dt, b = oracle_sample_rate(w, caches, n, threads)
     return {"value": round(rate, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
             "sample": f"first {n} of {w.B} sequences (all 40 heads), {b/1e9:.3f} GB of KV, {dt:.1f} s"}
+
+
+def row_keys(w):
+    """Visible keys of every (token, query head) row of a workload, row index t * H_q + h."""
+    import numpy as np
+
+    keys = np.empty(w.T, dtype=np.int64)
+    cu = w.cu_seqlens_q.tolist()
+    for b in range(w.B):
+        qb, ctx = w.q_lens[b], w.ctx_lens[b]
+        keys[cu[b]:cu[b + 1]] = ctx - qb + 1 + np.arange(qb)
+    return np.repeat(keys, w.H_q)
+
+
+def oracle_extrapolated(w, seconds: float, threads: int, seed: int):
+    """Time the fp64 oracle on a seeded random sample of the workload's query rows, sized to about
+    `seconds` of host time, and extrapolate to the whole workload by visible keys (its work per
+    row is one dot product and one accumulation per visible key).  Returns (seconds for the
+    whole workload, description of the sample)."""
+    import numpy as np
+
+    import oracle
+
+    kc, vc = oracle_caches(w)
+    keys = row_keys(w)
+    order = np.random.default_rng(seed).permutation(keys.shape[0])
+
+    def run(n):
+        rows = np.sort(order[:n])
+        t0 = time.perf_counter()
+        oracle.paged_attention(w.q, kc, vc, oracle.dtype_code(w.dtype), w.block_tables, w.cu_seqlens_q,
+                               w.context_lens, w.H_kv, w.scale, rows=rows, n_threads=threads)
+        return time.perf_counter() - t0, int(keys[rows].sum())
+
+    n = min(64, keys.shape[0])
+    dt, k = run(n)
+    n = int(min(keys.shape[0], max(n, n * seconds / max(dt, 1e-3))))
+    dt, k = run(n)
+    total = float(dt) * float(keys.sum()) / max(k, 1)
+    return total, f"{n} of {keys.shape[0]} query rows drawn at random (seed {seed}), {k} visible keys, {dt:.1f} s"
+
+
+def cpu_baseline_configs(seconds: float):
+    """The oracle on the other configurations' workloads (bounded samples, extrapolated): the
+    causal varlen prefill (TFLOP/s of exact causal pairs), the long-context GQA decode with a
+    shared prefix (GB/s of distinct bytes) and the mixed continuous-batching step (tokens/s of
+    the two attention calls)."""
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import attn_bytes, attn_flops
+
+    threads = os.cpu_count() or 1
+    res = {}
+    w3 = W.config3(seed=shard_seed(34_003, 0))
+    t3, smp = oracle_extrapolated(w3, seconds, threads, 3)
+    res["cfg3_prefill"] = {"value": round(attn_flops(w3) / t3 / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+                           "kind": "oracle", "sample": smp}
+    del w3
+    w4 = W.config4(seed=shard_seed(34_004, 0))
+    t4, smp = oracle_extrapolated(w4, seconds, threads, 4)
+    res["cfg4_gqa_decode"] = {"value": round(attn_bytes(w4) / t4 / 1e9, 4), "unit": "GB/s", "cores": threads,
+                              "kind": "oracle", "sample": smp}
+    del w4
+    w5 = W.config5(seed=shard_seed(34_005, 0))
+    t5, smp = oracle_extrapolated(w5, seconds, threads, 5)
+    res["cfg5_mixed_step"] = {"value": round(w5.T / t5, 1), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                              "sample": smp, "step_s": round(t5, 3)}
+    return res
 
 
 def run_reference(args):

@@ -223,6 +223,10 @@ size_t pa_shared_prefix_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int
  * max_group_tokens set PA_ERR_ARG in the status word (every sequence is then
  * computed alone).  Launches: a one-CTA plan kernel, the sequence order, the
  * attention kernel (prefix CTAs first, then the sequences'), the merge.
+ * When the sharing saves little -- estimated from the host bounds as
+ * (n - 1) / n x 16 max_prefix_blocks / max_ctx < 1/4 with n = B / n_groups --
+ * the call runs the plain decode over the same tables instead (same result,
+ * faster there; the groups are still checked).
  */
 int pa_paged_attn_decode_shared_prefix(void *out, const void *q, const void *key_cache, const void *value_cache,
                                        int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,

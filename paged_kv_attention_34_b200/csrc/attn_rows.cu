@@ -23,57 +23,16 @@
 // every stage (several warps on different pages when there are <= 32 rows,
 // merged at the end like splits).  S = Q K^T and O += P V run on mma.sync
 // m16n8k16 with fp32 accumulators; P is rounded to the input type for P V.
+#include <algorithm>
 #include <cmath>
 
 #include <cuda_fp8.h>
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "rows_common.cuh"
 
 namespace pa {
-
-constexpr int kRowsPerCta = 64;
-constexpr int kPagesPerStage = 4;
-constexpr int kMaxTablePages = 256;  // page ids of one split (split_pages <= this)
-constexpr int kThreads = 128;
-
-// What the rows of a decode CTA see: causal (the new tokens in order), a tree-verification mask
-// over the new tokens, or the shared-prefix pass (causal sequence CTAs plus prefix CTAs whose
-// rows see every prefix key).
-constexpr int kModeCausal = 0;
-constexpr int kModeTree = 1;
-constexpr int kModeShared = 2;
-
-struct RowsParams {
-    const void *q;
-    void *out;
-    const int32_t *block_tables;
-    const int32_t *cu_seqlens;
-    const int32_t *context_lens;
-    float *ws_o;    // [max_splits][T][H_q][D] normalised partial outputs
-    float *ws_lse;  // [max_splits][T][H_q] log2-sum-exp of the scaled scores
-    const int32_t *order;  // [B] sequences by decreasing page count: grid z -> sequence
-    const int32_t *tree;   // [T] tree verification: bit j = the token sees new token j; nullptr = causal
-    const float *k_scale;  // FP8 cache: [num_blocks][H_kv][16] scale of every stored K row
-    const float *v_scale;  // ... and V row
-    // shared-prefix decode
-    const int32_t *group_start;    // [n_groups + 1] the sequences of group v: [group_start[v], group_start[v+1])
-    const int32_t *prefix_blocks;  // [n_groups] blocks shared by group v at the head of its tables
-    int32_t *seq_prefix;           // [B] prefix blocks of each sequence's group (set by the plan kernel)
-    int n_groups;
-    int prefix_split_pages;  // pages per split of a prefix
-    int prefix_slots;        // workspace slots of the prefix splits (the sequences' own splits follow)
-    int32_t *status;
-    int64_t num_blocks;
-    int64_t T;
-    int max_blocks;
-    int B, H_q, H_kv, G;
-    int max_ctx;
-    int max_q_len;
-    int n_rg;         // row groups of 64 rows per (sequence, KV head)
-    int split_pages;  // pages per split
-    float scale_log2;  // scale * log2(e)
-};
 
 // Epilogue buffer of a rows CTA: partial O, max and sum of every warp's 16 rows.
 template <int D>
@@ -99,25 +58,6 @@ struct RowsSmem {
     static constexpr int kBytes = kFlagOff + 16;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (swizzle atoms)
 };
-
-__device__ __forceinline__ int seq_of_token(const int32_t *cu, int B, int64_t t)
-{
-    int lo = 0, hi = B;  // cu[lo] <= t < cu[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(cu + mid) <= t)
-            lo = mid;
-        else
-            hi = mid;
-    }
-    return lo;
-}
-
-// Sequence checks shared by the attention and merge kernels.
-__device__ __forceinline__ bool seq_ok(int qb, int ctx, const RowsParams &p, int64_t q1)
-{
-    return qb >= 1 && ctx >= qb && qb <= p.max_q_len && ctx <= p.max_ctx && ctx <= p.max_blocks * 16 && q1 <= p.T;
-}
 
 // One 16-key page for one warp: S = Q K^T for its m-tile (mma.sync m16n8k16 from ldmatrix of the
 // swizzled K page), mask, online softmax of its two rows, O += P V.  `kbase` and `vbase` are shared
@@ -317,8 +257,16 @@ __device__ __forceinline__ void rows_epilogue(float *e_o, const RowsParams &p, c
     }
 }
 
+// CTAs of the 16-bit rows kernel resident on an SM (sets the register budget), and its ring depth.
+#ifndef PA_ROWS_MIN_BLOCKS
+#define PA_ROWS_MIN_BLOCKS 3
+#endif
+#ifndef PA_ROWS_STAGES
+#define PA_ROWS_STAGES 2
+#endif
+
 template <int D, bool BF16, int STAGES, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, PA_ROWS_MIN_BLOCKS)
     pa_attn_rows_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                         const RowsParams p)
 {
@@ -341,59 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // ---- which (sequence, KV head, row group, split) --------------------------------
-    // Shared-prefix mode: grid z < n_groups is the prefix of group z -- every token of the
-    // group's sequences against the group's shared blocks, read once for all of them (no mask:
-    // the prefix precedes every new token); z >= n_groups is one sequence's own keys, from the
-    // first block after its group's prefix.
     const int split = blockIdx.x;
     const int g = blockIdx.y / p.n_rg, rg = blockIdx.y % p.n_rg;
-    int q0, q1, ctx, page_base = 0, sp = p.split_pages, slot0 = 0;
-    bool prefix_cta = false;
-    const int32_t *table;
-    if constexpr (MODE == kModeShared) {
-        const int sp_pre = p.prefix_split_pages;
-        if (static_cast<int>(blockIdx.z) < p.n_groups) {
-            // the group's arrays were checked by the plan kernel (status); clamp them here so a
-            // bad call stays inside its buffers
-            const int v = blockIdx.z;
-            const int s0 = min(max(__ldg(p.group_start + v), 0), p.B);
-            const int s1 = min(max(__ldg(p.group_start + v + 1), s0), p.B);
-            if (s0 >= s1)
-                return;
-            q0 = __ldg(p.cu_seqlens + s0);
-            q1 = max(__ldg(p.cu_seqlens + s1), q0);
-            ctx = min(max(__ldg(p.prefix_blocks + v), 0), min(p.max_blocks, p.prefix_slots * sp_pre)) * 16;
-            table = p.block_tables + (int64_t)s0 * p.max_blocks;
-            sp = p.prefix_split_pages;
-            prefix_cta = true;
-            if (q0 < 0 || q1 > p.T || ctx == 0)
-                return;
-        } else {
-            const int b = __ldg(p.order + (blockIdx.z - p.n_groups));
-            q0 = __ldg(p.cu_seqlens + b);
-            q1 = __ldg(p.cu_seqlens + b + 1);
-            ctx = __ldg(p.context_lens + b);
-            if (!seq_ok(q1 - q0, ctx, p, q1)) {
-                if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
-                    set_status(p.status, PA_ERR_SEQ);
-                return;
-            }
-            table = p.block_tables + (int64_t)b * p.max_blocks;
-            page_base = min(max(__ldg(p.seq_prefix + b), 0), (ctx - (q1 - q0)) / 16);
-            slot0 = p.prefix_slots;
-        }
-    } else {
-        const int b = __ldg(p.order + blockIdx.z);
-        q0 = __ldg(p.cu_seqlens + b);
-        q1 = __ldg(p.cu_seqlens + b + 1);
-        ctx = __ldg(p.context_lens + b);
-        if (!seq_ok(q1 - q0, ctx, p, q1)) {
-            if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0)
-                set_status(p.status, PA_ERR_SEQ);
-            return;
-        }
-        table = p.block_tables + (int64_t)b * p.max_blocks;
-    }
+    DecodeUnit u;
+    if (!decode_unit<MODE>(p, tid, u))
+        return;
+    const int q0 = u.q0, q1 = u.q1, ctx = u.ctx, page_base = u.page_base, sp = u.sp, slot0 = u.slot0;
+    const bool prefix_cta = u.prefix_cta;
+    const int32_t *table = u.table;
     const int qb = q1 - q0;
     const int G = p.G;
     const int R = G * qb;
@@ -605,9 +508,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // fp32 scores (K) and the probabilities before P V (V).  Pipeline and epilogue as the 16-bit
 // kernel: a four-stage TMA ring (one 16 x d-byte box per page for K and one for V), refilled by
 // the last warp done with a stage.
+#ifndef PA_FP8_NARROW_STAGES
+#define PA_FP8_NARROW_STAGES 2
+#endif
+#ifndef PA_FP8_NARROW_CTAS
+#define PA_FP8_NARROW_CTAS 5
+#endif
 constexpr int kFp8Stages = 4;
-constexpr int kNarrowStages = 3;     // narrow variant: a shallower ring ...
-constexpr int kNarrowCtasPerSm = 4;  // ... and more CTAs on an SM
+constexpr int kNarrowStages = PA_FP8_NARROW_STAGES;  // narrow variant: a shallower ring ...
+constexpr int kNarrowCtasPerSm = PA_FP8_NARROW_CTAS;  // ... and more CTAs on an SM
 
 // Epilogue buffer of a narrow FP8 CTA: O^T, max and sum of every warp's 8 rows.
 template <int D>
@@ -1298,15 +1207,26 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
     }
 }
 
-// Shared-prefix decode, before the rows kernel: seq_prefix[b] = the prefix blocks of sequence b's
-// group, or 0 where the shared pass must not be used for b -- its table does not start with the
-// group leader's prefix blocks, or the prefix reaches its new tokens; such a sequence is computed
-// over its own table alone (the result is the same).  Malformed groups (not a partition of the
-// sequences into consecutive runs, a prefix outside the table, more new tokens than the rows
-// planned for a group, a prefix longer than the planned bound) set PA_ERR_ARG and turn every
-// sequence into the unshared case.
-__global__ void __launch_bounds__(1024) pa_shared_plan_kernel(const RowsParams p)
+// Shared-prefix decode, before the rows kernel (one CTA): the longest-first order of the
+// sequences, the checks of the groups and, with fill_prefix, seq_prefix[b] = the prefix blocks of
+// sequence b's group, or 0 where the shared pass must not be used for b -- its table does not
+// start with the group leader's prefix blocks, or the prefix reaches its new tokens; such a
+// sequence is computed over its own table alone (the result is the same).  Malformed groups (not a
+// partition of the sequences into consecutive runs, a prefix outside the table, more new tokens
+// than the rows planned for a group, a prefix longer than the planned bound) set PA_ERR_ARG and
+// turn every sequence into the unshared case.
+__global__ void __launch_bounds__(kOrderThreads) pa_shared_plan_kernel(const RowsParams p, int32_t *order,
+                                                                         int fill_prefix)
 {
+    // first the longest-first order of the sequences (as pa_seq_order_kernel), in this same launch
+    order_by_key_desc(
+        p.B,
+        [&](int b) {
+            const int ctx = __ldg(p.context_lens + b);
+            const int pages = ctx > 0 ? (ctx + 15) / 16 : 0;
+            return min(pages, kOrderKeys - 1);
+        },
+        order);
     __shared__ int bad;
     const int tid = threadIdx.x;
     if (tid == 0)
@@ -1325,11 +1245,15 @@ __global__ void __launch_bounds__(1024) pa_shared_plan_kernel(const RowsParams p
     if (bad) {
         if (tid == 0)
             set_status(p.status, PA_ERR_ARG);
-        for (int b = tid; b < p.B; b += blockDim.x)
+        for (int b = tid; b < p.B && fill_prefix; b += blockDim.x)
             p.seq_prefix[b] = 0;
         return;
     }
-    for (int b = tid; b < p.B; b += blockDim.x) {
+    if (!fill_prefix)  // the plain decode computes the result: only the checks above are wanted
+        return;
+    // one warp per sequence: its lanes compare the prefix entries with the leader's side by side
+    const int lane = tid & 31;
+    for (int b = tid >> 5; b < p.B; b += blockDim.x >> 5) {
         // b's group: the last v with group_start[v] <= b (groups may be empty)
         int lo = 0, hi = p.n_groups - 1;
         while (lo < hi) {
@@ -1342,19 +1266,26 @@ __global__ void __launch_bounds__(1024) pa_shared_plan_kernel(const RowsParams p
         const int s0 = __ldg(p.group_start + lo);
         const int P = __ldg(p.prefix_blocks + lo);
         const int q_b = __ldg(p.cu_seqlens + b + 1) - __ldg(p.cu_seqlens + b);
-        int use = (int64_t)P * 16 <= (int64_t)__ldg(p.context_lens + b) - q_b ? P : 0;
+        const int use = (int64_t)P * 16 <= (int64_t)__ldg(p.context_lens + b) - q_b ? P : 0;
         const int32_t *mine = p.block_tables + (int64_t)b * p.max_blocks;
         const int32_t *lead = p.block_tables + (int64_t)s0 * p.max_blocks;
-        for (int i = 0; i < use; ++i)
-            if (__ldg(mine + i) != __ldg(lead + i))
-                use = 0;
-        p.seq_prefix[b] = use;
+        bool same = true;
+        for (int i = lane; i < use; i += 32)
+            same &= __ldg(mine + i) == __ldg(lead + i);
+        same = __all_sync(0xffffffffu, same);
+        if (lane == 0)
+            p.seq_prefix[b] = same ? use : 0;
     }
 }
 
 // ---- host side ------------------------------------------------------------------------------
 
-constexpr int kStages = 3;
+constexpr int kStages = PA_ROWS_STAGES;
+// Rows per (sequence, KV head) from which a 16-bit decode goes to the tcgen05 rows kernel.
+#ifndef PA_WIDE_ROWS
+#define PA_WIDE_ROWS 16
+#endif
+constexpr int kWideRows = PA_WIDE_ROWS;
 
 template <int D, bool BF16, int MODE>
 static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
@@ -1440,6 +1371,11 @@ static int split_pages_override()
     return v;
 }
 
+// Decode CTAs the split planner counts on per SM.
+#ifndef PA_PLAN_CTAS_PER_SM
+#define PA_PLAN_CTAS_PER_SM 3
+#endif
+
 DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
 {
     DecodePlan pl;
@@ -1452,7 +1388,7 @@ DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
     // splits mean fewer CTAs and less fixed cost; the wave count rounds up, so a split that fills
     // the last wave beats a slightly shorter one that leaves it nearly empty.
     const int64_t units = (int64_t)B * H_kv * pl.row_groups;
-    const int64_t slots = (int64_t)sm_count() * 2;
+    const int64_t slots = (int64_t)sm_count() * PA_PLAN_CTAS_PER_SM;
     const int64_t page_bytes = 2 * 16 * (int64_t)d * 2;
     const int64_t cta_cost = (80 * 1024 + page_bytes - 1) / page_bytes;
     int64_t sp = kMaxTablePages, best = -1;
@@ -1521,6 +1457,24 @@ size_t shared_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
     return PA_STATUS_BYTES + 2 * seq_order_bytes(B) + rows * d * sizeof(float) + rows * sizeof(float) + 256;
 }
 
+// Does the shared-prefix pass pay for itself?  Reading a group's prefix once saves (n - 1) / n of
+// the prefix keys of a group of n sequences, about (n - 1) / n x prefix / context of the keys the
+// batch reads; the pass costs the prefix CTAs (a whole group's rows on every prefix page), a
+// partial output for every row and the merge.  Below a quarter of the keys saved it loses to the
+// plain decode, which also finds repeated prefix blocks in L2 (measured: 16 sequences sharing 2048
+// of 32768 tokens, 6 % of the keys: 0.89x the plain decode; 64 requests in groups of 16 sharing
+// 4096 of <= 4608 tokens, 83 %: 4.7x).  Host bounds only: mean group size B / n_groups, prefix
+// max_prefix_blocks, context max_ctx (an overestimate, so the plain path is taken when unsure).
+static bool shared_pass_pays(const AttnArgs &a)
+{
+    if (a.n_groups < 1 || a.max_ctx < 1 || a.max_prefix_blocks < 1)
+        return false;
+    const double n = static_cast<double>(a.B) / a.n_groups;
+    const double prefix = 16.0 * a.max_prefix_blocks;
+    const double saved = (n - 1.0) / n * (prefix < a.max_ctx ? prefix : a.max_ctx) / a.max_ctx;
+    return saved >= 0.25;
+}
+
 template <int D, bool BF16>
 static int run(const AttnArgs &a)
 {
@@ -1576,16 +1530,33 @@ static int run(const AttnArgs &a)
         if (z > 65535 || (int64_t)a.H_kv * sp.row_groups > 65535)
             return PA_ERR_UNSUPPORTED;
         dim3 grid(max(sp.own.max_splits, sp.prefix_slots), a.H_kv * sp.row_groups, static_cast<unsigned>(z));
-        pa_shared_plan_kernel<<<1, 1024, 0, a.stream>>>(rp);
+        // one launch writes the sequence order and checks the groups (status), whichever path
+        // computes the result
+        const bool pays = shared_pass_pays(a);
+        pa_shared_plan_kernel<<<1, kOrderThreads, 0, a.stream>>>(rp, order, pays ? 1 : 0);
         count_launch();
         rc = cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-        if (rc == PA_OK)
-            rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
-        if (rc == PA_OK)
-            rc = launch_rows<D, BF16, kModeShared>(rp, tk, tv, grid, a.stream);
-        if (rc == PA_OK)
-            rc = launch_merge<D, BF16>(rp, a.stream);
-        return rc;
+        if (rc != PA_OK)
+            return rc;
+        if (pays) {
+            // (the prefix rows of a group stay on the mma.sync kernel: with three CTAs per SM it
+            // beat the tcgen05 rows kernel on the prefix pass, which it shares one launch with)
+            if (rc == PA_OK)
+                rc = launch_rows<D, BF16, kModeShared>(rp, tk, tv, grid, a.stream);
+            if (rc == PA_OK)
+                rc = launch_merge<D, BF16>(rp, a.stream);
+            return rc;
+        }
+        // the plain decode over the same tables: its workspace (status, order, partials) is no
+        // larger than this one and starts at the same place (the plan kernel wrote no per-sequence
+        // prefix lengths)
+        rp.group_start = nullptr;
+        rp.prefix_blocks = nullptr;
+        rp.seq_prefix = nullptr;
+        rp.n_groups = 0;
+        rp.prefix_slots = 0;
+        rp.ws_o = nullptr;
+        rp.ws_lse = nullptr;
     }
     {
         const DecodePlan pl = decode_plan(a.B, a.H_q, a.H_kv, a.d, a.max_ctx);
@@ -1602,13 +1573,30 @@ static int run(const AttnArgs &a)
         if (a.B > 65535 || (int64_t)a.H_kv * pl.row_groups > 65535)
             return PA_ERR_UNSUPPORTED;
         dim3 grid(pl.max_splits, a.H_kv * pl.row_groups, a.B);
-        rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
-        if (rc == PA_OK)
+        // 16-bit cache where every sequence has 16 or more rows per KV head (G query heads x its
+        // new tokens, at least T - 8 (B - 1) of them): the tcgen05 rows kernel.  A batch that
+        // mixes narrow and wide sequences stays on the mma.sync kernel: one launch over all of
+        // them beats two launches in a row (measured on the mixed continuous-batching step).
+        const int64_t max_q = std::min<int64_t>(8, a.T - a.B + 1);
+        const int64_t min_q = std::max<int64_t>(1, a.T - 8 * (int64_t)(a.B - 1));
+        const int tc_rows = rows_tc_rows_per_cta(rp.G, static_cast<int>(max_q));
+        const bool all_wide = !fp8 && tc_rows > 0 && (int64_t)rp.G * min_q >= kWideRows;
+        if (!a.group_start)  // the shared-prefix call's plan kernel has written the order already
+            rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
+        if (rc == PA_OK && all_wide) {
+            RowsParams rt = rp;
+            rt.n_rg = static_cast<int>(((int64_t)rp.G * max_q + tc_rows - 1) / tc_rows);
+            const dim3 grid_tc(pl.max_splits, a.H_kv * rt.n_rg, a.B);
+            rc = launch_rows_tc(rt, tk, tv, D, a.dtype, rp.tree ? kModeTree : kModeCausal, tc_rows, grid_tc,
+                                a.stream);
+        }
+        if (rc == PA_OK && !all_wide) {
             // single-token decode with at most 8 query heads per KV head: keys on the MMA's M side
             rc = fp8 && a.T == a.B && rp.G <= 8 ? launch_rows_fp8<D, BF16, true>(rp, tk, tv, grid, a.stream)
                  : fp8     ? launch_rows_fp8<D, BF16, false>(rp, tk, tv, grid, a.stream)
                  : rp.tree ? launch_rows<D, BF16, kModeTree>(rp, tk, tv, grid, a.stream)
                            : launch_rows<D, BF16, kModeCausal>(rp, tk, tv, grid, a.stream);
+        }
         if (rc == PA_OK && pl.max_splits > 1)
             rc = launch_merge<D, BF16>(rp, a.stream);
         return rc;

@@ -272,6 +272,45 @@ def test_tree_verify_small(idx):
     assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
 
 
+# Every sequence with 16 or more rows per KV head (G x its new tokens): the calls run on the
+# tcgen05 rows kernel (rows on the MMA's M side, 64-key tiles, S double-buffered in TMEM).
+# (B, q_b of every sequence or None = random 1..8, ctx_max, H_kv, G, d, dtype, tree)
+WIDE_CASES = [
+    (5, 4, 700, 2, 4, 128, W.BF16, False),    # 16 rows, one warp's worth
+    (4, 8, 2000, 1, 8, 64, W.F16, False),     # 64 rows, several splits
+    (3, None, 300, 2, 16, 128, W.BF16, False),  # 16..128 rows (G = 16 is wide for any q_b)
+    (4, 8, 1500, 2, 2, 128, W.F16, True),     # tree masks, 16 rows, splits
+    (3, 6, 60, 2, 4, 64, W.BF16, True),       # tree masks, tiny contexts and partial pages
+    (2, 8, 500, 1, 32, 128, W.BF16, False),   # 256 rows: two row groups of 128
+    (3, 8, 400, 2, 3, 64, W.F16, False),      # G = 3: 24 rows per CTA
+]
+
+
+def _wide_id(c):
+    return "B{}q{}c{}h{}g{}d{}{}{}".format(c[0], c[1] or "r", c[2], c[3], c[4], c[5],
+                                          "bf16" if c[6] == W.BF16 else "f16", "tree" if c[7] else "")
+
+
+@pytest.mark.parametrize("idx", range(len(WIDE_CASES)), ids=lambda i: _wide_id(WIDE_CASES[i]))
+def test_decode_wide_rows_tensor_cores(idx):
+    B, q, ctx_max, H_kv, G, d, dt, tree = WIDE_CASES[idx]
+    g = torch.Generator().manual_seed(900 + idx)
+    q_lens = [q if q else int(torch.randint(1, 9, (1,), generator=g)) for _ in range(B)]
+    ctx_lens = [int(torch.randint(qb, ctx_max + 1, (1,), generator=g)) for qb in q_lens]
+    w = W.build_workload(f"wide{idx}", q_lens=q_lens, ctx_lens=ctx_lens, H_q=H_kv * G, H_kv=H_kv, d=d, dtype=dt,
+                         seed=910 + idx, calls=[W.AttnCall("decode", 0, B)], pool_extra=3)
+    if tree:
+        tm = W.random_tree_masks(920 + idx, w.q_lens)
+        out, _ = _tree_run(w, tm)  # checks the status words
+        ref, _, _ = oracle_step(w, oracle.lib(), tree_mask=tm)
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        err = np.abs(got - ref).max()
+        assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
+    else:
+        run_and_compare(w)
+
+
 def test_tree_chain_mask_is_the_causal_verify():
     # the chain mask takes exactly the decisions of the causal rule: the same bits out
     w = W.random_workload(71, B=5, q_max=8, ctx_max=900, H_kv=2, G=4, d=128, dtype=W.BF16, kind="decode")
@@ -639,7 +678,7 @@ SHARED_CASES = [
     (8, 3, 64, (1, 40), 3, 8, 2, 64, W.F16),          # ragged verify rows, GQA 4
     (6, 2, 256, (16, 300), 1, 4, 4, 128, W.BF16),     # MHA decode
     (16, 1, 2048, (1, 100), 2, 32, 8, 128, W.BF16),   # one group, long prefix (several prefix splits), 2 row groups
-    (20, 4, 512, (1, 2000), 1, 16, 2, 128, W.F16),    # long own keys: several splits of their own
+    (20, 4, 512, (1, 1000), 1, 16, 2, 128, W.F16),    # long own keys: several splits of their own
     (3, 3, 32, (5, 9), 4, 2, 1, 64, W.BF16),          # one sequence per group
 ]
 
