@@ -21,8 +21,8 @@
 //     softmax of tile j runs, so the softmax never waits for a product;
 //   * one thread per row (warps 4-7, TMEM lane = row; a warp without a row sits out) loads its S
 //     row, masks, keeps m and l, and writes P (16-bit) back over S; O += P V with P from TMEM and
-//     V (MN-major) from shared memory, fp32 in TMEM; O is rescaled only when a row's max grows by more than 2^8 (after the
-//     products already issued for that row have completed);
+//     V (MN-major) from shared memory, fp32 in TMEM; O is rescaled only when a row's max grows by
+//     more than 2^8 (after the products already issued for that row have completed);
 //   * warp 0 loads Q and feeds the K tiles, warp 2 the V tiles (lanes 0-3 one page each; K of a
 //     tile is released once its S is complete, V once its P V is), warp 1 issues the MMAs (one
 //     thread).
@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // ---- the CTA's rows and keys (uniform over the CTA: early returns precede every barrier) ----
     const int split = blockIdx.x;
-    const int g = blockIdx.y / p.n_rg, rg = blockIdx.y % p.n_rg;
+    // the heaviest row groups (the last tokens, which see the most keys) are dispatched first
+    const int g = blockIdx.y / p.n_rg, rg = p.n_rg - 1 - static_cast<int>(blockIdx.y % p.n_rg);
     DecodeUnit u;
     if (!decode_unit<MODE>(p, tid, u))
         return;
