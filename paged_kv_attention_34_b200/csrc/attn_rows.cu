@@ -287,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, PA_ROWS_MIN_BLOCKS)
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_wait();     // the sequence order comes from the kernel before this one
+    griddep_release();  // the split merge after this kernel may be scheduled (it waits for this grid)
 
     // ---- which (sequence, KV head, row group, split) --------------------------------
     const int split = blockIdx.x;
@@ -886,6 +888,8 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
     volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_wait();     // the sequence order comes from the kernel before this one
+    griddep_release();  // the split merge after this kernel may be scheduled (it waits for this grid)
 
     // ---- which (sequence, KV head, row group, split): as the 16-bit kernel ----------------
     const int b = __ldg(p.order + blockIdx.z);
@@ -1149,6 +1153,7 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
 {
+    griddep_wait();  // the partials of the attention kernel
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 8 + warp;
     if (row >= p.T * p.H_q)
@@ -1218,6 +1223,10 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
 __global__ void __launch_bounds__(kOrderThreads) pa_shared_plan_kernel(const RowsParams p, int32_t *order,
                                                                          int fill_prefix)
 {
+    if (threadIdx.x == 0)
+        *p.status = PA_OK;  // the call's status word: this is its first kernel
+    __syncthreads();        // before any thread records a malformed group
+    griddep_release();      // the attention kernel waits for the order and the group checks
     // first the longest-first order of the sequences (as pa_seq_order_kernel), in this same launch
     order_by_key_desc(
         p.B,
@@ -1303,9 +1312,10 @@ static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtens
             return PA_ERR_CUDA;
         configured |= bit;
     }
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(tk, tv, rp);
+    const cudaError_t e = launch_dependent(kern, grid, dim3(kThreads), L::kAlloc, stream, tk, tv, rp);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 template <int D, bool BF16, bool NARROW>
@@ -1324,16 +1334,21 @@ static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CU
             return PA_ERR_CUDA;
         configured |= bit;
     }
-    kern<<<grid, kThreads, L::kAlloc, stream>>>(tk, tv, rp);
+    const cudaError_t e = launch_dependent(kern, grid, dim3(kThreads), L::kAlloc, stream, tk, tv, rp);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // Longest sequences first: decode CTAs are dispatched in grid order, so putting the sequences with
 // the most pages at the front leaves short CTAs for the last wave (longest-processing-time-first
 // list scheduling; the order among equal page counts is arbitrary and changes no result).
-__global__ void __launch_bounds__(kOrderThreads) pa_seq_order_kernel(const int32_t *context_lens, int B, int32_t *order)
+__global__ void __launch_bounds__(kOrderThreads)
+    pa_seq_order_kernel(const int32_t *context_lens, int B, int32_t *order, int32_t *status)
 {
+    if (threadIdx.x == 0)
+        *status = PA_OK;  // the call's status word: this is its first kernel
+    griddep_release();    // the attention kernel's CTAs may be scheduled now; they wait for the order
     order_by_key_desc(
         B,
         [&](int b) {
@@ -1344,9 +1359,9 @@ __global__ void __launch_bounds__(kOrderThreads) pa_seq_order_kernel(const int32
         order);
 }
 
-int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, cudaStream_t stream)
+int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, cudaStream_t stream)
 {
-    pa_seq_order_kernel<<<1, kOrderThreads, 0, stream>>>(context_lens, B, order);
+    pa_seq_order_kernel<<<1, kOrderThreads, 0, stream>>>(context_lens, B, order, status);
     count_launch();
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -1356,9 +1371,11 @@ static int launch_merge(const RowsParams &rp, cudaStream_t stream)
 {
     const int64_t rows = rp.T * rp.H_q;
     const int64_t blocks = (rows + 7) / 8;
-    pa_split_merge_kernel<D, BF16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(rp);
+    const cudaError_t e =
+        launch_dependent(pa_split_merge_kernel<D, BF16>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream, rp);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 static int split_pages_override()
@@ -1582,7 +1599,7 @@ static int run(const AttnArgs &a)
         const int tc_rows = rows_tc_rows_per_cta(rp.G, static_cast<int>(max_q));
         const bool all_wide = !fp8 && tc_rows > 0 && (int64_t)rp.G * min_q >= kWideRows;
         if (!a.group_start)  // the shared-prefix call's plan kernel has written the order already
-            rc = launch_seq_order(a.context_lens, a.B, order, a.stream);
+            rc = launch_seq_order(a.context_lens, a.B, order, rp.status, a.stream);
         if (rc == PA_OK && all_wide) {
             RowsParams rt = rp;
             rt.n_rg = static_cast<int>(((int64_t)rp.G * max_q + tc_rows - 1) / tc_rows);

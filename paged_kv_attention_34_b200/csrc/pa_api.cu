@@ -169,10 +169,9 @@ extern "C" int pa_paged_attn_decode(void *out, const void *q, const void *key_ca
         return rc;
     if (workspace_bytes < decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx))
         return PA_ERR_WORKSPACE;
-    rc = reset_status(workspace, a.stream);
-    if (rc != PA_OK || B == 0 || T == 0)
-        return rc;
-    return launch_decode(a);
+    if (B == 0 || T == 0)
+        return reset_status(workspace, a.stream);  // nothing to launch
+    return launch_decode(a);  // its first kernel clears the status word
 }
 
 extern "C" int pa_paged_attn_decode_tree(void *out, const void *q, const void *key_cache, const void *value_cache,
@@ -197,10 +196,9 @@ extern "C" int pa_paged_attn_decode_tree(void *out, const void *q, const void *k
     }
     if (workspace_bytes < decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx))
         return PA_ERR_WORKSPACE;
-    rc = reset_status(workspace, a.stream);
-    if (rc != PA_OK || B == 0 || T == 0)
-        return rc;
-    return launch_decode(a);
+    if (B == 0 || T == 0)
+        return reset_status(workspace, a.stream);  // nothing to launch
+    return launch_decode(a);  // its first kernel clears the status word
 }
 
 extern "C" size_t pa_shared_prefix_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx,
@@ -246,10 +244,9 @@ extern "C" int pa_paged_attn_decode_shared_prefix(void *out, const void *q, cons
     if (workspace_bytes <
         shared_workspace_bytes(T, B, H_q, H_kv, d, max_ctx, n_groups, max_prefix_blocks, max_group_tokens))
         return PA_ERR_WORKSPACE;
-    rc = reset_status(workspace, a.stream);
-    if (rc != PA_OK || B == 0 || T == 0)
-        return rc;
-    return launch_decode(a);
+    if (B == 0 || T == 0)
+        return reset_status(workspace, a.stream);  // nothing to launch
+    return launch_decode(a);  // its first kernel clears the status word
 }
 
 extern "C" int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t *key_cache,
@@ -274,10 +271,9 @@ extern "C" int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t 
     }
     if (workspace_bytes < decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx))
         return PA_ERR_WORKSPACE;
-    rc = reset_status(workspace, a.stream);
-    if (rc != PA_OK || B == 0 || T == 0)
-        return rc;
-    return launch_decode(a);
+    if (B == 0 || T == 0)
+        return reset_status(workspace, a.stream);  // nothing to launch
+    return launch_decode(a);  // its first kernel clears the status word
 }
 
 extern "C" size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len)
@@ -302,10 +298,9 @@ extern "C" int pa_paged_attn_prefill(void *out, const void *q, const void *key_c
         return rc;
     if (workspace_bytes < pa_prefill_workspace_bytes(B, H_q, H_kv, d, max_q_len))
         return PA_ERR_WORKSPACE;
-    rc = reset_status(workspace, a.stream);
-    if (rc != PA_OK || B == 0 || T == 0)
-        return rc;
-    return launch_prefill(a);
+    if (B == 0 || T == 0)
+        return reset_status(workspace, a.stream);  // nothing to launch
+    return launch_prefill(a);  // its first kernel clears the status word
 }
 
 extern "C" int pa_read_status(const void *workspace, int32_t *host_status, void *stream)

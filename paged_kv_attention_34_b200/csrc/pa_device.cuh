@@ -106,6 +106,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------
+// griddep_wait: in a kernel started by launch_dependent, returns once the kernel before it on the
+// stream has completed and its writes are visible (at once for a kernel launched the ordinary
+// way).  griddep_release: lets the kernel after this one on the stream be scheduled early.
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- TMA ------------------------------------------------------------------------
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m)

@@ -24,6 +24,30 @@ struct CallRange {
 // Counts every kernel launch of the library (pa_launch_count).
 void count_launch(uint64_t n = 1);
 
+// Launches `kern` as a programmatic dependent of the kernel before it on `stream` (a kernel of the
+// same library call): its CTAs may be scheduled while that kernel still runs and must call
+// griddep_wait() before they read anything it writes.  Hides the launch latency between the
+// kernels of one call.
+#ifndef PA_DEPENDENT_LAUNCH
+#define PA_DEPENDENT_LAUNCH 1
+#endif
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args &&...args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = PA_DEPENDENT_LAUNCH;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // True when p is non-null and 16-byte aligned.
 inline bool aligned16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -106,9 +130,10 @@ size_t shared_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
                               int max_prefix_blocks, int max_group_tokens);
 
 // Sequence order by decreasing page count (one CTA, on `stream`): order[r] = the sequence of rank r.
-// The workspace holds it right after the status area, seq_order_bytes(B) bytes.
+// The workspace holds it right after the status area, seq_order_bytes(B) bytes.  The kernel is the
+// first of its call and also clears the call's status word.
 size_t seq_order_bytes(int B);
-int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, cudaStream_t stream);
+int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, cudaStream_t stream);
 int launch_decode(const AttnArgs &a);
 size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int max_q_len);
 int launch_prefill(const AttnArgs &a);

@@ -148,8 +148,14 @@ __device__ __forceinline__ int pair_kv_tiles(int pair, int qb, int ctx, int tok_
 // K/V tiles, so the heaviest items are drawn first and short ones fill the end.
 __global__ void __launch_bounds__(kOrderThreads) pa_prefill_order_kernel(const int32_t *cu_seqlens,
                                                                            const int32_t *context_lens, int B,
-                                                                           int n_pairs, int tok_per_tile, int32_t *order)
+                                                                           int n_pairs, int tok_per_tile, int32_t *order,
+                                                                           int *counter, int32_t *status)
 {
+    if (threadIdx.x == 0) {
+        *status = PA_OK;  // the call's status word: this is its first kernel
+        *counter = 0;     // the work counter the attention kernel's CTAs draw items from
+    }
+    griddep_release();  // the attention kernel's CTAs may be scheduled now; they wait for this grid
     order_by_key_desc(
         n_pairs * B,
         [&](int e) {
@@ -225,6 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kTmemCols = 512;
     // TMEM columns: S_A, S_B (P written over their first 64 columns), O_A, O_B
 
+    griddep_wait();  // the item order and the zeroed work counter come from the order kernel
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBars);
@@ -790,10 +797,8 @@ static int run(const AttnArgs &a)
         rc = make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
     if (rc != PA_OK)
         return rc;
-    if (cudaMemsetAsync(p.counter, 0, sizeof(int), a.stream) != cudaSuccess)
-        return PA_ERR_CUDA;
     pa_prefill_order_kernel<<<1, kOrderThreads, 0, a.stream>>>(a.cu_seqlens_q, a.context_lens, a.B, p.n_pairs_max,
-                                                                 p.tok_per_tile, order);
+                                                                 p.tok_per_tile, order, p.counter, p.status);
     count_launch();
     if (cudaGetLastError() != cudaSuccess)
         return PA_ERR_CUDA;
@@ -817,9 +822,10 @@ static int run(const AttnArgs &a)
         configured |= bit;
     }
     const int grid = static_cast<int>(std::min<int64_t>(items, sm_count()));
-    kern<<<grid, kThreads, L::kAlloc, a.stream>>>(tq, tk, tv, p);
+    const cudaError_t e = launch_dependent(kern, dim3(grid), dim3(kThreads), L::kAlloc, a.stream, tq, tk, tv, p);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace tcp

@@ -133,6 +133,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tail + 8 * L::kNumBars + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    griddep_wait();     // the sequence order comes from the kernel before this one
+    griddep_release();  // the split merge after this kernel may be scheduled (it waits for this grid)
 
     // ---- the CTA's rows and keys (uniform over the CTA: early returns precede every barrier) ----
     const int split = blockIdx.x;
@@ -500,9 +502,11 @@ static int launch(const RowsParams &rp, const CUtensorMap &tq, const CUtensorMap
     if (bytes > kSmemPerCta)
         return PA_ERR_UNSUPPORTED;
     const int oob_row = static_cast<int>(rp.num_blocks * rp.H_kv * 16);
-    kern<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, rp, rows_per_cta, n_st, oob_row);
+    const cudaError_t e =
+        launch_dependent(kern, grid, dim3(kThreads), bytes, stream, tq, tk, tv, rp, rows_per_cta, n_st, oob_row);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace rtc

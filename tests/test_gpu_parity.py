@@ -311,6 +311,51 @@ def test_decode_wide_rows_tensor_cores(idx):
         run_and_compare(w)
 
 
+# Split-KV decode with a workspace that starts as garbage and an output that starts as NaN: every
+# sequence has several KV splits, so the order, the partials and the merge all go through the
+# workspace; a row the merge misses stays NaN, and a second call on the same (now used) workspace
+# must give the same bytes.  (name, q_lens, ctx_lens, H_kv, G, d, dtype, tree)
+MERGE_CASES = [
+    ("mma_sync_many_splits", [1, 1, 1], [9000, 5000, 300], 2, 1, 128, W.F16, False),
+    ("mma_sync_verify_rows", [3, 5], [4000, 7000], 2, 4, 128, W.BF16, False),
+    ("tcgen05_rows", [8, 8], [6000, 2500], 2, 4, 128, W.BF16, False),
+    ("tcgen05_tree", [8, 8, 8], [3000, 5000, 40], 1, 2, 64, W.F16, True),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(MERGE_CASES)), ids=lambda i: MERGE_CASES[i][0])
+def test_split_decode_with_a_dirty_workspace(idx):
+    name, q_lens, ctx_lens, H_kv, G, d, dt, tree = MERGE_CASES[idx]
+    w = W.build_workload(f"merge{idx}", q_lens=q_lens, ctx_lens=ctx_lens, H_q=H_kv * G, H_kv=H_kv, d=d, dtype=dt,
+                         seed=1300 + idx, calls=[W.AttnCall("decode", 0, len(q_lens))], pool_extra=3)
+    st = DeviceStep(w)
+    st.copy_blocks()
+    st.write()
+    call = st.calls[0]
+    nbytes = pa.decode_workspace_bytes(call.q.shape[0], w.B, w.H_q, w.H_kv, w.d, call.max_ctx)
+    assert nbytes > pa.PA_STATUS_BYTES + 256  # the plan splits these contexts
+    ws = torch.full((nbytes,), 0x5A, dtype=torch.uint8, device="cuda")
+    tm = W.random_tree_masks(1310 + idx, w.q_lens) if tree else None
+    outs = []
+    for _ in range(2):
+        out = torch.full_like(call.q, float("nan"))
+        if tree:
+            pa.paged_attn_decode_tree(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, tm.cuda(),
+                                      call.max_ctx, w.scale, out=out, workspace=ws)
+        else:
+            pa.paged_attn_decode(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, call.max_ctx,
+                                 w.scale, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        assert pa.read_status(ws) == 0
+        outs.append(out)
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    ref, _, _ = oracle_step(w, oracle.lib(), tree_mask=tm) if tree else oracle_step(w, oracle.lib())
+    got = outs[0].double().cpu().numpy()
+    assert np.isfinite(got).all()
+    err = np.abs(got - ref).max()
+    assert err <= TOL[w.dtype], f"max abs err {err:.3e}"
+
+
 def test_tree_chain_mask_is_the_causal_verify():
     # the chain mask takes exactly the decisions of the causal rule: the same bits out
     w = W.random_workload(71, B=5, q_max=8, ctx_max=900, H_kv=2, G=4, d=128, dtype=W.BF16, kind="decode")
