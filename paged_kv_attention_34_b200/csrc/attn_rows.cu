@@ -1393,21 +1393,14 @@ static int split_pages_override()
 #define PA_PLAN_CTAS_PER_SM 3
 #endif
 
-DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
+// Pages per split for `units` independent (sequence, KV head, row group) units of up to `pages`
+// pages on `slots` resident CTAs: the multiple of the stage size in [16, kMaxTablePages] that
+// minimises the time of a batch whose every unit has `pages` pages, modelled as (full waves of
+// CTAs) x (split length + a fixed per-CTA cost of `cta_cost` pages).  Longer splits mean fewer CTAs
+// and less fixed cost; the wave count rounds up, so a split that fills the last wave beats a
+// slightly shorter one that leaves it nearly empty.
+static int plan_split_pages(int64_t units, int64_t pages, int64_t slots, int64_t cta_cost)
 {
-    DecodePlan pl;
-    const int G = H_q / H_kv;
-    pl.row_groups = (8 * G + kRowsPerCta - 1) / kRowsPerCta;
-    const int64_t pages = (int64_t)(max_ctx + 15) / 16;
-    // Pages per split: the multiple of the stage size in [16, kMaxTablePages] that minimises the
-    // time of a batch whose every sequence has max_ctx keys, modelled as (full waves of CTAs over
-    // 2 per SM) x (split length + a per-CTA cost of ~80 KB of streaming, in pages).  Longer
-    // splits mean fewer CTAs and less fixed cost; the wave count rounds up, so a split that fills
-    // the last wave beats a slightly shorter one that leaves it nearly empty.
-    const int64_t units = (int64_t)B * H_kv * pl.row_groups;
-    const int64_t slots = (int64_t)sm_count() * PA_PLAN_CTAS_PER_SM;
-    const int64_t page_bytes = 2 * 16 * (int64_t)d * 2;
-    const int64_t cta_cost = (80 * 1024 + page_bytes - 1) / page_bytes;
     int64_t sp = kMaxTablePages, best = -1;
     for (int64_t c = kMaxTablePages; c >= 16 && units > 0 && pages > 0; c -= kPagesPerStage) {
         const int64_t ctas = units * ((pages + c - 1) / c);
@@ -1419,10 +1412,42 @@ DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
             sp = c;
         }
     }
+    return static_cast<int>(sp);
+}
+
+DecodePlan decode_plan(int B, int H_q, int H_kv, int d, int max_ctx)
+{
+    DecodePlan pl;
+    const int G = H_q / H_kv;
+    pl.row_groups = (8 * G + kRowsPerCta - 1) / kRowsPerCta;
+    const int64_t pages = (int64_t)(max_ctx + 15) / 16;
+    // the mma.sync kernels: PA_PLAN_CTAS_PER_SM CTAs per SM, a per-CTA cost of ~80 KB of streaming
+    const int64_t page_bytes = 2 * 16 * (int64_t)d * 2;
+    const int64_t cta_cost = (80 * 1024 + page_bytes - 1) / page_bytes;
+    int64_t sp = plan_split_pages((int64_t)B * H_kv * pl.row_groups, pages, (int64_t)sm_count() * PA_PLAN_CTAS_PER_SM,
+                                  cta_cost);
     const int ov = split_pages_override();
     if (ov > 0)
         sp = ov < kMaxTablePages ? ov : kMaxTablePages;
     pl.split_pages = static_cast<int>(sp);
+    pl.max_splits = pages > 0 ? static_cast<int>((pages + sp - 1) / sp) : 1;
+    return pl;
+}
+
+// Split plan of the tcgen05 rows kernel for `units` (sequence, KV head, row group) units: two CTAs
+// per SM, and a per-CTA cost of 32 pages (its TMEM allocation, Q load and the first K/V tiles'
+// latency before the ring streams, the partials and the merge of every extra split) -- fitted to
+// tree verification of 64 sequences x 8 drafts over contexts U[512, 4096] with 32/8 heads, where
+// splits of 64 / 128 / 256 pages measured 0.141 / 0.126 / 0.113 ms.  Never finer than `ws`, the
+// plan the workspace was sized for.
+static DecodePlan decode_plan_tc(int64_t units, int max_ctx, const DecodePlan &ws)
+{
+    DecodePlan pl = ws;
+    const int64_t pages = (int64_t)(max_ctx + 15) / 16;
+    int sp = plan_split_pages(units, pages, (int64_t)sm_count() * 2, 32);
+    if (split_pages_override() > 0 || sp < ws.split_pages)
+        sp = ws.split_pages;
+    pl.split_pages = sp;
     pl.max_splits = pages > 0 ? static_cast<int>((pages + sp - 1) / sp) : 1;
     return pl;
 }
@@ -1600,11 +1625,14 @@ static int run(const AttnArgs &a)
         const bool all_wide = !fp8 && tc_rows > 0 && (int64_t)rp.G * min_q >= kWideRows;
         if (!a.group_start)  // the shared-prefix call's plan kernel has written the order already
             rc = launch_seq_order(a.context_lens, a.B, order, rp.status, a.stream);
+        int merge_splits = pl.max_splits;  // splits of the kernel launched below
         if (rc == PA_OK && all_wide) {
-            RowsParams rt = rp;
-            rt.n_rg = static_cast<int>(((int64_t)rp.G * max_q + tc_rows - 1) / tc_rows);
-            const dim3 grid_tc(pl.max_splits, a.H_kv * rt.n_rg, a.B);
-            rc = launch_rows_tc(rt, tk, tv, D, a.dtype, rp.tree ? kModeTree : kModeCausal, tc_rows, grid_tc,
+            rp.n_rg = static_cast<int>(((int64_t)rp.G * max_q + tc_rows - 1) / tc_rows);
+            const DecodePlan tp = decode_plan_tc((int64_t)a.B * a.H_kv * rp.n_rg, a.max_ctx, pl);
+            rp.split_pages = tp.split_pages;
+            merge_splits = tp.max_splits;
+            const dim3 grid_tc(tp.max_splits, a.H_kv * rp.n_rg, a.B);
+            rc = launch_rows_tc(rp, tk, tv, D, a.dtype, rp.tree ? kModeTree : kModeCausal, tc_rows, grid_tc,
                                 a.stream);
         }
         if (rc == PA_OK && !all_wide) {
@@ -1614,7 +1642,7 @@ static int run(const AttnArgs &a)
                  : rp.tree ? launch_rows<D, BF16, kModeTree>(rp, tk, tv, grid, a.stream)
                            : launch_rows<D, BF16, kModeCausal>(rp, tk, tv, grid, a.stream);
         }
-        if (rc == PA_OK && pl.max_splits > 1)
+        if (rc == PA_OK && merge_splits > 1)
             rc = launch_merge<D, BF16>(rp, a.stream);
         return rc;
     }
