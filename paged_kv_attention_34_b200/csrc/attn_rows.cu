@@ -527,8 +527,8 @@ struct NarrowEpi {
     static constexpr int kBytes = (4 * 8 * kStride + 2 * 4 * 8) * 4;
 };
 
-// NARROW: no scale table (each warp loads its page's scales into registers one stage ahead), so
-// three CTAs fit on an SM.
+// NARROW: no scale table for the whole split; each stage carries its pages' scales (K then V, 16
+// floats per page), loaded by TMA with the codes, so five CTAs fit on an SM.
 template <int D, bool NARROW>
 struct Fp8Smem {
     static constexpr int kStages = NARROW ? kNarrowStages : kFp8Stages;
@@ -537,8 +537,13 @@ struct Fp8Smem {
     static_assert(NARROW || RowsEpi<D>::kBytes <= kStages * kStage, "the epilogue reuses the ring");
     static_assert(NarrowEpi<D>::kBytes <= kStages * kStage, "the epilogue reuses the ring");
     static constexpr int kRingOff = 0;
-    static constexpr int kScaleOff = kStages * kStage;          // [page of the split][K, V][16 keys]
-    static constexpr int kBarOff = kScaleOff + (NARROW ? 0 : kMaxTablePages * 2 * 16 * 4);
+    // NARROW: floats of a stage's scales, [K, V][page of the stage][32]: 16 keys and 16 floats of
+    // padding, as a TMA destination in shared memory must be 128-byte aligned
+    static constexpr int kScaleSlot = 32;
+    static constexpr int kStageScales = 2 * kPagesPerStage * kScaleSlot;
+    // wide: [page of the split][K, V][16 keys]; NARROW: [stage][K, V][page of the stage][32]
+    static constexpr int kScaleOff = kStages * kStage;
+    static constexpr int kBarOff = kScaleOff + (NARROW ? kStages * kStageScales * 4 : kMaxTablePages * 2 * 16 * 4);
     static constexpr int kCountOff = kBarOff + 8 * kStages;     // warps done with each stage
     static constexpr int kIssuedOff = kCountOff + 4 * kStages;  // loads issued into each stage
     static constexpr int kTableOff = kIssuedOff + 4 * kStages;
@@ -870,6 +875,7 @@ __device__ __forceinline__ void narrow_epilogue(float *e, const RowsParams &p, c
 template <int D, bool BF16, bool NARROW>
 __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
     pa_attn_rows_fp8_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                            const __grid_constant__ CUtensorMap tmap_ks, const __grid_constant__ CUtensorMap tmap_vs,
                             const RowsParams p)
 {
     using L = Fp8Smem<D, NARROW>;
@@ -937,17 +943,25 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
         }
         return pg;
     };
+    // bytes a page brings into a stage: its K and V codes and, NARROW, its 16 K and 16 V scales
+    constexpr int kPageTx = 2 * L::kPage + (NARROW ? 2 * 16 * 4 : 0);
     auto load_page = [&](int slot, int k, int pg) {
         uint8_t *kb = s_ring + slot * L::kStage;
         const int y = (pg * p.H_kv + g) * 16;
         tma_load_2d(kb + k * L::kPage, &tmap_k, 0, y, &s_bar[slot]);
         tma_load_2d(kb + (kPagesPerStage + k) * L::kPage, &tmap_v, 0, y, &s_bar[slot]);
+        if constexpr (NARROW) {
+            // a bad page id was replaced by num_blocks: its scale row is past the map, zero filled
+            float *sc = s_scale + slot * L::kStageScales;
+            tma_load_2d(sc + k * L::kScaleSlot, &tmap_ks, 0, pg * p.H_kv + g, &s_bar[slot]);
+            tma_load_2d(sc + (kPagesPerStage + k) * L::kScaleSlot, &tmap_vs, 0, pg * p.H_kv + g, &s_bar[slot]);
+        }
     };
     auto issue = [&](int st) {  // one thread; the page ids from the shared-memory copy
         const int slot = st % STAGES;
         const int np = min(kPagesPerStage, n_pages - st * kPagesPerStage);
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&s_bar[slot], np * 2 * L::kPage);
+        mbar_arrive_expect_tx(&s_bar[slot], np * kPageTx);
         s_issued[slot] += 1;
         for (int k = 0; k < np; ++k)
             load_page(slot, k, s_pages[st * kPagesPerStage + k]);
@@ -966,6 +980,10 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
             fence_barrier_init();
             prefetch_tmap(&tmap_k);
             prefetch_tmap(&tmap_v);
+            if constexpr (NARROW) {
+                prefetch_tmap(&tmap_ks);
+                prefetch_tmap(&tmap_vs);
+            }
         }
         const int first = min(STAGES, n_stages);
         const bool mine = lane < first * kPagesPerStage && lane < n_pages;
@@ -973,7 +991,7 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
         __syncwarp();
         if (lane == 0) {
             for (int st = 0; st < first; ++st) {
-                mbar_arrive_expect_tx(&s_bar[st], min(kPagesPerStage, n_pages - st * kPagesPerStage) * 2 * L::kPage);
+                mbar_arrive_expect_tx(&s_bar[st], min(kPagesPerStage, n_pages - st * kPagesPerStage) * kPageTx);
                 s_issued[st] += 1;
             }
         }
@@ -1068,26 +1086,6 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
         on[i][0] = on[i][1] = on[i][2] = on[i][3] = 0.f;
     const float sl2 = p.scale_log2;
 
-    // narrow: the scales of keys 2g, 2g + 1 of this warp's page of a stage, loaded a stage ahead
-    auto load_scales = [&](int pidx, float2 &kf, float2 &vf) {
-        kf = vf = make_float2(0.f, 0.f);
-        if (pidx < n_pages) {
-            const int pg = s_pages[pidx];
-            const int key0 = (page_lo + pidx) * 16 + 2 * (lane >> 2);
-            if (pg < p.num_blocks) {
-                const int64_t at = ((int64_t)pg * p.H_kv + g) * 16 + 2 * (lane >> 2);
-                kf = __ldg(reinterpret_cast<const float2 *>(p.k_scale + at));
-                vf = __ldg(reinterpret_cast<const float2 *>(p.v_scale + at));
-            }
-            if (key0 >= ctx)
-                kf.x = vf.x = 0.f;
-            if (key0 + 1 >= ctx)
-                kf.y = vf.y = 0.f;
-        }
-    };
-    float2 kf_next = make_float2(0.f, 0.f), vf_next = make_float2(0.f, 0.f);
-    if constexpr (NARROW)
-        load_scales(kg, kf_next, vf_next);
 
     // ---- main loop over stages (as the 16-bit kernel) ------------------------------------------
     for (int it = 0; it < n_stages; ++it) {
@@ -1098,12 +1096,18 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
             set_status(p.status, PA_ERR_TIMEOUT);
         }
         if constexpr (NARROW) {
-            // one page per warp per stage (KG = 4)
-            const float2 kf = kf_next, vf = vf_next;
-            load_scales((it + 1) * kPagesPerStage + kg, kf_next, vf_next);
+            // one page per warp per stage (KG = 4); the scales of its keys 2g, 2g + 1.  A key past
+            // the context end is masked from the scores whatever its K scale; its V scale (which
+            // may be anything, NaN included) becomes 0 so that P = 0 stays 0.
             const int pidx = it * kPagesPerStage + kg;
             const int j0 = (page_lo + pidx) * 16;
             if (ok && has_rows && pidx < n_pages && j0 <= lim_warp) {
+                const float *sc = s_scale + slot * L::kStageScales + 2 * (lane >> 2);
+                const float2 kf = *reinterpret_cast<const float2 *>(sc + kg * L::kScaleSlot);
+                float2 vf = *reinterpret_cast<const float2 *>(sc + (kPagesPerStage + kg) * L::kScaleSlot);
+                const int key0 = j0 + 2 * (lane >> 2);
+                vf.x = key0 < ctx ? vf.x : 0.f;
+                vf.y = key0 + 1 < ctx ? vf.y : 0.f;
                 const uint8_t *st = s_ring + slot * L::kStage;
                 narrow_page_fp8<D, BF16>(st + kg * L::kPage, st + (kPagesPerStage + kg) * L::kPage, kf, vf, j0, lane,
                                          qn, on, m_n, l_n, lim_n, ctx, sl2);
@@ -1319,8 +1323,8 @@ static int launch_rows(const RowsParams &rp, const CUtensorMap &tk, const CUtens
 }
 
 template <int D, bool BF16, bool NARROW>
-static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv, dim3 grid,
-                           cudaStream_t stream)
+static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CUtensorMap &tv,
+                           const CUtensorMap &tks, const CUtensorMap &tvs, dim3 grid, cudaStream_t stream)
 {
     using L = Fp8Smem<D, NARROW>;
     auto kern = pa_attn_rows_fp8_kernel<D, BF16, NARROW>;
@@ -1334,7 +1338,7 @@ static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CU
             return PA_ERR_CUDA;
         configured |= bit;
     }
-    const cudaError_t e = launch_dependent(kern, grid, dim3(kThreads), L::kAlloc, stream, tk, tv, rp);
+    const cudaError_t e = launch_dependent(kern, grid, dim3(kThreads), L::kAlloc, stream, tk, tv, tks, tvs, rp);
     count_launch();
     const cudaError_t e2 = cudaGetLastError();
     return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -1527,6 +1531,11 @@ static int run(const AttnArgs &a)
     if (rc == PA_OK)
         rc = fp8 ? make_cache_tmap_fp8(&tv, a.value_cache, a.num_blocks, a.H_kv, D)
                  : make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
+    CUtensorMap tks{}, tvs{};  // FP8: the row scales, which the narrow kernel loads with each stage
+    if (rc == PA_OK && fp8)
+        rc = make_scale_tmap(&tks, a.key_scale, a.num_blocks, a.H_kv);
+    if (rc == PA_OK && fp8)
+        rc = make_scale_tmap(&tvs, a.value_scale, a.num_blocks, a.H_kv);
     if (rc != PA_OK)
         return rc;
     RowsParams rp{};
@@ -1637,8 +1646,8 @@ static int run(const AttnArgs &a)
         }
         if (rc == PA_OK && !all_wide) {
             // single-token decode with at most 8 query heads per KV head: keys on the MMA's M side
-            rc = fp8 && a.T == a.B && rp.G <= 8 ? launch_rows_fp8<D, BF16, true>(rp, tk, tv, grid, a.stream)
-                 : fp8     ? launch_rows_fp8<D, BF16, false>(rp, tk, tv, grid, a.stream)
+            rc = fp8 && a.T == a.B && rp.G <= 8 ? launch_rows_fp8<D, BF16, true>(rp, tk, tv, tks, tvs, grid, a.stream)
+                 : fp8     ? launch_rows_fp8<D, BF16, false>(rp, tk, tv, tks, tvs, grid, a.stream)
                  : rp.tree ? launch_rows<D, BF16, kModeTree>(rp, tk, tv, grid, a.stream)
                            : launch_rows<D, BF16, kModeCausal>(rp, tk, tv, grid, a.stream);
         }

@@ -79,6 +79,21 @@ int make_cache_tmap_fp8(CUtensorMap *map, const void *cache, int64_t num_blocks,
     return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+int make_scale_tmap(CUtensorMap *map, const float *scale, int64_t num_blocks, int H_kv)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return PA_ERR_CUDA;
+    cuuint64_t dims[2] = {16, static_cast<cuuint64_t>(num_blocks * H_kv)};
+    cuuint64_t strides[1] = {16 * sizeof(float)};
+    cuuint32_t box[2] = {16, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(scale), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
 int make_q_tmap(CUtensorMap *map, const void *q, int64_t T, int H_q, int d, int G, int tok, pa_dtype dtype)
 {
     auto fn = encode_fn();

@@ -58,6 +58,10 @@ inline bool aligned4(const void *p) { return p && (reinterpret_cast<uintptr_t>(p
 int make_cache_tmap_fp8(CUtensorMap *map, const void *cache, int64_t num_blocks, int H_kv, int d);
 int make_cache_tmap(CUtensorMap *map, const void *cache, int64_t num_blocks, int H_kv, int d, pa_dtype dtype);
 
+// 2-D tensor map over FP8 row scales [num_blocks][H_kv][16] floats viewed as num_blocks * H_kv rows
+// of 16; box = one row (the 16 scales of one (block, head) page), no swizzle.
+int make_scale_tmap(CUtensorMap *map, const float *scale, int64_t num_blocks, int H_kv);
+
 // 3-D tensor map over Q [T][H_q][d] for query tiles of `tok` tokens x G heads of one
 // KV head: dims (d, H_q, T), box (64, G, tok), 128-byte swizzle.
 int make_q_tmap(CUtensorMap *map, const void *q, int64_t T, int H_q, int d, int G, int tok, pa_dtype dtype);
