@@ -552,17 +552,23 @@ struct Fp8Smem {
     static constexpr int kAlloc = kBytes + 128;  // slack to align the base to 128 B
 };
 
-// Two E4M3 codes (the low 16 bits of `pair`) -> two 16-bit values; exact, as every E4M3 value is
-// an f16 and a bf16 value.
+// Four E4M3 codes (the bytes of `w`, lowest first) -> two words of two 16-bit values: lo = codes 0,
+// 1 and hi = codes 2, 3; exact, as every E4M3 value is an f16 and a bf16 value.  The f16 form is
+// two conversions on the halves of the word, with no repacking around them.
 template <bool BF16>
-__device__ __forceinline__ uint32_t widen_e4m3x2(uint32_t pair)
+__device__ __forceinline__ void widen_e4m3x4(uint32_t w, uint32_t &lo, uint32_t &hi)
 {
-    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pair & 0xffffu), __NV_E4M3);
+    asm volatile("{\n\t.reg .b16 c0, c1;\n\t"
+        "mov.b32 {c0, c1}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c0;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, c1;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
     if constexpr (BF16) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
-        return pack2<true>(f.x, f.y);
-    } else {
-        return static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+        lo = pack2<true>(a.x, a.y);
+        hi = pack2<true>(b.x, b.y);
     }
 }
 
@@ -602,7 +608,8 @@ __device__ __forceinline__ void rows_page_fp8(const uint8_t *kp, const uint8_t *
         }
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ++ks) {
-            const uint32_t b0 = widen_e4m3x2<BF16>(w[ks]), b1 = widen_e4m3x2<BF16>(w[ks] >> 16);
+            uint32_t b0, b1;
+            widen_e4m3x4<BF16>(w[ks], b0, b1);
             if (ks & 1)
                 mma16816<BF16>(s2[t], qa[ks], b0, b1);
             else
@@ -687,7 +694,9 @@ __device__ __forceinline__ void rows_page_fp8(const uint8_t *kp, const uint8_t *
 #pragma unroll
     for (int nd = 0; nd < NT; ++nd) {
         const uint32_t w = *reinterpret_cast<const uint32_t *>(vp + (8 * nd + r) * 16 + 4 * kq) & vmask;
-        mma16816<BF16>(o[nd], pa_, widen_e4m3x2<BF16>(w), widen_e4m3x2<BF16>(w >> 16));
+        uint32_t b0, b1;
+        widen_e4m3x4<BF16>(w, b0, b1);
+        mma16816<BF16>(o[nd], pa_, b0, b1);
     }
 }
 
@@ -715,28 +724,23 @@ __device__ __forceinline__ void narrow_page_fp8(const uint8_t *kp, const uint8_t
     {
         const uint8_t *r0 = kp + (2 * g) * D + t * SPAN;
         const uint8_t *r1 = r0 + D;
-        uint32_t w0[SPAN / 4], w1[SPAN / 4];
+        // 16 bytes of each key row at a time (four k-steps), converted next to their products
 #pragma unroll
         for (int i = 0; i < SPAN / 16; ++i) {
-            const uint4 a = *reinterpret_cast<const uint4 *>(r0 + i * 16);
-            const uint4 b = *reinterpret_cast<const uint4 *>(r1 + i * 16);
-            w0[4 * i] = a.x;
-            w0[4 * i + 1] = a.y;
-            w0[4 * i + 2] = a.z;
-            w0[4 * i + 3] = a.w;
-            w1[4 * i] = b.x;
-            w1[4 * i + 1] = b.y;
-            w1[4 * i + 2] = b.z;
-            w1[4 * i + 3] = b.w;
-        }
+            const uint4 a4 = *reinterpret_cast<const uint4 *>(r0 + i * 16);
+            const uint4 b4 = *reinterpret_cast<const uint4 *>(r1 + i * 16);
+            const uint32_t w0[4] = {a4.x, a4.y, a4.z, a4.w}, w1[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-        for (int ks = 0; ks < KSTEPS; ++ks) {
-            const uint32_t a[4] = {widen_e4m3x2<BF16>(w0[ks]), widen_e4m3x2<BF16>(w1[ks]),
-                                   widen_e4m3x2<BF16>(w0[ks] >> 16), widen_e4m3x2<BF16>(w1[ks] >> 16)};
-            if (ks & 1)
-                mma16816<BF16>(s2, a, qb[ks][0], qb[ks][1]);
-            else
-                mma16816<BF16>(s, a, qb[ks][0], qb[ks][1]);
+            for (int q = 0; q < 4; ++q) {
+                const int ks = 4 * i + q;
+                uint32_t a[4];
+                widen_e4m3x4<BF16>(w0[q], a[0], a[2]);
+                widen_e4m3x4<BF16>(w1[q], a[1], a[3]);
+                if (ks & 1)
+                    mma16816<BF16>(s2, a, qb[ks][0], qb[ks][1]);
+                else
+                    mma16816<BF16>(s, a, qb[ks][0], qb[ks][1]);
+            }
         }
     }
     // x0 = (key 2g, row 2t), x1 = (2g, 2t+1), x2 = (2g+1, 2t), x3 = (2g+1, 2t+1): key scales,
@@ -795,8 +799,9 @@ __device__ __forceinline__ void narrow_page_fp8(const uint8_t *kp, const uint8_t
     for (int mt = 0; mt < MT; ++mt) {
         const uint32_t wa = *reinterpret_cast<const uint32_t *>(vp + (16 * mt + g) * 16 + 4 * t) & vmask;
         const uint32_t wb = *reinterpret_cast<const uint32_t *>(vp + (16 * mt + g + 8) * 16 + 4 * t) & vmask;
-        const uint32_t a[4] = {widen_e4m3x2<BF16>(wa), widen_e4m3x2<BF16>(wb), widen_e4m3x2<BF16>(wa >> 16),
-                               widen_e4m3x2<BF16>(wb >> 16)};
+        uint32_t a[4];
+        widen_e4m3x4<BF16>(wa, a[0], a[2]);
+        widen_e4m3x4<BF16>(wb, a[1], a[3]);
         mma16816<BF16>(o[mt], a, pb0, pb1);
     }
 }
