@@ -51,8 +51,8 @@ if ROOT not in sys.path:
 METRIC = "paged decode attn HBM GB/s & prefill attn TFLOPS, as % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu DRAM bytes (read + written) / algorithmic bytes of the 16-bit decode kernel, captured on the
-# 13B-shaped decode layer with 16 sequences: 702.95 MB / 696.53 MB
-TRAFFIC_RATIO_DECODE_13B = 702.95 / 696.53
+# 13B-shaped decode layer with 16 sequences: (698.58 + 5.11) MB / 696.53 MB
+TRAFFIC_RATIO_DECODE_13B = (698.58 + 5.11) / 696.53
 HEADLINE = "LLaMA-2-13B-shaped decode layer: B 64, q_len 1, 40/40 heads, d 128, fp16, ctx U[128,4096], block 16"
 
 
