@@ -155,7 +155,10 @@ size_t pa_decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int
  *   scale        multiplies Q K^T (normally 1/sqrt(d))
  *   workspace    >= pa_decode_workspace_bytes(T, B, H_q, H_kv, d, max_ctx) bytes; its
  *                first PA_STATUS_BYTES hold the status word, which this call resets
- *                to PA_OK on `stream` before launching.
+ *                to PA_OK on `stream`: its first kernel clears it before any other
+ *                kernel of the call runs (a call with B = 0 or T = 0 launches nothing and
+ *                clears it with a memset).  After a call that returns an error code
+ *                it holds no result of that call.
  */
 int pa_paged_attn_decode(void *out, const void *q, const void *key_cache, const void *value_cache,
                          int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
@@ -291,7 +294,8 @@ int pa_paged_attn_decode_fp8(void *out, const void *q, const uint8_t *key_cache,
  *     array's device address (cudaGetSymbolAddress) and keeps it: make that
  *     first call before any stream capture;
  *   - all calls on a device share the array and it keeps the last call's
- *     contents; the status word is cleared on `stream` before each launch.
+ *     contents; the status word is cleared on `stream` by each call, as in
+ *     pa_paged_attn_decode.
  *     Calls that overlap on the GPU (different streams without ordering) race;
  *   - status: optional device int32 (may be NULL) that receives the call's
  *     device status word (copied on `stream` after the kernels).
@@ -323,7 +327,8 @@ size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len
  * softmax of iopencloud section 2.2 runs between the two products.
  *   out, q        [T][H_q][d]        cu_seqlens_q [B+1] (q_b >= 1)   context_lens [B]
  *   max_q_len     host upper bound of q_b;  max_ctx host upper bound of ctx_b
- *   workspace     >= pa_prefill_workspace_bytes(...) bytes; status word reset on stream.
+ *   workspace     >= pa_prefill_workspace_bytes(...) bytes; status word reset on stream
+ *                 (by the call's first kernel, as in pa_paged_attn_decode).
  */
 int pa_paged_attn_prefill(void *out, const void *q, const void *key_cache, const void *value_cache,
                           int64_t num_blocks, const int32_t *block_tables, int max_blocks_per_seq,
