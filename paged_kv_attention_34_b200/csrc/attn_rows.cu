@@ -714,7 +714,6 @@ __device__ __forceinline__ void narrow_page_fp8(const uint8_t *kp, const uint8_t
                                                 const uint32_t (&qb)[D / 16][2], float (&o)[D / 16][4], float (&m)[2],
                                                 float (&l)[2], const int (&lim)[2], int ctx, float sl2)
 {
-    constexpr int KSTEPS = D / 16;  // k-steps of S^T
     constexpr int MT = D / 16;      // m-tiles of O^T
     constexpr int SPAN = D / 4;     // code bytes of a key row per lane quad
     const int g = lane >> 2, t = lane & 3;
