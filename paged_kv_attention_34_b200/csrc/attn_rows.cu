@@ -1187,6 +1187,48 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
         return;
     auto slot = [&](int s) -> int64_t { return s < nps ? s : own_slot + (s - nps); };
     const int64_t stride = p.T * p.H_q;
+    constexpr int LANES = D / 4;
+    if (ns <= 32) {
+        // one split per lane: its log2-sum-exp read once, the weights 2^(lse_s - max) / sum in
+        // registers, then the partials read four splits at a time (independent loads in flight)
+        const float l = lane < ns ? p.ws_lse[slot(lane) * stride + row] : -INFINITY;
+        float M = l;
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float w = l == -INFINITY ? 0.f : fast_exp2(l - M);
+        float Z = w;
+#pragma unroll
+        for (int o = 16; o; o >>= 1)
+            Z += __shfl_xor_sync(0xffffffffu, Z, o);
+        w *= Z > 0.f ? 1.f / Z : 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < ns; s0 += 4) {
+            float ws[4];
+            float4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                ws[k] = __shfl_sync(0xffffffffu, w, (s0 + k) & 31);
+                if (s0 + k >= ns)
+                    ws[k] = 0.f;
+                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (ws[k] != 0.f && lane < LANES)
+                    v[k] = *reinterpret_cast<const float4 *>(p.ws_o + (slot(s0 + k) * stride + row) * D + lane * 4);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (ws[k] == 0.f)
+                    continue;
+                acc.x += ws[k] * v[k].x;
+                acc.y += ws[k] * v[k].y;
+                acc.z += ws[k] * v[k].z;
+                acc.w += ws[k] * v[k].w;
+            }
+        }
+        if (lane < LANES)
+            store4<BF16>(static_cast<uint8_t *>(p.out) + (row * D + lane * 4) * 2, acc.x, acc.y, acc.z, acc.w);
+        return;
+    }
     float M = -INFINITY;
     for (int s = lane; s < ns; s += 32)
         M = fmaxf(M, p.ws_lse[slot(s) * stride + row]);
@@ -1202,7 +1244,6 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
     for (int o = 16; o; o >>= 1)
         Z += __shfl_xor_sync(0xffffffffu, Z, o);
     const float invZ = Z > 0.f ? 1.f / Z : 0.f;
-    constexpr int LANES = D / 4;
     if (lane < LANES) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int s = 0; s < ns; ++s) {
