@@ -257,16 +257,36 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
 
 constexpr int kOrderKeys = 4096;
 constexpr int kOrderThreads = 1024;
+constexpr int kOrderSmall = 256;  // up to this many elements: ranks by comparison
 
 // One CTA of kOrderThreads threads, all of which call this: order[r] = the element of rank r when
 // the n elements are sorted by decreasing key_of(e) in [0, kOrderKeys) (a counting sort; elements
-// with equal keys in arbitrary order).
+// with equal keys in arbitrary order; up to kOrderSmall elements, ranks by comparison, equal keys
+// by index).
 template <class KeyOf>
 __device__ void order_by_key_desc(int n, KeyOf key_of, int32_t *order)
 {
+    const int tid = threadIdx.x;
+    if (n <= kOrderSmall) {
+        // few elements: each one's rank by comparison with all of them (ties by index), one barrier
+        __shared__ int key[kOrderSmall];
+        if (tid < n)
+            key[tid] = key_of(tid);
+        __syncthreads();
+        if (tid < n) {
+            const int k = key[tid];
+            int r = 0;
+            for (int u = 0; u < n; ++u) {
+                const int ku = key[u];
+                r += (ku > k || (ku == k && u < tid)) ? 1 : 0;
+            }
+            order[r] = tid;
+        }
+        return;
+    }
     __shared__ int cnt[kOrderKeys];
     __shared__ int warp_tot[kOrderThreads / 32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int lane = tid & 31, warp = tid >> 5;
     for (int i = tid; i < kOrderKeys; i += kOrderThreads)
         cnt[i] = 0;
     __syncthreads();
