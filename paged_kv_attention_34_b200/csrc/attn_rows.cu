@@ -1272,6 +1272,7 @@ __global__ void __launch_bounds__(256) pa_split_merge_kernel(const RowsParams p)
 __global__ void __launch_bounds__(kOrderThreads) pa_shared_plan_kernel(const RowsParams p, int32_t *order,
                                                                          int fill_prefix)
 {
+    griddep_wait();  // the kernel before this call's on the stream (its writes are visible after this)
     if (threadIdx.x == 0)
         *p.status = PA_OK;  // the call's status word: this is its first kernel
     __syncthreads();        // before any thread records a malformed group
@@ -1395,6 +1396,7 @@ static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CU
 __global__ void __launch_bounds__(kOrderThreads)
     pa_seq_order_kernel(const int32_t *context_lens, int B, int32_t *order, int32_t *status)
 {
+    griddep_wait();  // the kernel before this call's on the stream (its writes are visible after this)
     if (threadIdx.x == 0)
         *status = PA_OK;  // the call's status word: this is its first kernel
     griddep_release();    // the attention kernel's CTAs may be scheduled now; they wait for the order
@@ -1410,9 +1412,11 @@ __global__ void __launch_bounds__(kOrderThreads)
 
 int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, cudaStream_t stream)
 {
-    pa_seq_order_kernel<<<1, kOrderThreads, 0, stream>>>(context_lens, B, order, status);
+    const cudaError_t e = launch_dependent(pa_seq_order_kernel, dim3(1), dim3(kOrderThreads), 0, stream, context_lens, B,
+                                           order, status);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 template <int D, bool BF16>
@@ -1629,9 +1633,11 @@ static int run(const AttnArgs &a)
         // one launch writes the sequence order and checks the groups (status), whichever path
         // computes the result
         const bool pays = shared_pass_pays(a);
-        pa_shared_plan_kernel<<<1, kOrderThreads, 0, a.stream>>>(rp, order, pays ? 1 : 0);
+        const cudaError_t e =
+            launch_dependent(pa_shared_plan_kernel, dim3(1), dim3(kOrderThreads), 0, a.stream, rp, order, pays ? 1 : 0);
         count_launch();
-        rc = cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+        const cudaError_t e2 = cudaGetLastError();
+        rc = e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
         if (rc != PA_OK)
             return rc;
         if (pays) {

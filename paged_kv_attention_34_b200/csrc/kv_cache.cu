@@ -24,6 +24,9 @@ __global__ void __launch_bounds__(256) kv_cache_write_kernel(const uint4 *__rest
                                                              uint4 *__restrict__ value_cache, int64_t num_blocks,
                                                              int H_kv, int32_t *status)
 {
+    // a programmatic dependent of the kernel before it on the stream: wait for it before any access
+    griddep_wait();
+    griddep_release();
     const int64_t items = T * H_kv * CH;
     const int64_t n_slots = num_blocks * 16;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < items; i += (int64_t)gridDim.x * blockDim.x) {
@@ -54,6 +57,9 @@ __global__ void __launch_bounds__(256) kv_block_copy_kernel(uint4 *__restrict__ 
                                                             const int32_t *__restrict__ pairs, int64_t n,
                                                             int32_t *status)
 {
+    // a programmatic dependent of the kernel before it on the stream: wait for it before any access
+    griddep_wait();
+    griddep_release();
     const int64_t items = n * chunks_per_block;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < items; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t p = i / chunks_per_block;
@@ -80,6 +86,9 @@ __global__ void __launch_bounds__(256) kv_block_swap_kernel(uint4 *__restrict__ 
                                                             const int32_t *__restrict__ pairs, int64_t n, int to_host,
                                                             int32_t *status)
 {
+    // a programmatic dependent of the kernel before it on the stream: wait for it before any access
+    griddep_wait();
+    griddep_release();
     const int64_t items = n * chunks_per_block;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < items; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t p = i / chunks_per_block;
@@ -116,6 +125,9 @@ __global__ void __launch_bounds__(256) kv_cache_write_fp8_kernel(const void *__r
                                                                  uint8_t *__restrict__ value_cache, float *key_scale,
                                                                  float *value_scale, int64_t num_blocks, int32_t *status)
 {
+    // a programmatic dependent of the kernel before it on the stream: wait for it before any access
+    griddep_wait();
+    griddep_release();
     constexpr int VPL = D / 32;  // values per lane (2 or 4)
     const int lane = threadIdx.x & 31;
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -206,19 +218,23 @@ extern "C" int pa_kv_cache_write(const void *k_new, const void *v_new, const int
         return PA_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int threads = 256;
+    cudaError_t e;
     if (d == 128) {
         const int64_t items = T * H_kv * 16;
-        kv_cache_write_kernel<16><<<grid_for(items, threads), threads, 0, s>>>(
-            static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slot_mapping, T,
-            static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), num_blocks, H_kv, status);
+        e = launch_dependent(kv_cache_write_kernel<16>, dim3(grid_for(items, threads)), dim3(threads), 0, s,
+                             static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slot_mapping, T,
+                             static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), num_blocks, H_kv,
+                             status);
     } else {
         const int64_t items = T * H_kv * 8;
-        kv_cache_write_kernel<8><<<grid_for(items, threads), threads, 0, s>>>(
-            static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slot_mapping, T,
-            static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), num_blocks, H_kv, status);
+        e = launch_dependent(kv_cache_write_kernel<8>, dim3(grid_for(items, threads)), dim3(threads), 0, s,
+                             static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slot_mapping, T,
+                             static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), num_blocks, H_kv,
+                             status);
     }
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" int pa_kv_block_copy(void *key_cache, void *value_cache, int64_t num_blocks, int H_kv, int d,
@@ -237,10 +253,12 @@ extern "C" int pa_kv_block_copy(void *key_cache, void *value_cache, int64_t num_
         return PA_ERR_ALIGN;
     const int64_t chunks = (int64_t)H_kv * 16 * d * 2 / 16;
     const int threads = 256;
-    kv_block_copy_kernel<<<grid_for(n * chunks, threads), threads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), num_blocks, chunks, pairs, n, status);
+    const cudaError_t e = launch_dependent(kv_block_copy_kernel, dim3(grid_for(n * chunks, threads)), dim3(threads), 0,
+                                           static_cast<cudaStream_t>(stream), static_cast<uint4 *>(key_cache),
+                                           static_cast<uint4 *>(value_cache), num_blocks, chunks, pairs, n, status);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // The device-mapped address of page-locked host memory at `p`, or nullptr when `p` is not
@@ -284,11 +302,13 @@ extern "C" int pa_kv_block_swap(void *key_cache, void *value_cache, int64_t num_
         return PA_ERR_ALIGN;
     const int64_t chunks = (int64_t)H_kv * 16 * d * 2 / 16;
     const int threads = 256;
-    kv_block_swap_kernel<<<grid_for(n * chunks, threads), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+    const cudaError_t e = launch_dependent(
+        kv_block_swap_kernel, dim3(grid_for(n * chunks, threads)), dim3(threads), 0, static_cast<cudaStream_t>(stream),
         static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache), num_blocks, static_cast<uint4 *>(hk),
         static_cast<uint4 *>(hv), host_blocks, chunks, pairs, n, direction == PA_SWAP_OUT ? 1 : 0, status);
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 extern "C" int pa_kv_cache_write_fp8(const void *k_new, const void *v_new, const int32_t *slot_mapping, int64_t T,
@@ -312,13 +332,15 @@ extern "C" int pa_kv_cache_write_fp8(const void *k_new, const void *v_new, const
     const int grid = grid_for(warps_needed * 32, threads);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 #define PA_LAUNCH_WRITE8(DD, BB)                                                                                   \
-    kv_cache_write_fp8_kernel<DD, BB><<<grid, threads, 0, s>>>(k_new, v_new, slot_mapping, T, H_kv, key_cache,     \
-                                                               value_cache, key_scale, value_scale, num_blocks, status)
+    launch_dependent(kv_cache_write_fp8_kernel<DD, BB>, dim3(grid), dim3(threads), 0, s, k_new, v_new, slot_mapping, T, \
+                     H_kv, key_cache, value_cache, key_scale, value_scale, num_blocks, status)
+    cudaError_t e;
     if (d == 128)
-        dtype == PA_BF16 ? PA_LAUNCH_WRITE8(128, true) : PA_LAUNCH_WRITE8(128, false);
+        e = dtype == PA_BF16 ? PA_LAUNCH_WRITE8(128, true) : PA_LAUNCH_WRITE8(128, false);
     else
-        dtype == PA_BF16 ? PA_LAUNCH_WRITE8(64, true) : PA_LAUNCH_WRITE8(64, false);
+        e = dtype == PA_BF16 ? PA_LAUNCH_WRITE8(64, true) : PA_LAUNCH_WRITE8(64, false);
 #undef PA_LAUNCH_WRITE8
     count_launch();
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

@@ -24,10 +24,10 @@ struct CallRange {
 // Counts every kernel launch of the library (pa_launch_count).
 void count_launch(uint64_t n = 1);
 
-// Launches `kern` as a programmatic dependent of the kernel before it on `stream` (a kernel of the
-// same library call): its CTAs may be scheduled while that kernel still runs and must call
-// griddep_wait() before they read anything it writes.  Hides the launch latency between the
-// kernels of one call.
+// Launches `kern` as a programmatic dependent of the kernel before it on `stream`: its CTAs may be
+// scheduled while that kernel still runs, and every kernel of the library calls griddep_wait()
+// before it touches memory (a kernel launched the ordinary way before it, or any other stream
+// operation, still completes first).  Hides the launch latency between kernels.
 #ifndef PA_DEPENDENT_LAUNCH
 #define PA_DEPENDENT_LAUNCH 1
 #endif

@@ -151,6 +151,7 @@ __global__ void __launch_bounds__(kOrderThreads) pa_prefill_order_kernel(const i
                                                                            int n_pairs, int tok_per_tile, int32_t *order,
                                                                            int *counter, int32_t *status)
 {
+    griddep_wait();  // the kernel before this call's on the stream (its writes are visible after this)
     if (threadIdx.x == 0) {
         *status = PA_OK;  // the call's status word: this is its first kernel
         *counter = 0;     // the work counter the attention kernel's CTAs draw items from
@@ -797,10 +798,11 @@ static int run(const AttnArgs &a)
         rc = make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
     if (rc != PA_OK)
         return rc;
-    pa_prefill_order_kernel<<<1, kOrderThreads, 0, a.stream>>>(a.cu_seqlens_q, a.context_lens, a.B, p.n_pairs_max,
-                                                                 p.tok_per_tile, order, p.counter, p.status);
+    const cudaError_t eo = launch_dependent(pa_prefill_order_kernel, dim3(1), dim3(kOrderThreads), 0, a.stream,
+                                            a.cu_seqlens_q, a.context_lens, a.B, p.n_pairs_max, p.tok_per_tile, order,
+                                            p.counter, p.status);
     count_launch();
-    if (cudaGetLastError() != cudaSuccess)
+    if (eo != cudaSuccess || cudaGetLastError() != cudaSuccess)
         return PA_ERR_CUDA;
 
     auto kern = pa_prefill_tc_kernel<D, BF16>;
