@@ -494,10 +494,6 @@ __global__ void __launch_bounds__(kThreads, PA_ROWS_MIN_BLOCKS)
     // [0, prefix_slots), a sequence's own splits after them
     rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_stage), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0, q0, g,
                            slot0 + split, MODE != kModeShared && n_splits == 1, KG);
-    if (MODE != kModeShared && n_splits > 1 && p.merge_cnt != nullptr) {
-        __threadfence();
-        merge_splits_if_last<D, BF16>(p, n_splits, rows_here, row0, q0, g, reinterpret_cast<int *>(smem + L::kFlagOff) + 1);
-    }
 }
 
 // ---- FP8 (E4M3) cache -----------------------------------------------------------------------
@@ -1158,10 +1154,6 @@ __global__ void __launch_bounds__(kThreads, NARROW ? kNarrowCtasPerSm : 1)
     else
         rows_epilogue<D, BF16>(reinterpret_cast<float *>(s_ring), p, o, m_a, m_b, l_a, l_b, has_rows, rows_here, row0,
                                q0, g, split, n_splits == 1, KG);
-    if (n_splits > 1 && p.merge_cnt != nullptr) {
-        __threadfence();
-        merge_splits_if_last<D, BF16>(p, n_splits, rows_here, row0, q0, g, reinterpret_cast<int *>(smem + L::kFlagOff) + 1);
-    }
 }
 
 // One warp per (token, query head) row of a sequence with more than one split:
@@ -1402,14 +1394,11 @@ static int launch_rows_fp8(const RowsParams &rp, const CUtensorMap &tk, const CU
 // the most pages at the front leaves short CTAs for the last wave (longest-processing-time-first
 // list scheduling; the order among equal page counts is arbitrary and changes no result).
 __global__ void __launch_bounds__(kOrderThreads)
-    pa_seq_order_kernel(const int32_t *context_lens, int B, int32_t *order, int32_t *status, int32_t *clear,
-                        int n_clear)
+    pa_seq_order_kernel(const int32_t *context_lens, int B, int32_t *order, int32_t *status)
 {
     griddep_wait();  // the kernel before this call's on the stream (its writes are visible after this)
     if (threadIdx.x == 0)
         *status = PA_OK;  // the call's status word: this is its first kernel
-    for (int i = threadIdx.x; i < n_clear; i += kOrderThreads)
-        clear[i] = 0;  // the split-merge counters of the attention kernel
     griddep_release();    // the attention kernel's CTAs may be scheduled now; they wait for the order
     order_by_key_desc(
         B,
@@ -1421,11 +1410,10 @@ __global__ void __launch_bounds__(kOrderThreads)
         order);
 }
 
-int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, int32_t *clear,
-                     int n_clear, cudaStream_t stream)
+int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, cudaStream_t stream)
 {
     const cudaError_t e = launch_dependent(pa_seq_order_kernel, dim3(1), dim3(kOrderThreads), 0, stream, context_lens, B,
-                                           order, status, clear, clear ? n_clear : 0);
+                                           order, status);
     count_launch();
     const cudaError_t e2 = cudaGetLastError();
     return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
@@ -1452,12 +1440,6 @@ static int split_pages_override()
     }
     return v;
 }
-
-// Most splits per sequence that the attention kernel merges itself (more: pa_split_merge_kernel).
-#ifndef PA_FUSED_MERGE_MAX_SPLITS
-#define PA_FUSED_MERGE_MAX_SPLITS 4
-#endif
-constexpr int kFusedMergeMaxSplits = PA_FUSED_MERGE_MAX_SPLITS;
 
 // Decode CTAs the split planner counts on per SM.
 #ifndef PA_PLAN_CTAS_PER_SM
@@ -1524,13 +1506,8 @@ static DecodePlan decode_plan_tc(int64_t units, int max_ctx, const DecodePlan &w
 }
 
 // Workspace: status word area, the sequence order, then (with more than one split) the partial
-// outputs and their log-sum-exps, and one merge counter per (sequence, KV head, row group).
+// outputs and their log-sum-exps.
 size_t seq_order_bytes(int B) { return (static_cast<size_t>(B) * sizeof(int32_t) + 255) / 256 * 256; }
-
-static size_t merge_counter_bytes(int B, int H_kv, int row_groups)
-{
-    return (static_cast<size_t>(B) * H_kv * row_groups * sizeof(int32_t) + 255) / 256 * 256;
-}
 
 size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int max_ctx)
 {
@@ -1541,7 +1518,6 @@ size_t decode_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
         bytes += rows * d * sizeof(float);
         bytes += rows * sizeof(float);
         bytes += 256;
-        bytes += merge_counter_bytes(B, H_kv, pl.row_groups);
     }
     return bytes;
 }
@@ -1690,24 +1666,11 @@ static int run(const AttnArgs &a)
         rp.split_pages = pl.split_pages;
         int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES);
         rp.order = order;
-        int n_cnt = 0;
         if (pl.max_splits > 1) {
             const size_t rows = static_cast<size_t>(pl.max_splits) * static_cast<size_t>(a.T) * a.H_q;
             uint8_t *ws = static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES + seq_order_bytes(a.B);
             rp.ws_o = reinterpret_cast<float *>(ws);
             rp.ws_lse = reinterpret_cast<float *>(ws + rows * D * sizeof(float));
-            // With few splits the attention kernel merges them itself: the last split of a unit to
-            // finish combines its partials (measured on the mixed continuous-batching step, 3
-            // splits: 4 us less than the merge kernel).  With many, every CTA's fence and counter
-            // round trip cost more than the merge kernel (32 K GQA decode, 10 splits: 7 us more).
-            // The counters are cleared by the order kernel, so a shared-prefix call that fell back
-            // here (its order comes from the plan kernel) keeps the merge kernel, as do batches with
-            // more counters than that one CTA clears quickly.
-            const int64_t units = (int64_t)a.B * a.H_kv * pl.row_groups;
-            if (pl.max_splits <= kFusedMergeMaxSplits && !a.group_start && units <= (1 << 16)) {
-                rp.merge_cnt = reinterpret_cast<int32_t *>(ws + rows * D * sizeof(float) + rows * sizeof(float) + 256);
-                n_cnt = static_cast<int>(units);
-            }
         }
         if (a.B > 65535 || (int64_t)a.H_kv * pl.row_groups > 65535)
             return PA_ERR_UNSUPPORTED;
@@ -1721,7 +1684,7 @@ static int run(const AttnArgs &a)
         const int tc_rows = rows_tc_rows_per_cta(rp.G, static_cast<int>(max_q));
         const bool all_wide = !fp8 && tc_rows > 0 && (int64_t)rp.G * min_q >= kWideRows;
         if (!a.group_start)  // the shared-prefix call's plan kernel has written the order already
-            rc = launch_seq_order(a.context_lens, a.B, order, rp.status, rp.merge_cnt, n_cnt, a.stream);
+            rc = launch_seq_order(a.context_lens, a.B, order, rp.status, a.stream);
         int merge_splits = pl.max_splits;  // splits of the kernel launched below
         if (rc == PA_OK && all_wide) {
             rp.n_rg = static_cast<int>(((int64_t)rp.G * max_q + tc_rows - 1) / tc_rows);
@@ -1739,7 +1702,7 @@ static int run(const AttnArgs &a)
                  : rp.tree ? launch_rows<D, BF16, kModeTree>(rp, tk, tv, grid, a.stream)
                            : launch_rows<D, BF16, kModeCausal>(rp, tk, tv, grid, a.stream);
         }
-        if (rc == PA_OK && merge_splits > 1 && !rp.merge_cnt)
+        if (rc == PA_OK && merge_splits > 1)
             rc = launch_merge<D, BF16>(rp, a.stream);
         return rc;
     }

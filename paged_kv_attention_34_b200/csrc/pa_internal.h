@@ -135,11 +135,9 @@ size_t shared_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
 
 // Sequence order by decreasing page count (one CTA, on `stream`): order[r] = the sequence of rank r.
 // The workspace holds it right after the status area, seq_order_bytes(B) bytes.  The kernel is the
-// first of its call; it also clears the call's status word and the n_clear ints at `clear` (the
-// split-merge counters of the attention kernel that follows, or none).
+// first of its call and also clears the call's status word.
 size_t seq_order_bytes(int B);
-int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, int32_t *clear,
-                     int n_clear, cudaStream_t stream);
+int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, cudaStream_t stream);
 int launch_decode(const AttnArgs &a);
 size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int max_q_len);
 int launch_prefill(const AttnArgs &a);

@@ -28,10 +28,6 @@ struct RowsParams {
     const int32_t *context_lens;
     float *ws_o;    // [max_splits][T][H_q][D] normalised partial outputs
     float *ws_lse;  // [max_splits][T][H_q] log2-sum-exp of the scaled scores
-    // [gridDim.z][gridDim.y] splits of each (sequence, KV head, row group) that have stored their
-    // partials, zeroed by the order kernel; the split that completes a unit merges it.  nullptr:
-    // pa_split_merge_kernel merges after the attention kernel.
-    int32_t *merge_cnt;
     const int32_t *order;  // [B] sequences by decreasing page count: grid z -> sequence
     const int32_t *tree;   // [T] tree verification: bit j = the token sees new token j; nullptr = causal
     const float *k_scale;  // FP8 cache: [num_blocks][H_kv][16] scale of every stored K row
@@ -144,60 +140,6 @@ __device__ __forceinline__ bool decode_unit(const RowsParams &p, int tid, Decode
         u.table = p.block_tables + (int64_t)b * p.max_blocks;
         return true;
     }
-}
-
-// Split-KV merge inside the attention kernel, for calls with few splits: after every thread of the
-// CTA has stored its part of the split's partials (normalised O and log2-sum-exp, workspace slot
-// `split`) and executed __threadfence(), one arrival per split on the unit's counter; the CTA that
-// arrives last combines the n_splits partials of its rows_here rows into `out` (the arithmetic of
-// pa_split_merge_kernel: weights 2^(lse_s - max lse) / sum, partials summed in split order) and
-// clears the counter.  The partials of other CTAs are read through L2 (ld.global.cg).  Every thread
-// of the CTA calls this (it holds __syncthreads); `s_flag` is one int of shared memory.
-template <int D, bool BF16>
-__device__ __forceinline__ void merge_splits_if_last(const RowsParams &p, int n_splits, int rows_here, int row0, int q0,
-                                                     int g, int *s_flag)
-{
-    const int tid = threadIdx.x, nthr = blockDim.x;
-    int32_t *cnt = p.merge_cnt + (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
-    __syncthreads();
-    if (tid == 0)
-        *s_flag = atomicAdd(cnt, 1) == n_splits - 1;
-    __syncthreads();
-    if (!*s_flag)
-        return;
-    __threadfence();
-    const int G = p.G;
-    const int64_t stride = p.T * p.H_q;
-    constexpr int C4 = D / 4;
-    for (int i = tid; i < rows_here * C4; i += nthr) {
-        const int r = i / C4, c4 = i % C4;
-        const int ridx = row0 + r;
-        const int64_t orow = (q0 + ridx / G) * p.H_q + g * G + ridx % G;
-        float M = -INFINITY;
-        for (int s = 0; s < n_splits; ++s)
-            M = fmaxf(M, __ldcg(p.ws_lse + s * stride + orow));
-        float Z = 0.f;
-        for (int s = 0; s < n_splits; ++s) {
-            const float l = __ldcg(p.ws_lse + s * stride + orow);
-            Z += l == -INFINITY ? 0.f : fast_exp2(l - M);
-        }
-        const float invZ = Z > 0.f ? 1.f / Z : 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < n_splits; ++s) {
-            const float l = __ldcg(p.ws_lse + s * stride + orow);
-            const float w = l == -INFINITY ? 0.f : fast_exp2(l - M) * invZ;
-            if (w == 0.f)
-                continue;
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.ws_o + (s * stride + orow) * D) + c4);
-            acc.x += w * v.x;
-            acc.y += w * v.y;
-            acc.z += w * v.z;
-            acc.w += w * v.w;
-        }
-        store4<BF16>(static_cast<uint8_t *>(p.out) + (orow * D + c4 * 4) * 2, acc.x, acc.y, acc.z, acc.w);
-    }
-    if (tid == 0)
-        *cnt = 0;
 }
 
 // The tcgen05 rows kernel (rows_tc.cu) for wide row groups: the rows one CTA holds for G query

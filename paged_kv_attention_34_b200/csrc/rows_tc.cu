@@ -64,7 +64,7 @@ struct Smem {
     // q_full, k_full, v_full, k_empty, v_empty [kMaxStages each], s_full[2], p_full[2], pv_done,
     // o_done, land, drain
     static constexpr int kNumBars = 1 + 4 * kMaxStages + 2 + 2 + 4;
-    static constexpr int kTail = 8 * kNumBars + 16;      // barriers, TMEM slot, abort flag, merge flag
+    static constexpr int kTail = 8 * kNumBars + 16;      // barriers, TMEM slot, abort flag
     __host__ __device__ static constexpr int q_rows(int rows) { return (rows + 7) / 8 * 8; }
     __host__ __device__ static constexpr int ring(int rows) { return kKB * q_rows(rows) * 128; }
     __host__ __device__ static constexpr int bars(int rows, int stages) { return ring(rows) + stages * 2 * kTile; }
@@ -474,18 +474,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
 
-    // with a few splits, the last split of the unit to finish merges the unit's partials
-    const bool merge_here = MODE != kModeShared && n_splits > 1 && p.merge_cnt != nullptr;
-    if (merge_here)
-        __threadfence();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     if (warp == 0)
         tc::tmem_dealloc(tmem, kTmemCols);
-    if (merge_here)
-        merge_splits_if_last<D, BF16>(p, n_splits, rows_here, row0, u.q0, g,
-                                      reinterpret_cast<int *>(tail + 8 * L::kNumBars + 8));
 }
 
 template <int D, bool BF16, int MODE>
