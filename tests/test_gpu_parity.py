@@ -339,12 +339,14 @@ def test_split_decode_with_a_dirty_workspace(idx):
     outs = []
     for _ in range(2):
         out = torch.full_like(call.q, float("nan"))
+        n0 = pa.launch_count()
         if tree:
             pa.paged_attn_decode_tree(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, tm.cuda(),
                                       call.max_ctx, w.scale, out=out, workspace=ws)
         else:
             pa.paged_attn_decode(call.q, st.key_cache, st.value_cache, call.bt, call.cu, call.ctx, call.max_ctx,
                                  w.scale, out=out, workspace=ws)
+        assert pa.launch_count() - n0 == 3  # order, attention and merge kernels
         torch.cuda.synchronize()
         assert pa.read_status(ws) == 0
         outs.append(out)
@@ -633,6 +635,29 @@ def test_block_swap_refuses_pageable_host_memory():
                                    ctypes.c_void_p(host.data_ptr()), ctypes.c_void_p(host.data_ptr()), HB, H, d, 0,
                                    ctypes.c_void_p(pairs.data_ptr()), 1, 0, None, None)
     assert rc == -1 and pa.launch_count() == n0
+
+
+def test_interleaved_calls_on_one_stream_give_each_call_its_result():
+    # Every kernel of the library is launched as a programmatic dependent of the kernel before it
+    # and waits for it before touching memory.  Calls of two workloads (block copies, cache writes,
+    # a decode with several KV splits, a chunked prefill) issued back to back on one stream with no
+    # host synchronisation in between must each give their own result.
+    wa = W.random_workload(31, B=4, q_max=3, ctx_max=3000, H_kv=2, G=4, d=128, dtype=W.BF16, kind="decode")
+    wb = W.random_workload(32, B=3, q_max=150, ctx_max=400, H_kv=2, G=4, d=128, dtype=W.BF16, kind="prefill")
+    sa, sb = DeviceStep(wa), DeviceStep(wb)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        sa.run()
+        sb.run()
+    out_a, out_b = sa.out.clone(), sb.out.clone()
+    torch.cuda.synchronize()
+    for st, w, out in ((sa, wa, out_a), (sb, wb, out_b)):
+        assert st.statuses() == [0] * (1 + len(st.calls)), st.statuses()
+        ref, _, _ = oracle_step(w, oracle.lib())
+        got = out.double().cpu().numpy()
+        assert np.isfinite(got).all()
+        err = np.abs(got - ref).max()
+        assert err <= TOL[w.dtype], f"{w.name}: max abs err {err:.3e}"
 
 
 def test_repeat_runs_identical():
