@@ -20,6 +20,8 @@ The same JSON line carries:
   prefill       causal varlen prefill (8 prompts U[256,2048], 40/40 heads, bf16):
                 TFLOP/s of exact causal pairs vs the measured bf16 peak
   legs          the GQA shared-prefix decode step, the mixed continuous-batching step, the
+                last 512-token chunk of a 32 K-token prompt (chunked prefill over a long context,
+                tensor + HBM roofline), the
                 tree-attention verify of speculative drafts (HBM roofline), the FP8 (E4M3) KV
                 cache on the 13B decode layer (HBM roofline, speed-up over 16 bits), and
                 the preemption swap of KV blocks to a pinned host pool and back (GB/s against
@@ -392,6 +394,7 @@ def run_ours(args):
         result["legs"] = {
             "gqa_shared_prefix": leg_gqa(args, stream, device, hbm_peak, rank),
             "mixed_step": leg_mixed(args, stream, device, hbm_peak, bf16_peak, rank),
+            "long_chunk_prefill": leg_long_chunk(args, stream, device, hbm_peak, bf16_peak, rank),
             "tree_verify": leg_tree(args, stream, device, hbm_peak, rank),
             "fp8_cache": leg_fp8(args, stream, device, hbm_peak, rank),
             "shared_prefix": leg_shared(args, stream, device, hbm_peak, rank),
@@ -544,6 +547,28 @@ def leg_prefill(args, stream, device, bf16_peak, peak_src, rank):
         "tokens_per_s": round(w.T / (step_ms * 1e-3), 1),
         "prefill_ms_stats": st.call_stats["paged_attn_prefill"],
     }
+
+
+LONG_CHUNK = "long-context chunked prefill: the last 512-token chunk of a 32 K-token prompt, 32/8 heads, d 128, bf16"
+
+
+def leg_long_chunk(args, stream, device, hbm_peak, bf16_peak, rank):
+    """Chunked prefill of a long prompt: its last 512-token chunk over the 32 K tokens before it
+    (LLaMA-3-8B-shaped attention: 32 query heads, 8 KV heads, d 128, bf16).  Its 64 work items
+    (8 query-tile pairs x 8 KV heads) would leave most of the 148 SMs idle, so the call takes the
+    split schedule; roofline = tensor time of its FLOP + HBM time of its K/V bytes."""
+    from paged_kv_attention_34_b200 import workloads as W
+    from paged_kv_attention_34_b200.step import attn_bytes, attn_flops
+
+    w = W.build_workload("long_chunk", q_lens=[512], ctx_lens=[32768], H_q=32, H_kv=8, d=128, dtype=W.BF16,
+                         seed=shard_seed(34_006, rank), calls=[W.AttnCall("prefill", 0, 1)])
+    st, per, step_ms = bench_leg(w, max(args.steps, 5), args.warmup, stream, device)
+    flops, nbytes = attn_flops(w), attn_bytes(w)
+    ms = per["paged_attn_prefill"]
+    t_roof = flops / (bf16_peak * 1e12) + nbytes / (hbm_peak * 1e9)
+    return {"workload": LONG_CHUNK, "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 2),
+            "frac": round(t_roof / (ms * 1e-3), 4), "flop_per_launch": flops, "kv_bytes": nbytes,
+            "avg_launch_ms": round(ms, 5), "prefill_ms_stats": st.call_stats["paged_attn_prefill"]}
 
 
 def leg_gqa(args, stream, device, hbm_peak, rank):
@@ -955,6 +980,8 @@ def run_one_leg(args):
         res = leg_fp8(args, stream, device, hbm, 0)
     elif args.only == "shared":
         res = leg_shared(args, stream, device, hbm, 0)
+    elif args.only == "long_chunk":
+        res = leg_long_chunk(args, stream, device, hbm, bf16, 0)
     else:
         res = leg_mixed(args, stream, device, hbm, bf16, 0)
     print(json.dumps({"leg": args.only, **res}), flush=True)
@@ -969,7 +996,8 @@ def main(argv=None):
     ap.add_argument("--no-legs", action="store_true", help="headline decode step only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="host time budget of the cpu_baseline sample")
-    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap", "tree", "fp8", "shared"], default=None,
+    ap.add_argument("--only", choices=["prefill", "gqa", "mixed", "swap", "tree", "fp8", "shared", "long_chunk"],
+                    default=None,
                     help="run one leg alone and print its JSON object (profiling runs)")
     ap.add_argument("--batch", type=int, default=64,
                     help="sequences of the headline decode workload (64 = the 13B-shaped layer; smaller for profiling)")

@@ -310,9 +310,15 @@ int pa_paged_attn_decode_noalloc(void *out, const void *q, const void *key_cache
 
 /*
  * pa_prefill_workspace_bytes -- device workspace of pa_paged_attn_prefill:
- * the status word area (with the work counter of the tile scheduler) and the
- * order in which the (query-tile pair, sequence) work is handed out, written
- * by the call itself (most K/V tiles first).  Pure host function.
+ * the status word area (with the work counter of the tile scheduler and the
+ * word naming the schedule the call chose), the order in which the
+ * (query-tile pair, sequence) work is handed out (most K/V tiles first), and,
+ * for calls whose longest work items outlast a balanced share of an SM (a
+ * long-context chunk among few items), the per-SM starts of the split
+ * schedule with its arrival counters and the partial outputs (fp32) and
+ * log-sum-exps of two split pieces per SM: about 2 * 160 * 2 * 128 * (d + 1)
+ * * 4 bytes (42 MB at d = 128), independent of the sizes.  All of it is
+ * written by the call itself.  Pure host function.
  */
 size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len);
 
@@ -324,7 +330,10 @@ size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len
  * a chunk with earlier context attends to that context too (chunked prefill).
  * Tiles of 128 queries x 128 keys run on the tcgen05 tensor cores with fp32
  * accumulators in tensor memory, fed by TMA from the cache blocks; the online
- * softmax of iopencloud section 2.2 runs between the two products.
+ * softmax of iopencloud section 2.2 runs between the two products.  Work
+ * items too long for a balanced share of an SM are cut along the keys into
+ * pieces on neighbouring SMs and their partial results merged by log-sum-exp
+ * (the split-KV and merge of the FlashDecoding answer, interview Q&A page).
  *   out, q        [T][H_q][d]        cu_seqlens_q [B+1] (q_b >= 1)   context_lens [B]
  *   max_q_len     host upper bound of q_b;  max_ctx host upper bound of ctx_b
  *   workspace     >= pa_prefill_workspace_bytes(...) bytes; status word reset on stream

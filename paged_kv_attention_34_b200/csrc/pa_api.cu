@@ -295,7 +295,7 @@ extern "C" size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, in
 {
     if (B < 0 || H_q < 1 || H_kv < 1 || (d != 64 && d != 128) || max_q_len < 0 || H_q % H_kv)
         return 0;
-    return prefill_workspace_bytes(B, H_q, H_kv, max_q_len);
+    return prefill_workspace_bytes(B, H_q, H_kv, d, max_q_len);
 }
 
 extern "C" int pa_paged_attn_prefill(void *out, const void *q, const void *key_cache, const void *value_cache,

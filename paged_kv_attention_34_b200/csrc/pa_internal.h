@@ -139,7 +139,7 @@ size_t shared_workspace_bytes(int64_t T, int B, int H_q, int H_kv, int d, int ma
 size_t seq_order_bytes(int B);
 int launch_seq_order(const int32_t *context_lens, int B, int32_t *order, int32_t *status, cudaStream_t stream);
 int launch_decode(const AttnArgs &a);
-size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int max_q_len);
+size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len);
 int launch_prefill(const AttnArgs &a);
 
 }  // namespace pa

@@ -32,7 +32,14 @@
 //     while the other tile's softmax runs;
 //   * warp 2 hands out work items from a global counter, heaviest first (sequences with the most
 //     pages first, and within one the later query tiles, which see more keys), loads the Q tiles
-//     and feeds the K ring; warp 3 feeds the V ring and clears the
+//     and feeds the K ring.  A call with too few items to give most SMs one (a long-context chunk:
+//     a few query tiles over many keys) runs the split instance of the kernel instead: the items
+//     are laid end to end by cost and cut into equal consecutive ranges, one per CTA
+//     (McNaughton's wrap-around rule), so an item crossing a cut runs as pieces on neighbouring
+//     CTAs, each over its own K/V tiles; a piece writes its normalised partial O and log2-sum-exp
+//     to the workspace, and the last piece of each row to finish (a per-warp arrival counter)
+//     combines them and writes the output (the split-KV and merge of the FlashDecoding answer,
+//     interview Q&A page).  Warp 3 feeds the V ring and clears the
 //     V rows past the context end in the tile that holds it (P is 0 there, but 0 * NaN is NaN);
 //     lanes 0-7 each fetch one page of a tile (one thread issuing all boxes of a tile is limited
 //     by the per-instruction issue cost of TMA).  The first warpgroup shrinks its register budget
@@ -63,6 +70,14 @@ constexpr int kItemSlots = 2;
 constexpr int kItemReaders = 11;  // warps 0, 1, 3 and 4-11 each acknowledge a work item
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr size_t kCounterOffset = 64;      // work counter inside the status area of the workspace
+constexpr size_t kPlanOffset = 128;        // split schedule: T, the cost range of a CTA
+// The split schedule: costs in K/V tiles, plus kItemCost per item for its start and end (the first
+// tiles' latency, the epilogue); at most kMaxCtas CTAs (the workspace holds two partial slots per
+// CTA) and kMaxPieces pieces per item.  A call takes it when its items would keep at most 3/4 of
+// the CTAs busy (4 items <= 3 CTAs).
+constexpr int kMaxCtas = 160;
+constexpr int kItemCost = 2;
+constexpr int kMaxPieces = 8;
 
 struct Params {
     const int32_t *block_tables;
@@ -86,6 +101,16 @@ struct Params {
     float scale_log2;
 };
 
+// The split schedule's buffers (in the workspace), a kernel argument of their own.
+struct SplitParams {
+    int *plan;       // [0] = T, the cost range of a CTA (written by the plan kernel)
+    int4 *starts;    // [kMaxCtas] CTA c's first item {b, g, pair, its start relative to c T}
+    int *merge_cnt;  // [kMaxCtas][2 tiles][4 warps] arrivals of the pieces of the item that starts in c
+    float *part_o;   // [2 kMaxCtas slots][2 tiles][D][kRows] normalised partial O (column-major)
+    float *part_lse; // [2 kMaxCtas slots][2 tiles][kRows] log2-sum-exp of the scaled scores
+    int n_ctas;      // grid size
+};
+
 // One query tile of a work item.
 struct Tile {
     bool on;      // the tile has at least one query token
@@ -103,12 +128,30 @@ struct Item {
 
 // What the scheduler hands to the other roles: the item index (-1 = no more work) and the
 // decoded item, so that no role re-reads the sequence metadata from global memory.
+// The split schedule's piece of an item, handed to the roles with it (the tile counts in the
+// item are the piece's).
+struct Split {
+    int k0;        // first K/V tile of the piece
+    int n_kv_all;  // K/V tiles of the whole item (its last one may hold the context end)
+    int c0;        // the CTA whose range the item starts in
+    int j;         // this piece (running on CTA c0 + j)
+    int ns[2];     // per query tile: pieces holding its keys (1: its output is written directly)
+    int jf[2];     // ... and the first of them
+};
+
+template <bool SPLIT>
 struct ItemSlot {
     int it;
     Item I;
 };
+template <>
+struct ItemSlot<true> {
+    int it;
+    Item I;
+    Split sp;
+};
 
-template <int D>
+template <int D, bool SPLIT>
 struct Smem {
     static constexpr int kKB = D / 64;               // 128-byte column blocks
     static constexpr int kTile = kKB * kRows * 128;  // one 128-row x D tile
@@ -118,7 +161,7 @@ struct Smem {
     static constexpr int kBars = kV + kStages * kTile;
     static constexpr int kNumBars = 2 * 2 + 4 * kStages + 4 * 2 + 2 * kItemSlots + 4;
     static constexpr int kItems = kBars + 8 * kNumBars;
-    static constexpr int kTmemSlot = kItems + ((int(sizeof(ItemSlot)) * kItemSlots + 15) / 16) * 16;
+    static constexpr int kTmemSlot = kItems + ((int(sizeof(ItemSlot<SPLIT>)) * kItemSlots + 15) / 16) * 16;
     static constexpr int kAbort = kTmemSlot + 8;
     static constexpr int kBytes = kAbort + 8;
     static constexpr int kAlloc = kBytes + 1024;
@@ -196,6 +239,235 @@ __device__ __forceinline__ bool get_item(const Params &p, int it, Item &I, bool 
     return true;
 }
 
+// ---- the split schedule ------------------------------------------------------------------------
+
+// The checks every sequence of a call must pass (PA_ERR_SEQ otherwise; its items are skipped).
+__device__ __forceinline__ bool seq_valid(const Params &p, int q0, int q1, int ctx)
+{
+    const int qb = q1 - q0;
+    return qb >= 1 && ctx >= qb && qb <= p.max_q_len && ctx <= p.max_ctx && ctx <= p.max_blocks * 16 && q1 <= p.T &&
+           q0 >= 0;
+}
+
+// Query-tile pairs of a sequence with qb new tokens.
+__device__ __forceinline__ int seq_pairs(int qb, int tok_per_tile) { return (qb + 2 * tok_per_tile - 1) / (2 * tok_per_tile); }
+
+__device__ __forceinline__ long long floor_div(long long a, long long b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+// The split schedule's plan (one CTA, the call's first kernel): clears the status word and the
+// merge counters, reports inconsistent sequences, and lays the items end to end in (sequence b,
+// KV head g, query-tile pair) order, an item costing its K/V tiles + kItemCost.  With W the cost
+// of all items and M the largest, a CTA's range is T = ceil(W / n_ctas), at least kItemCost + 1
+// (so that only the first piece of an item can be empty) and at least M / (kMaxPieces - 1) (so
+// that no item has more than kMaxPieces pieces); CTA c takes [c T, (c + 1) T), and starts[c] is
+// the item holding position c T.  The call takes this schedule only with B <= kOrderThreads.
+__global__ void __launch_bounds__(kOrderThreads) pa_prefill_split_plan_kernel(const Params p, const SplitParams sq)
+{
+    griddep_wait();  // the kernel before this call's on the stream (its writes are visible after this)
+    const int tid = threadIdx.x;
+    if (tid == 0)
+        *p.status = PA_OK;  // the call's status word: this is its first kernel
+    for (int i = tid; i < kMaxCtas * 8; i += kOrderThreads)
+        sq.merge_cnt[i] = 0;
+    __syncthreads();    // the status word is clear before any thread reports
+    griddep_release();  // the attention kernel's CTAs may be scheduled now; they wait for this grid
+    const int tpt = p.tok_per_tile;
+    __shared__ long long pre[kOrderThreads + 1];  // exclusive prefix of the sequences' costs
+    __shared__ long long red_s[kOrderThreads / 32];
+    __shared__ int red_m[kOrderThreads / 32];
+    const int lane = tid & 31, warp = tid >> 5;
+    // sequence tid: the cost of its items (all KV heads) and its largest item
+    long long c = 0;
+    int m = 0;
+    if (tid < p.B) {
+        const int q0 = __ldg(p.cu_seqlens + tid), q1 = __ldg(p.cu_seqlens + tid + 1);
+        const int ctx = __ldg(p.context_lens + tid);
+        if (!seq_valid(p, q0, q1, ctx)) {
+            set_status(p.status, PA_ERR_SEQ);
+        } else {
+            const int np = seq_pairs(q1 - q0, tpt);
+            for (int pr = 0; pr < np; ++pr) {
+                const int k = pair_kv_tiles(pr, q1 - q0, ctx, tpt) + kItemCost;
+                c += k;
+                m = max(m, k);
+            }
+            c *= p.H_kv;
+        }
+    }
+    // block-wide inclusive scan of c (warp shuffles, then the warp totals) and max of m
+    long long incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+        m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    }
+    if (lane == 31)
+        red_s[warp] = incl;
+    if (lane == 0)
+        red_m[warp] = m;
+    __syncthreads();
+    long long base = 0, W = 0;
+    int M = 0;
+    for (int i = 0; i < kOrderThreads / 32; ++i) {
+        if (i < warp)
+            base += red_s[i];
+        W += red_s[i];
+        M = max(M, red_m[i]);
+    }
+    pre[tid] = base + incl - c;
+    if (tid == 0)
+        pre[kOrderThreads] = W;
+    __syncthreads();
+    long long T = (W + sq.n_ctas - 1) / sq.n_ctas;
+    T = max(T, (long long)kItemCost + 1);
+    T = max(T, (long long)((M + kMaxPieces - 2) / (kMaxPieces - 1)));
+    if (T >= (1ll << 30)) {
+        if (tid == 0)
+            set_status(p.status, PA_ERR_TOO_LARGE);
+        T = 1ll << 30;
+    }
+    for (int cta = tid; cta < sq.n_ctas; cta += kOrderThreads) {
+        const long long pos = (long long)cta * T;
+        int4 st = make_int4(-1, 0, 0, 0);
+        if (pos < W) {
+            int lo = 0, hi = p.B;  // pre[lo] <= pos < pre[hi] (pre[B] = W)
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (pre[mid] <= pos)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            const int b = lo;
+            const int q0 = __ldg(p.cu_seqlens + b), qb = __ldg(p.cu_seqlens + b + 1) - q0;
+            const int ctx = __ldg(p.context_lens + b);
+            const long long cb = (pre[b + 1] - pre[b]) / p.H_kv;  // one KV head's items of b
+            const long long off = pos - pre[b];
+            const int g = static_cast<int>(off / cb);
+            const long long r = off - g * cb;
+            int pr = 0;
+            long long acc = 0;
+            for (;; ++pr) {
+                const long long k = pair_kv_tiles(pr, qb, ctx, tpt) + kItemCost;
+                if (acc + k > r)
+                    break;
+                acc += k;
+            }
+            st = make_int4(b, g, pr, static_cast<int>(acc - r));
+        }
+        sq.starts[cta] = st;
+    }
+    if (tid == 0)
+        sq.plan[0] = static_cast<int>(T);
+}
+
+// Item (b, g, pair) of the split schedule, with the whole item's tile counts; false when the pair
+// has no query token or the sequence is invalid (the plan kernel reports it).
+__device__ __forceinline__ bool item_of(const Params &p, int b, int g, int pair, Item &I)
+{
+    I.b = b;
+    I.g = g;
+    I.q0 = __ldg(p.cu_seqlens + b);
+    const int q1 = __ldg(p.cu_seqlens + b + 1);
+    I.qb = q1 - I.q0;
+    I.ctx = __ldg(p.context_lens + b);
+    if (!seq_valid(p, I.q0, q1, I.ctx))
+        return false;
+    make_tile(p, I, 2 * pair, I.A);
+    make_tile(p, I, 2 * pair + 1, I.Bt);
+    if (!I.A.on)
+        return false;
+    I.n_kv = max(I.A.n_kv, I.Bt.n_kv);
+    const int lim_hi = I.ctx - I.qb + (I.Bt.on ? I.Bt.t_begin + I.Bt.n_tok : I.A.t_begin + I.A.n_tok) - 1;
+    I.n_pages = lim_hi / 16 + 1;
+    return true;
+}
+
+// Where a CTA of the split schedule is in its range: the next item (b, g, pair) and its start
+// relative to the range's start.
+struct Walk {
+    int b, g, pair;
+    long long rel;
+};
+
+// The next piece of this CTA's range [0, T) (relative positions), advancing `w`; false when the
+// range is exhausted.  An item is cut where the CTA ranges cut its cost: with prel its start
+// within the range of the CTA c0 where it begins, piece i covers the K/V tiles [kc(i), kc(i + 1)),
+// kc(i) = clamp(i T - prel - kItemCost, 0, tiles) for 0 < i < n, kc(0) = 0, kc(n) = tiles, and
+// runs on CTA c0 + i.  I gets the piece's tile counts, sp the rest.
+__device__ bool walk_next(const Params &p, int T, Walk &w, Item &I, Split &sp)
+{
+    const int tpt = p.tok_per_tile;
+    while (w.b < p.B && w.rel < T) {
+        const int b = w.b, g = w.g, pair = w.pair;
+        const int q0 = __ldg(p.cu_seqlens + b), q1 = __ldg(p.cu_seqlens + b + 1), ctx = __ldg(p.context_lens + b);
+        const int np = seq_valid(p, q0, q1, ctx) ? seq_pairs(q1 - q0, tpt) : 0;
+        if (np == 0) {  // no cost in the plan
+            w.b = b + 1;
+            w.g = 0;
+            w.pair = 0;
+            continue;
+        }
+        const int t = pair_kv_tiles(pair, q1 - q0, ctx, tpt);
+        const long long start = w.rel, cost = t + kItemCost;
+        w.rel += cost;
+        if (++w.pair >= np) {
+            w.pair = 0;
+            if (++w.g >= p.H_kv) {
+                w.g = 0;
+                ++w.b;
+            }
+        }
+        const long long lo = start < 0 ? -start - kItemCost : 0;
+        const long long hi = start + cost > T ? T - start - kItemCost : t;
+        const int k0 = static_cast<int>(min(max(lo, 0ll), (long long)t));
+        const int k1 = static_cast<int>(min(max(hi, 0ll), (long long)t));
+        // nothing here but the item's start or end cost; or no query token (not for pair < np)
+        if (k0 >= k1 || !item_of(p, b, g, pair, I))
+            continue;
+        const long long sh = floor_div(start, T);
+        const long long prel = start - sh * T;  // in [0, T)
+        sp.c0 = static_cast<int>(blockIdx.x + sh);
+        sp.j = static_cast<int>(-sh);
+        sp.k0 = k0;
+        sp.n_kv_all = I.n_kv;
+        const int n = static_cast<int>((prel + cost + T - 1) / T);
+        auto kc = [&](int i) -> int {
+            if (i <= 0)
+                return 0;
+            if (i >= n)
+                return t;
+            return static_cast<int>(min(max((long long)i * T - prel - kItemCost, 0ll), (long long)t));
+        };
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            Tile &tl = x == 0 ? I.A : I.Bt;
+            int ns = 0, jf = 0;
+            if (tl.on) {
+                for (int i = 0; i < n && i < kMaxPieces; ++i) {
+                    const int a = kc(i);
+                    if (a < kc(i + 1) && a < tl.n_kv) {
+                        if (ns == 0)
+                            jf = i;
+                        ++ns;
+                    }
+                }
+                tl.n_kv = max(0, min(k1, tl.n_kv) - k0);
+                tl.on = tl.n_kv > 0;
+            }
+            sp.ns[x] = ns;
+            sp.jf[x] = jf;
+        }
+        if (!I.A.on && !I.Bt.on)
+            continue;
+        I.n_kv = k1 - k0;
+        return true;
+    }
+    return false;
+}
+
 // Bounded wait that also gives up once another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int32_t *status)
 {
@@ -222,12 +494,100 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
 __device__ __forceinline__ uint32_t full_par(int k) { return static_cast<uint32_t>(k & 1); }
 __device__ __forceinline__ uint32_t free_par(int k) { return static_cast<uint32_t>((k & 1) ^ 1); }
 
+// Epilogue of one query tile (x) of a piece of a split item, for the row of this thread: the
+// piece's normalised partial O and its log2-sum-exp go to the piece's slot -- 2 (c0 + j) + 1 for
+// the piece that begins an item in CTA c0's range (the last item of that range), 2 (c0 + j) for a
+// piece that goes on from an earlier range (the first item of its range) -- then each warp counts
+// itself in on the item's counter, and the warp whose arrival completes the count combines the
+// pieces of its 32 rows, O = sum_i 2^(lse_i - M) O_i / sum_i 2^(lse_i - M), M = max_i lse_i,
+// and writes them out.  `o_free` is arrived on once O has been read from TMEM.
 template <int D, bool BF16>
+__device__ __forceinline__ void split_epilogue(const Params &p, const SplitParams &sq, const Split &sp, int x, int sub,
+                                               int r, int lane,
+                                               uint32_t o_tmem, float inv, float m, float l, bool row_valid,
+                                               uint8_t *orow, uint64_t *o_free)
+{
+    auto slot_of = [&](int jj) { return 2 * (sp.c0 + jj) + (jj == 0 ? 1 : 0); };
+    const int own = slot_of(sp.j);
+    {
+        float *po = sq.part_o + ((int64_t)own * 2 + x) * (D * kRows) + r;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tc::ld32(o_tmem + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                __stcg(po + (c * 32 + i) * kRows, __uint_as_float(o[i]) * inv);
+        }
+    }
+    tc::fence_before_sync();
+    mbar_arrive(o_free);  // O_X has been read
+    __stcg(sq.part_lse + (own * 2 + x) * kRows + r, l > 0.f ? m + __log2f(l) : -INFINITY);
+    __threadfence();  // the partial is visible device-wide before the warp counts itself in
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0)
+        prev = atomicAdd(sq.merge_cnt + (sp.c0 * 2 + x) * 4 + sub, 1);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    const int ns = sp.ns[x];
+    if (prev != ns - 1)
+        return;
+    __threadfence();  // every other piece's partial of these rows is visible
+    float lse[kMaxPieces], M = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMaxPieces; ++i) {
+        lse[i] = i < ns ? __ldcg(sq.part_lse + (slot_of(sp.jf[x] + i) * 2 + x) * kRows + r) : -INFINITY;
+        M = fmaxf(M, lse[i]);
+    }
+    if (!row_valid || M == -INFINITY)
+        return;
+    float wgt[kMaxPieces], Z = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPieces; ++i) {
+        wgt[i] = lse[i] == -INFINITY ? 0.f : fast_exp2(lse[i] - M);
+        Z += wgt[i];
+    }
+    const float iz = 1.f / Z;  // Z >= 1: the largest term is 2^0
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+        float acc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            acc[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxPieces; ++k) {
+            if (wgt[k] == 0.f)
+                continue;
+            const float *src =
+                sq.part_o + ((int64_t)slot_of(sp.jf[x] + k) * 2 + x) * (D * kRows) + (c * 32) * kRows + r;
+            const float wk = wgt[k] * iz;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                acc[i] += wk * __ldcg(src + i * kRows);
+        }
+        uint32_t o[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+            o[i >> 1] = pack2<BF16>(acc[i], acc[i + 1]);
+        uint8_t *dst = orow + c * 64;
+        if (p.out_align32) {
+            st_global_v8(dst, o);
+            st_global_v8(dst + 32, o + 8);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<uint4 *>(dst + i * 4) = make_uint4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        }
+    }
+}
+
+// SPLIT: the split schedule (pieces of items, walked per CTA); otherwise the queue.
+template <int D, bool BF16, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     pa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                         const __grid_constant__ CUtensorMap tmap_v, const Params p)
+                         const __grid_constant__ CUtensorMap tmap_v, const Params p, const SplitParams sq)
 {
-    using L = Smem<D>;
+    using L = Smem<D, SPLIT>;
     constexpr int KB = L::kKB;
     constexpr uint32_t kTmemCols = 512;
     // TMEM columns: S_A, S_B (P written over their first 64 columns), O_A, O_B
@@ -251,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *drain = item_empty + kItemSlots;  // [1] both MMA threads' products complete
     uint64_t *v_land = drain + 1;               // [1] V tile with a context end landed (before zeroing)
     uint64_t *tok = v_land + 1;                 // [2] tok[X]: MMA thread X may issue its next batch
-    ItemSlot *item_slot = reinterpret_cast<ItemSlot *>(smem + L::kItems);
+    ItemSlot<SPLIT> *item_slot = reinterpret_cast<ItemSlot<SPLIT> *>(smem + L::kItems);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kAbort);
 
@@ -448,22 +808,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *ring = smem + (is_v ? L::kV : L::kK);
         int n_item = 0, n_tiles = 0, q_n[2] = {0, 0}, z_n = 0;
         bool ok = true;
+        // split schedule: the scheduler walks this CTA's range from its first item
+        Walk walk{p.B, 0, 0, 0};
+        int split_T = 0;
+        if constexpr (SPLIT) {
+            if (!is_v) {
+                split_T = sq.plan[0];
+                const int4 s0 = sq.starts[blockIdx.x];
+                if (s0.x >= 0)
+                    walk = Walk{s0.x, s0.y, s0.z, s0.w};
+            }
+        }
         for (;;) {
             int it = -1;
             Item I;
+            Split sp;
             if (!is_v) {
-                // next work item that has query tokens (lane 0 draws, the warp follows)
-                for (;;) {
-                    // lane 0 decides for the whole warp (the abort flag may change between lanes' reads)
-                    int cand = -1;
-                    if (lane == 0 && ok && !*abort_flag)
-                        cand = atomicAdd(p.counter, 1);
-                    cand = __shfl_sync(0xffffffffu, cand, 0);
-                    if (cand < 0 || cand >= p.n_items)
-                        break;
-                    if (get_item(p, cand, I, lane == 0)) {
-                        it = cand;
-                        break;
+                if constexpr (SPLIT) {
+                    // the next piece of this CTA's range (every lane walks the same state; lane 0
+                    // decides whether to go on, the abort flag may change between lanes' reads)
+                    int go = 0;
+                    if (lane == 0)
+                        go = ok && !*abort_flag;
+                    go = __shfl_sync(0xffffffffu, go, 0);
+                    if (go && walk_next(p, split_T, walk, I, sp))
+                        it = 0;
+                } else {
+                    // next work item that has query tokens (lane 0 draws, the warp follows)
+                    for (;;) {
+                        // lane 0 decides for the whole warp (the abort flag may change between lanes' reads)
+                        int cand = -1;
+                        if (lane == 0 && ok && !*abort_flag)
+                            cand = atomicAdd(p.counter, 1);
+                        cand = __shfl_sync(0xffffffffu, cand, 0);
+                        if (cand < 0 || cand >= p.n_items)
+                            break;
+                        if (get_item(p, cand, I, lane == 0)) {
+                            it = cand;
+                            break;
+                        }
                     }
                 }
                 // publish it (or the end marker -1) to the other roles
@@ -473,6 +856,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = ok && got;
                     item_slot[slot].it = ok ? it : -1;
                     item_slot[slot].I = I;
+                    if constexpr (SPLIT)
+                        item_slot[slot].sp = sp;
                     mbar_arrive(&item_full[slot]);
                 }
                 ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -483,8 +868,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wait_bar(&item_full[slot], full_par(n_item / kItemSlots), abort_flag, p.status);
                 ok = __all_sync(0xffffffffu, ok);
                 it = ok ? item_slot[slot].it : -1;
-                if (it >= 0)
+                if (it >= 0) {
                     I = item_slot[slot].I;
+                    if constexpr (SPLIT)
+                        sp = item_slot[slot].sp;
+                }
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&item_empty[slot]);
@@ -492,6 +880,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++n_item;
             if (it < 0)
                 break;
+            // K/V tile j of the item is tile k_first + j of its whole causal range (a piece of a split
+            // item starts later), and n_kv_all the whole range's tiles
+            int k_first = 0, n_kv_all = I.n_kv;
+            if constexpr (SPLIT) {
+                k_first = sp.k0;
+                n_kv_all = sp.n_kv_all;
+            }
             const int32_t *table = p.block_tables + (int64_t)I.b * p.max_blocks;
             // TMA row of page `pidx` of the item (lanes 0-7); pages past the item's range, and bad
             // block ids, read rows past the pool, which TMA fills with zeros
@@ -509,16 +904,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // The last page of the context may be partly filled: its V rows past the context end can
             // hold anything (NaN included) and P is 0 there, but 0 * NaN is NaN, so the V warp clears
             // them before the tile is handed on.  That happens only when this item reads up to the
-            // context end.
+            // context end, in the last tile of its whole range.
             const int last_page = (I.ctx + 15) / 16 - 1;
-            const int zpg = last_page - 8 * (I.n_kv - 1);  // page of the last tile holding the context end
-            const int zr0 = I.ctx & 15;                   // first row to clear
+            const int zpg = last_page - 8 * (n_kv_all - 1);  // page of the last tile holding the context end
+            const int zr0 = I.ctx & 15;                     // first row to clear
             const bool zero_tail = is_v && zr0 != 0 && I.n_pages == last_page + 1 && zpg >= 0 && zpg < 8;
-            int y = page_row(lane);
+            int y = page_row(k_first * 8 + lane);
             for (int j = 0; j < I.n_kv; ++j) {
-                const int y_next = j + 1 < I.n_kv ? page_row((j + 1) * 8 + lane) : p.oob_row;  // in flight meanwhile
+                const int y_next = j + 1 < I.n_kv ? page_row((k_first + j + 1) * 8 + lane) : p.oob_row;  // in flight meanwhile
                 const int st = n_tiles % kStages;
-                const bool z = zero_tail && j == I.n_kv - 1;
+                const bool z = zero_tail && k_first + j == n_kv_all - 1;
                 uint64_t *done = z ? v_land : &full[st];
                 if (lane == 0) {
                     ok = wait_bar(&empty[st], free_par(n_tiles / kStages), abort_flag, p.status);
@@ -615,14 +1010,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             const int it = ok ? item_slot[slot].it : -1;
             Item I;
-            if (it >= 0)
+            Split sp;
+            if (it >= 0) {
                 I = item_slot[slot].I;
+                if constexpr (SPLIT)
+                    sp = item_slot[slot].sp;
+            }
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&item_empty[slot]);
             ++n_item;
             if (it < 0)
                 break;
+            int k_first = 0;  // first K/V tile of a piece of a split item
+            if constexpr (SPLIT)
+                k_first = sp.k0;
             const Tile &t = x == 0 ? I.A : I.Bt;
             if (!t.on)
                 continue;
@@ -641,7 +1043,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++s_n;
                 tc::fence_after_sync();
                 // the whole S row in one TMEM load; masked keys (causal / context end) become -inf
-                const int key0 = j * kKeys;
+                const int key0 = (k_first + j) * kKeys;
                 uint32_t raw[kKeys];
                 tc::ld128(s_tmem, raw);
                 if (key0 + kKeys - 1 > lim) {
@@ -720,6 +1122,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++o_n;
             tc::fence_after_sync();
             const float inv = l > 0.f ? 1.f / l : 0.f;
+            if constexpr (SPLIT) {
+                if (sp.ns[x] > 1) {
+                    split_epilogue<D, BF16>(p, sq, sp, x, sub, r, lane, o_tmem, inv, m, l, row_valid, orow,
+                                            &o_free[x]);
+                    continue;
+                }
+            }
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -753,22 +1162,76 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- host ---------------------------------------------------------------------------------------
 
+// The split schedule is taken when the call's items would keep at most 3/4 of the CTAs busy.
+static bool use_split(int64_t items, int n_ctas, int B) { return B <= kOrderThreads && 4 * items <= 3 * (int64_t)n_ctas; }
+
+// Workspace of a call: the status area (status word, work counter, split plan word), the queue
+// order, and for the split schedule the CTAs' starts, the merge counters and two partial slots
+// (O and log2-sum-exp of both query tiles) per CTA.
+struct WsLayout {
+    size_t order, starts, merge_cnt, part_lse, part_o, bytes;
+};
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+static WsLayout ws_layout(int B, int64_t n_pairs, int D, bool split)
+{
+    WsLayout w;
+    w.order = PA_STATUS_BYTES;
+    w.starts = w.order + align256(static_cast<size_t>(n_pairs) * B * sizeof(int32_t));
+    w.merge_cnt = w.starts + (split ? align256(kMaxCtas * sizeof(int4)) : 0);
+    w.part_lse = w.merge_cnt + (split ? align256(kMaxCtas * 8 * sizeof(int)) : 0);
+    w.part_o = w.part_lse + (split ? align256(static_cast<size_t>(2 * kMaxCtas) * 2 * kRows * sizeof(float)) : 0);
+    w.bytes = w.part_o + (split ? static_cast<size_t>(2 * kMaxCtas) * 2 * D * kRows * sizeof(float) : 0);
+    return w;
+}
+
+// Launch one instance of the attention kernel (per device, once: the check of the register count
+// the warpgroups' register split relies on, and the shared-memory attribute).
+template <int D, bool BF16, bool SPLIT>
+static int launch_attention(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const Params &p,
+                            const SplitParams &sq, int grid, cudaStream_t stream)
+{
+    using L = Smem<D, SPLIT>;
+    auto kern = pa_prefill_tc_kernel<D, BF16, SPLIT>;
+    static uint64_t configured = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return PA_ERR_CUDA;
+    const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+    if (!bit || !(configured & bit)) {
+        // the per-warpgroup register split assumes exactly kLaunchRegs registers per thread at
+        // launch; with any other count the growing warpgroups could wait forever, so refuse
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+            return PA_ERR_CUDA;
+        if (fa.numRegs != kLaunchRegs)
+            return PA_ERR_UNSUPPORTED;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured |= bit;
+    }
+    const cudaError_t e = launch_dependent(kern, dim3(grid), dim3(kThreads), L::kAlloc, stream, tq, tk, tv, p, sq);
+    count_launch();
+    const cudaError_t e2 = cudaGetLastError();
+    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 template <int D, bool BF16>
 static int run(const AttnArgs &a)
 {
-    using L = Smem<D>;
     const int G = a.H_q / a.H_kv;
     if (G > kRows)
         return PA_ERR_UNSUPPORTED;
     Params p{};
+    SplitParams sq{};
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
     p.block_tables = a.block_tables;
     p.cu_seqlens = a.cu_seqlens_q;
     p.context_lens = a.context_lens;
     p.out = a.out;
-    p.status = static_cast<int32_t *>(a.workspace);
-    p.counter = reinterpret_cast<int *>(static_cast<uint8_t *>(a.workspace) + kCounterOffset);
-    int32_t *order = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(a.workspace) + PA_STATUS_BYTES);
-    p.order = order;
+    p.status = reinterpret_cast<int32_t *>(ws);
+    p.counter = reinterpret_cast<int *>(ws + kCounterOffset);
     p.num_blocks = a.num_blocks;
     p.T = a.T;
     p.max_blocks = a.max_blocks;
@@ -789,6 +1252,11 @@ static int run(const AttnArgs &a)
     p.oob_row = static_cast<int>(a.num_blocks * a.H_kv * 16);
     p.out_align32 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     p.scale_log2 = a.scale * 1.4426950408889634f;
+    const int n_ctas = std::min(sm_count(), kMaxCtas);
+    const bool split = use_split(items, n_ctas, a.B);
+    const WsLayout wl = ws_layout(a.B, p.n_pairs_max, D, split);
+    int32_t *order = reinterpret_cast<int32_t *>(ws + wl.order);
+    p.order = order;
 
     CUtensorMap tq, tk, tv;
     int rc = make_q_tmap(&tq, a.q, a.T, a.H_q, D, G, p.tok_per_tile, a.dtype);
@@ -798,47 +1266,42 @@ static int run(const AttnArgs &a)
         rc = make_cache_tmap(&tv, a.value_cache, a.num_blocks, a.H_kv, D, a.dtype);
     if (rc != PA_OK)
         return rc;
+    if (split) {
+        // every CTA walks its share of the items laid end to end (one CTA per SM, also when that
+        // is more CTAs than items: the items are cut to give every CTA a share)
+        sq.plan = reinterpret_cast<int *>(ws + kPlanOffset);
+        sq.starts = reinterpret_cast<int4 *>(ws + wl.starts);
+        sq.merge_cnt = reinterpret_cast<int *>(ws + wl.merge_cnt);
+        sq.part_lse = reinterpret_cast<float *>(ws + wl.part_lse);
+        sq.part_o = reinterpret_cast<float *>(ws + wl.part_o);
+        sq.n_ctas = n_ctas;
+        const cudaError_t eo =
+            launch_dependent(pa_prefill_split_plan_kernel, dim3(1), dim3(kOrderThreads), 0, a.stream, p, sq);
+        count_launch();
+        if (eo != cudaSuccess || cudaGetLastError() != cudaSuccess)
+            return PA_ERR_CUDA;
+        return launch_attention<D, BF16, true>(tq, tk, tv, p, sq, n_ctas, a.stream);
+    }
     const cudaError_t eo = launch_dependent(pa_prefill_order_kernel, dim3(1), dim3(kOrderThreads), 0, a.stream,
                                             a.cu_seqlens_q, a.context_lens, a.B, p.n_pairs_max, p.tok_per_tile, order,
                                             p.counter, p.status);
     count_launch();
     if (eo != cudaSuccess || cudaGetLastError() != cudaSuccess)
         return PA_ERR_CUDA;
-
-    auto kern = pa_prefill_tc_kernel<D, BF16>;
-    static uint64_t configured = 0;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return PA_ERR_CUDA;
-    const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
-    if (!bit || !(configured & bit)) {
-        // the per-warpgroup register split assumes exactly kLaunchRegs registers per thread at
-        // launch; with any other count the growing warpgroups could wait forever, so refuse
-        cudaFuncAttributes fa;
-        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
-            return PA_ERR_CUDA;
-        if (fa.numRegs != kLaunchRegs)
-            return PA_ERR_UNSUPPORTED;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
-            return PA_ERR_CUDA;
-        configured |= bit;
-    }
     const int grid = static_cast<int>(std::min<int64_t>(items, sm_count()));
-    const cudaError_t e = launch_dependent(kern, dim3(grid), dim3(kThreads), L::kAlloc, a.stream, tq, tk, tv, p);
-    count_launch();
-    const cudaError_t e2 = cudaGetLastError();
-    return e == cudaSuccess && e2 == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_attention<D, BF16, false>(tq, tk, tv, p, sq, grid, a.stream);
 }
 
 }  // namespace tcp
 
-// Workspace: the status area (status word, work counter), then the (pair, sequence) order.
-size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int max_q_len)
+// Workspace: see ws_layout (the split schedule's areas only for calls that take it).
+size_t prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len)
 {
     const int G = H_q / H_kv;
     const int tok = G >= 1 && G <= tcp::kRows ? tcp::kRows / G : 1;
     const int64_t n_pairs = ((int64_t)(max_q_len + tok - 1) / tok + 1) / 2;
-    return PA_STATUS_BYTES + (static_cast<size_t>(n_pairs) * B * sizeof(int32_t) + 255) / 256 * 256;
+    const int n_ctas = std::min(sm_count(), tcp::kMaxCtas);
+    return tcp::ws_layout(B, n_pairs, d, tcp::use_split(n_pairs * B * H_kv, n_ctas, B)).bytes;
 }
 
 int launch_prefill(const AttnArgs &a)

@@ -18,6 +18,7 @@ import torch
 
 import oracle
 import paged_kv_attention_34_b200 as pa
+import prefill_schedule_model as S
 from oracle_pins import oracle_step
 from paged_kv_attention_34_b200 import workloads as W
 from paged_kv_attention_34_b200.step import DeviceStep
@@ -128,6 +129,81 @@ def test_prefill_fresh_prompts_exact_lengths():
     w = W.build_workload("fresh", q_lens=L, ctx_lens=L, H_q=4, H_kv=2, d=128, dtype=W.BF16, seed=9,
                          calls=[W.AttnCall("prefill", 0, len(L))], pool_extra=5)
     run_and_compare(w)
+
+
+# Prefill calls with too few items to keep 3/4 of the SMs busy take the split schedule: items cut
+# into pieces on neighbouring CTAs, the pieces' partials merged by the last one to finish.
+# (name, q_lens, ctx_lens, H_kv, G, d, dtype)
+SPLIT_PREFILL_CASES = [
+    ("long_ctx_chunk", [512], [16384 + 37], 2, 4, 128, W.BF16),
+    ("few_items", [512, 100], [4000, 2500], 2, 4, 128, W.BF16),
+    ("g5_rows125_d64", [300], [9000], 1, 5, 64, W.F16),  # 125 rows per tile: three rows unused
+    ("g1_two_tiles_ragged", [200, 3], [20000, 7000], 1, 1, 128, W.F16),
+]
+
+
+def _split_workload(case, seed):
+    name, q, c, H_kv, G, d, dt = case
+    return W.build_workload(name, q_lens=q, ctx_lens=c, H_q=H_kv * G, H_kv=H_kv, d=d, dtype=dt, seed=seed,
+                            calls=[W.AttnCall("prefill", 0, len(q))], pool_extra=3)
+
+
+def _n_ctas():
+    return min(torch.cuda.get_device_properties(0).multi_processor_count, S.MAX_CTAS)
+
+
+def _prefill_plan(call, w):
+    """(T, starts, n_ctas) of the split schedule the prefill call wrote into its workspace."""
+    ws = call.ws.cpu()
+    T = ws[128:132].view(torch.int32).item()
+    tok = 128 // (w.H_q // w.H_kv)
+    n_pairs = ((call.max_q_len + tok - 1) // tok + 1) // 2
+    off = pa.PA_STATUS_BYTES + (n_pairs * (call.seq_hi - call.seq_lo) * 4 + 255) // 256 * 256
+    n_ctas = _n_ctas()
+    starts = [tuple(x) for x in ws[off:off + 16 * n_ctas].view(torch.int32).view(-1, 4).tolist()]
+    return T, starts, n_ctas
+
+
+@pytest.mark.parametrize("idx", range(len(SPLIT_PREFILL_CASES)), ids=lambda i: SPLIT_PREFILL_CASES[i][0])
+def test_prefill_split_items(idx):
+    case = SPLIT_PREFILL_CASES[idx]
+    w = _split_workload(case, 300 + idx)
+    st = DeviceStep(w)
+    call = st.calls[0]
+    # the call takes the split schedule, and its plan is the host model's
+    q, c = list(w.q_lens), list(w.ctx_lens)
+    st.run()
+    torch.cuda.synchronize()
+    T, starts, n_ctas = _prefill_plan(call, w)
+    model = S.plan(q, c, w.H_kv, w.H_q // w.H_kv, n_ctas)
+    assert model.mode == S.MODE_WRAP
+    assert (T, starts) == (model.T, model.starts)
+    rows = sample_rows(w, 1024) if w.T * w.H_q * max(c) > 3e7 else None
+    run_and_compare(w, rows=rows)
+
+
+
+def test_split_prefill_with_a_dirty_workspace():
+    # the merge counters and partials come from the call itself: a workspace full of garbage
+    # gives the same bytes as a clean one, call after call
+    w = _split_workload(SPLIT_PREFILL_CASES[1], 41)
+    st = DeviceStep(w)
+    st.copy_blocks()
+    st.write()
+    call = st.calls[0]
+    call.ws.fill_(0x5A)
+    call.out.fill_(float("nan"))
+    n0 = pa.launch_count()
+    st.attend(call)
+    o1 = call.out.clone()
+    st.attend(call)
+    torch.cuda.synchronize()
+    assert pa.launch_count() - n0 == 4  # plan + attention kernel per call
+    assert pa.read_status(call.ws) == 0
+    assert torch.equal(o1.view(torch.int16), call.out.view(torch.int16))
+    ref, _, _ = oracle_step(w, oracle.lib())
+    got = call.out.double().cpu().numpy().reshape(-1, w.d)
+    assert np.abs(got - ref.reshape(-1, w.d)).max() <= TOL[w.dtype]
 
 
 # ---- FP8 (E4M3) KV cache ---------------------------------------------------------------------
@@ -689,12 +765,14 @@ def test_decode_schedules_longest_sequences_first():
 
 
 def test_prefill_schedules_heaviest_work_first():
-    # prefill writes the (query-tile pair, sequence) entries by non-increasing K/V tiles
-    w = W.config5()
+    # short prompts take the queue schedule: the (query-tile pair, sequence) entries by
+    # non-increasing K/V tiles
+    w = W.config3()
     st = DeviceStep(w)
     st.run()
     torch.cuda.synchronize()
     call = next(c for c in st.calls if c.kind == "prefill")
+    assert not S.takes_split(w.B, call.max_q_len, w.H_kv, w.H_q // w.H_kv, _n_ctas())
     q = (call.cu[1:] - call.cu[:-1]).cpu().numpy()
     ctx = call.ctx.cpu().numpy()
     B = q.shape[0]
