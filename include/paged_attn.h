@@ -310,15 +310,16 @@ int pa_paged_attn_decode_noalloc(void *out, const void *q, const void *key_cache
 
 /*
  * pa_prefill_workspace_bytes -- device workspace of pa_paged_attn_prefill:
- * the status word area (with the work counter of the tile scheduler and the
- * word naming the schedule the call chose), the order in which the
- * (query-tile pair, sequence) work is handed out (most K/V tiles first), and,
- * for calls whose longest work items outlast a balanced share of an SM (a
- * long-context chunk among few items), the per-SM starts of the split
- * schedule with its arrival counters and the partial outputs (fp32) and
- * log-sum-exps of two split pieces per SM: about 2 * 160 * 2 * 128 * (d + 1)
- * * 4 bytes (42 MB at d = 128), independent of the sizes.  All of it is
- * written by the call itself.  Pure host function.
+ * the status word area (with the work counter of the tile scheduler), the
+ * order in which the (query-tile pair, sequence) work is handed out (most K/V
+ * tiles first), and, for calls whose work items would keep at most 3/4 of the
+ * SMs busy (n_pairs * B * H_kv <= 3/4 of min(SMs, 160), n_pairs =
+ * ceil(ceil(max_q_len / (128 / G)) / 2); a long-context chunk among few
+ * items), the split schedule's per-SM starts and arrival counters and the
+ * partial outputs (fp32) and log-sum-exps of two pieces per SM:
+ * 2 * 160 * 2 * 128 * (d + 1) * 4 bytes more (42 MB at d = 128).  All of it
+ * is written by the call itself.  Host function (reads the SM count of the
+ * current device once).
  */
 size_t pa_prefill_workspace_bytes(int B, int H_q, int H_kv, int d, int max_q_len);
 
