@@ -211,6 +211,18 @@ def test_workspace_queries(L):
     assert pa.decode_workspace_bytes(16, 16, 64, 8, 128, 65536) >= big
     assert L.pa_decode_workspace_bytes(1, 1, 6, 4, 128, 10) == 0  # invalid GQA ratio
     assert pa.prefill_workspace_bytes(8, 40, 40, 128, 2048) >= pa.PA_STATUS_BYTES
+    # prefill: the split schedule's areas (starts, counters, two fp32 partial slots per CTA for
+    # both query tiles) only for calls whose items would keep at most 3/4 of the CTAs busy (the
+    # SM count falls back to the B200's 148 without a device: 3/4 of 148 = 111 items)
+    queue = pa.prefill_workspace_bytes(8, 40, 40, 128, 2048)  # 8 x 8 pairs x 40 heads = 2560 items
+    assert queue == pa.PA_STATUS_BYTES + 256  # the order of 64 entries
+    split = pa.prefill_workspace_bytes(1, 32, 8, 128, 512)  # 8 pairs x 8 heads = 64 items
+    assert split >= 2 * 160 * 2 * 128 * (128 + 1) * 4
+    assert pa.prefill_workspace_bytes(1, 32, 8, 64, 512) < split  # d 64: half the partials
+    # 111 items take the split schedule, 112 the queue (G 1: 128 tokens per tile, 256 per pair)
+    assert pa.prefill_workspace_bytes(111, 1, 1, 128, 256) >= 2 * 160 * 2 * 128 * 129 * 4
+    assert pa.prefill_workspace_bytes(112, 1, 1, 128, 256) == pa.PA_STATUS_BYTES + 512
+    assert pa.prefill_workspace_bytes(14, 8, 8, 128, 256) == pa.PA_STATUS_BYTES + 256  # 112 items
     # shared-prefix decode: status, order and per-sequence prefix areas, then every row's partials
     sh = pa.shared_prefix_workspace_bytes(64, 64, 40, 40, 128, 4608, 4, 256, 16)
     assert sh >= pa.PA_STATUS_BYTES + 2 * 256 + 64 * 40 * 129 * 4
