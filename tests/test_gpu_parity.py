@@ -206,6 +206,26 @@ def test_split_prefill_with_a_dirty_workspace():
     assert np.abs(got - ref.reshape(-1, w.d)).max() <= TOL[w.dtype]
 
 
+def test_split_prefill_reports_an_inconsistent_sequence():
+    # under the split schedule the plan kernel checks the sequences: one whose context is shorter
+    # than its new tokens is reported (PA_ERR_SEQ) and left out of the plan, and the other
+    # sequence's rows are still right
+    w = _split_workload(("bad_seq", [300, 200], [5000, 4000], 2, 4, 128, W.BF16), 57)
+    assert S.takes_split(w.B, max(w.q_lens), w.H_kv, w.H_q // w.H_kv, _n_ctas())
+    st = DeviceStep(w)
+    st.copy_blocks()
+    st.write()
+    call = st.calls[0]
+    call.ctx[1] = 100  # < q_len 200
+    st.attend(call)
+    torch.cuda.synchronize()
+    assert pa.read_status(call.ws) == -8  # PA_ERR_SEQ
+    rows = np.arange(300 * w.H_q, dtype=np.int64)  # every row of sequence 0
+    ref, _, _ = oracle_step(w, oracle.lib(), rows=rows)
+    got = call.out.double().cpu().numpy().reshape(-1, w.d)[rows]
+    assert np.abs(got - ref).max() <= TOL[w.dtype]
+
+
 # ---- FP8 (E4M3) KV cache ---------------------------------------------------------------------
 
 def _fp8_device_cache(w):
