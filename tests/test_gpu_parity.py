@@ -123,6 +123,25 @@ def test_prefill_small(idx):
     run_and_compare(w)
 
 
+# The same kinds of small prefill calls with enough items (> 3/4 of the SMs) to stay on the queue
+# schedule: the cases above all have few items and take the split one.
+QUEUE_PREFILL_CASES = [
+    (8, 200, 300, 16, 1, 128, W.BF16),
+    (8, 130, 260, 8, 4, 128, W.BF16),  # chunks with earlier context, GQA
+    (8, 90, 90, 16, 1, 64, W.F16),
+    (16, 17, 40, 8, 8, 128, W.F16),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(QUEUE_PREFILL_CASES)), ids=lambda i: _case_id(QUEUE_PREFILL_CASES[i]))
+def test_prefill_small_queue_schedule(idx):
+    B, q_max, ctx_max, H_kv, G, d, dt = QUEUE_PREFILL_CASES[idx]
+    w = W.random_workload(177 + 31 * idx, B=B, q_max=q_max, ctx_max=ctx_max, H_kv=H_kv, G=G, d=d, dtype=dt,
+                          kind="prefill")
+    assert not S.takes_split(w.B, max(w.q_lens), w.H_kv, G, _n_ctas())
+    run_and_compare(w)
+
+
 def test_prefill_fresh_prompts_exact_lengths():
     # prompts of 1, 15, 16, 17, 127, 128, 129 tokens with no earlier context
     L = [1, 15, 16, 17, 127, 128, 129]
