@@ -106,3 +106,17 @@ def test_few_items_split_across_ctas():
     assert p.mode == S.MODE_WRAP
     n = sum(len(S.walk(p, [512], [4000], 2, 4, c)) for c in range(148))
     assert n > 16 * 4  # more pieces than items
+
+
+def test_piece_cap_sets_the_range_for_very_long_items():
+    # two items of ~1560 K/V tiles on 148 CTAs: the balanced share (~22) would cut each into ~70
+    # pieces; T is raised to M / 7 so that no item has more than 8, and CTAs past the work get none
+    q, c = [512], [200000]
+    p = _check_wrap(q, c, 1, 4, 148)
+    assert p.T == -(-p.M // (S.MAX_PIECES - 1)) > -(-p.W // 148)
+    per_item = {}
+    for cta in range(148):
+        for pc in S.walk(p, q, c, 1, 4, cta):
+            per_item.setdefault((pc.b, pc.g, pc.pair), []).append(pc)
+    assert all(len(v) <= S.MAX_PIECES for v in per_item.values())
+    assert p.starts[147][0] == -1  # positions past W: no work
